@@ -1,0 +1,81 @@
+"""Pins for cache assembly: window/tile split of the five workloads, the
+flush schedule of the 64-step append run, prefill-vs-append equivalence and
+the short-context edge cases."""
+
+import numpy as np
+import pytest
+
+from oracle import cache as ca
+from oracle import quantize as qz
+
+
+@pytest.mark.parametrize(
+    "T,S,R,expect",
+    [
+        (512, 4, 32, (4, 448, 60)),  # tiny
+        (4096, 4, 128, (4, 3936, 156)),  # llama3_8b
+        (8192, 4, 128, (4, 8032, 156)),  # qwen3_8b
+        (131072, 4, 128, (4, 130912, 156)),  # long_128k
+        (32768, 4, 128, (4, 32608, 156)),  # mistral_7b_b64
+        (3, 4, 32, (3, 0, 0)),
+        (20, 4, 32, (4, 0, 16)),
+        (36, 4, 32, (4, 0, 32)),
+        (67, 4, 32, (4, 0, 63)),
+        (68, 4, 32, (4, 32, 32)),
+        (0, 4, 32, (0, 0, 0)),
+        (40, 0, 0, (0, 32, 8)),
+    ],
+)
+def test_split_lengths(T, S, R, expect):
+    assert ca.split_lengths(T, S, R) == expect
+    s, tq, r = expect
+    if T >= S + R:
+        assert R <= r < R + 32
+
+
+def test_flush_schedule_of_append_run():
+    # 4096-token prefill, S=4, R=128: r = 156 -> flushes when r reaches 160, i.e.
+    # at appended steps 4 and 36 (1-based) of a 64-step run.
+    st = ca.StreamCache(64, 2, 2, 4, 128)
+    rng = np.random.default_rng(0)
+    k = rng.normal(size=(4096, 64)).astype(np.float32)
+    st.T = 4096
+    st.recent = [(p, k[0], k[0]) for p in range(4096 - 156, 4096)]
+    st.sink_k = [k[0]] * 4
+    st.sink_v = [k[0]] * 4
+    flushed = [step for step in range(1, 65) if st.append(k[1], k[1])]
+    assert flushed == [4, 36]
+
+
+@pytest.mark.parametrize("T0,T1,S,R", [(100, 230, 4, 32), (36, 99, 4, 32), (0, 80, 4, 32), (2, 70, 4, 0), (40, 200, 0, 16)])
+def test_prefill_then_append_equals_prefill(T0, T1, S, R):
+    rng = np.random.default_rng(T0 + T1)
+    d = 64
+    k = qz.bf16_bits_to_f32(rng.integers(0x3C00, 0x4100, size=(T1, d), dtype=np.uint16) ^ rng.integers(0, 2, size=(T1, d), dtype=np.uint16) << 15)
+    v = qz.bf16_bits_to_f32(rng.integers(0x3C00, 0x4100, size=(T1, d), dtype=np.uint16))
+    a = ca.StreamCache(d, 3, 2, S, R)
+    a.prefill(k[:T0], v[:T0])
+    for t in range(T0, T1):
+        a.append(k[t], v[t])
+    b = ca.StreamCache(d, 3, 2, S, R)
+    b.prefill(k, v)
+    assert a.T == b.T == T1 and a.n_tiles == b.n_tiles
+    for i in range(a.n_tiles):
+        assert np.array_equal(a.record(i), b.record(i))
+    assert a.window_rows().keys() == b.window_rows().keys()
+    for key, val in a.window_rows().items():
+        assert np.array_equal(val, b.window_rows()[key])
+    ka, va = a.dequantized()
+    assert ka.shape == (T1, d)
+    # sink and recent tokens are returned unchanged
+    s, tq, r = ca.split_lengths(T1, S, R)
+    assert np.array_equal(ka[:s], k[:s]) and np.array_equal(ka[s + tq :], k[s + tq :])
+    assert np.array_equal(va[:s], v[:s]) and np.array_equal(va[s + tq :], v[s + tq :])
+
+
+def test_ring_slots_never_collide_with_live_tokens():
+    S, R = 4, 32
+    for T in range(S, 400):
+        s, tq, r = ca.split_lengths(T, S, R)
+        slots = [ca.ring_slot(p, S, R) for p in range(S + tq, T)]
+        assert len(set(slots)) == len(slots)
