@@ -1,0 +1,450 @@
+"""Benchmark: quantized-KV decode attention on the long-context workload.
+
+One *step* = one serving decode step of the hot path on one request's cache:
+rq_append_token (bf16 ring write; every 32nd step also quantizes and packs
+a tile) followed by rq_decode_attention (split-K over the packed tiles plus
+the bf16 window, fused combine).  The per-head bit allocation (host) and the
+bulk prefill quantize run before the timed loop and are reported separately
+(alloc_ms, quantize_gbs).
+
+Workload: long_128k -- batch 1, 32 query / 8 kv heads, head_dim 128, 131072
+tokens, K outlier channels lognormal(1.5), 2-bit average over {2,3,4}.  Four
+independent caches (405 MB of packed data) are decoded round-robin so that a
+step never finds its cache in the 126 MB L2.
+
+value = algorithmic bytes of the K steps / device time of the K steps (GB/s),
+summed over ranks and divided by the slowest rank's time.  Algorithmic bytes
+per decode: packed codes + scale/zero of every tile, bf16 sink + recent
+window, q and the fp32 output; per append: the new bf16 K/V rows (and the
+flushed tile: 32 bf16 rows read, one record written).
+
+--impl reference runs the CPU oracle (numpy, fp64 attention) on a bounded
+sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "quantized-KV decode attention: effective HBM GB/s & µs/step; quantize GB/s"
+WORKLOAD = "long_128k"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------- byte counts
+def decode_bytes(wl, k_bits, v_bits, T):
+    """Algorithmic bytes of one decode over a cache of T tokens (all streams)."""
+    from oracle.cache import split_lengths  # pure arithmetic on lengths
+    from oracle.quantize import record_bytes
+
+    s, tq, r = split_lengths(T, wl.n_sink, wl.n_recent)
+    n_tiles = tq // 32
+    D, G = wl.head_dim, wl.group
+    total = 0
+    for l in range(wl.n_layers):
+        for h in range(wl.n_kv_heads):
+            per_stream = n_tiles * record_bytes(int(k_bits[l, h]), int(v_bits[l, h]), D)
+            per_stream += (s + r) * D * 2 * 2 + G * D * 2 + G * D * 4
+            total += per_stream * wl.batch
+    return total
+
+
+def append_bytes(wl, k_bits, v_bits, T_old):
+    from oracle.cache import split_lengths
+    from oracle.quantize import record_bytes
+
+    D = wl.head_dim
+    s, tq, r = split_lengths(T_old, wl.n_sink, wl.n_recent)
+    flush = T_old >= wl.n_sink and r + 1 == wl.n_recent + 32
+    total = 0
+    for l in range(wl.n_layers):
+        for h in range(wl.n_kv_heads):
+            b = 2 * D * 2 * 2  # read new rows, write them to the ring
+            if flush:
+                b += 32 * D * 2 * 2 + record_bytes(int(k_bits[l, h]), int(v_bits[l, h]), D)
+            total += b * wl.batch
+    return total
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"rq_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, _, flags in rows:
+            for n, fl in zip(names, flags):
+                if fl.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- oracle arm
+def oracle_sample(wl, seconds=12.0):
+    """Time the CPU oracle on a bounded sample: one kv-head stream of the
+    workload (its full context), one decode step.  Returns a dict."""
+    import torch
+
+    from oracle import attention as at
+    from oracle import cache as ca
+    from oracle import quantize as qz
+    from quantized_decode_attention_head_b200 import workloads
+
+    try:
+        from threadpoolctl import threadpool_info, threadpool_limits
+
+        threadpool_limits(os.cpu_count())
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    one = wl.with_(n_layers=1, batch=1, n_kv_heads=1, n_q_heads=wl.group)
+    k, v, f = workloads.kv_inputs(one, "cpu")
+    q, _, _ = workloads.step_inputs(one, 1, f, "cpu")
+    to32 = lambda t: qz.bf16_bits_to_f32(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+    kn, vn, qn = to32(k)[0, 0, 0], to32(v)[0, 0, 0], to32(q)[0, 0, 0].astype(np.float64)
+    st = ca.StreamCache(wl.head_dim, 2, 2, wl.n_sink, wl.n_recent)
+    t0 = time.perf_counter()
+    st.prefill(kn, vn)
+    t_quant = time.perf_counter() - t0
+    runs, t0 = 0, time.perf_counter()
+    while True:
+        kh, vh = st.dequantized()
+        at.attend(qn, kh, vh)
+        runs += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    t_dec = (time.perf_counter() - t0) / runs
+    kb = np.full((1, 1), 2)
+    bytes_dec = decode_bytes(one, kb, kb, wl.context)
+    bytes_q = wl.context * wl.head_dim * 2 * 2 + bytes_dec
+    return {
+        "decode_gbs": bytes_dec / t_dec / 1e9,
+        "decode_s": t_dec,
+        "quantize_gbs": bytes_q / t_quant / 1e9,
+        "threads": threads,
+        "sample": f"one of {wl.n_kv_heads} kv-head streams of {WORKLOAD} ({wl.context} tokens, {wl.group} query "
+                  f"heads, 2-bit K/V), one decode step (dequantize + fp64 attention), {runs} runs",
+    }
+
+
+def run_reference(args):
+    from quantized_decode_attention_head_b200 import workloads
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = workloads.CONFIGS[WORKLOAD]
+    seconds = max(5.0, 10.0 * (args.steps / max(args.steps, 1)))
+    res = oracle_sample(wl, seconds=seconds)
+    cb = {"value": res["decode_gbs"], "unit": "GB/s", "cores": res["threads"], "kind": "oracle",
+          "sample": res["sample"]}
+    line = {
+        "impl": "reference", "metric": METRIC, "value": res["decode_gbs"], "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["decode_s"] * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": res["sample"]},
+        "cpu_baseline": cb,
+        "e2e": {"value": res["decode_gbs"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def traffic_record():
+    """ncu DRAM traffic of the decode kernel recorded for the current sources."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    h = hashlib.sha256()
+    for name in ("rq_decode.cu", "rq_device.cuh", "rq_internal.h"):
+        h.update(open(os.path.join(ROOT, "quantized_decode_attention_head_b200", "csrc", name), "rb").read())
+    if rec.get("source_sha256") != h.hexdigest():
+        return None
+    return rec
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_decode_attention_head_b200 import QuantizedKVCache, rq_allocate_bits, workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    wl = workloads.CONFIGS[WORKLOAD]
+    NC = args.copies
+
+    # a1: allocation (host)
+    w, a, b, avg = workloads.allocation_inputs(wl)["kv"]
+    t0 = time.perf_counter()
+    alloc = rq_allocate_bits(w, a, b, avg, wl.allowed)
+    alloc_ms = (time.perf_counter() - t0) * 1e3
+    kb = alloc["b_int"].reshape(wl.n_layers, wl.n_kv_heads)
+
+    total_steps = args.warmup + args.steps
+    steps_per_copy = (total_steps + NC - 1) // NC + 1
+    max_tokens = wl.context + steps_per_copy + 32
+    caches, step_in = [], []
+    qbytes, qtimes = 0, []
+    stream = torch.cuda.current_stream()
+    for c in range(NC):
+        seed = wl.seed + 1000 * rank + c
+        k, v, f = workloads.kv_inputs(wl, "cuda", seed=seed)
+        cache = QuantizedKVCache(wl.n_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n_sink,
+                                 wl.n_recent, max_tokens, kb, kb)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        cache.rq_quantize_kv(k, v)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if c > 0:  # the first call pays one-time set-up
+            qtimes.append(e0.elapsed_time(e1) / 1e3)
+            qbytes = k.numel() * 2 * 2 + decode_bytes(wl, kb, kb, wl.context)
+        del k, v
+        q, kn, vn = workloads.step_inputs(wl, steps_per_copy, f, "cuda", seed=seed)
+        caches.append(cache)
+        step_in.append((q, kn, vn))
+    ws = caches[0].make_workspace(n_splits=args.splits)
+    outs = [torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=torch.float32, device="cuda") for _ in range(NC)]
+    torch.cuda.synchronize()
+
+    def do_step(i, timed_events=None):
+        c = i % NC
+        j = i // NC
+        cache, (q, kn, vn) = caches[c], step_in[c]
+        cache.rq_append_token(0, kn[j, 0], vn[j, 0])
+        if timed_events is not None:
+            timed_events[0].record(stream)
+        cache.rq_decode_attention(0, q[j, 0], out=outs[c], n_splits=args.splits, workspace=ws)
+        if timed_events is not None:
+            timed_events[1].record(stream)
+
+    lengths = [caches[c].length(0) for c in range(NC)]
+    for i in range(args.warmup):
+        do_step(i)
+    torch.cuda.synchronize()
+    step_bytes = 0
+    dec_bytes_steps = []
+    for i in range(args.warmup, total_steps):
+        c = i % NC
+        T_old = caches[c].length(0) + (i - args.warmup) // NC  # length before this step's append
+        ab = append_bytes(wl, kb, kb, T_old)
+        db = decode_bytes(wl, kb, kb, T_old + 1)
+        step_bytes += ab + db
+        dec_bytes_steps.append(db)
+    if world > 1:
+        dist.barrier()
+    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        torch.cuda.synchronize()
+        start.record(stream)
+        for n, i in enumerate(range(args.warmup, total_steps)):
+            do_step(i, dec_events[n])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed = start.elapsed_time(end) / 1e3
+    dec_times = [a.elapsed_time(b) / 1e3 for a, b in dec_events]
+    dec_avg = sum(dec_times) / len(dec_times)
+    dec_bytes_avg = sum(dec_bytes_steps) / len(dec_bytes_steps)
+    status = QuantizedKVCache.rq_decode_read_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+
+    # e2e: host buffers, copies inside the timed region
+    pin_q = [step_in[c][0].cpu().pin_memory() for c in range(NC)]
+    pin_k = [step_in[c][1].cpu().pin_memory() for c in range(NC)]
+    pin_v = [step_in[c][2].cpu().pin_memory() for c in range(NC)]
+    dq = [torch.empty_like(step_in[c][0][0, 0]) for c in range(NC)]
+    dk = [torch.empty_like(step_in[c][1][0, 0]) for c in range(NC)]
+    dv = [torch.empty_like(step_in[c][2][0, 0]) for c in range(NC)]
+    host_out = torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=torch.float32).pin_memory()
+    e2e_steps = min(args.steps, max(1, (steps_per_copy - (total_steps + NC - 1) // NC - 1) * NC))
+    base_len = [caches[c].length(0) for c in range(NC)]
+    e2e_bytes = 0
+    for i in range(e2e_steps):
+        c = i % NC
+        e2e_bytes += append_bytes(wl, kb, kb, base_len[c] + i // NC) + decode_bytes(wl, kb, kb, base_len[c] + i // NC + 1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    j0 = (total_steps + NC - 1) // NC
+    s2.record(stream)
+    for i in range(e2e_steps):
+        c = i % NC
+        j = j0 + i // NC
+        dq[c].copy_(pin_q[c][j, 0], non_blocking=True)
+        dk[c].copy_(pin_k[c][j, 0], non_blocking=True)
+        dv[c].copy_(pin_v[c][j, 0], non_blocking=True)
+        caches[c].rq_append_token(0, dk[c], dv[c])
+        caches[c].rq_decode_attention(0, dq[c], out=outs[c], n_splits=args.splits, workspace=ws)
+        host_out.copy_(outs[c], non_blocking=True)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_elapsed = s2.elapsed_time(e2) / 1e3
+    h2d = dq[0].numel() * 2 + dk[0].numel() * 2 + dv[0].numel() * 2
+    d2h = host_out.numel() * 4
+
+    # aggregate over ranks: bytes summed, time = slowest rank
+    vals = torch.tensor([elapsed, step_bytes, e2e_elapsed, e2e_bytes, dec_avg], dtype=torch.float64, device="cuda")
+    if world > 1:
+        mx = vals.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = vals.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        elapsed_all, bytes_all = mx[0].item(), sm[1].item()
+        e2e_el_all, e2e_b_all = mx[2].item(), sm[3].item()
+        dist.barrier()
+        dist.destroy_process_group()
+    else:
+        elapsed_all, bytes_all, e2e_el_all, e2e_b_all = elapsed, step_bytes, e2e_elapsed, e2e_bytes
+    if rank != 0:
+        return 0
+
+    peak, peak_kind = _peaks()
+    achieved = dec_bytes_avg / dec_avg / 1e9
+    tr = traffic_record()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": (tr["bytes_per_launch_scaled"] if tr else None),
+                "kernel": "decode_kernel<128,4> (split-K + fused combine)",
+                "peak_source": f"{peak_kind} hbm_gbs (burst)", "algorithmic_bytes_per_launch": dec_bytes_avg,
+                "avg_launch_us": dec_avg * 1e6}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        res = oracle_sample(wl, seconds=args.cpu_seconds)
+        cpu = {"value": res["decode_gbs"], "unit": "GB/s", "cores": res["threads"], "kind": "oracle",
+               "sample": res["sample"]}
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC,
+        "value": bytes_all / elapsed_all / 1e9,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": elapsed_all / args.steps * 1e3,
+        "us_per_step": elapsed_all / args.steps * 1e6,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u2+f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
+                   "head_dim": wl.head_dim, "context": wl.context, "bits": "K=V=2 on every head (avg 2 over {2,3,4})",
+                   "splits": args.splits or "auto", "l2": f"{NC} caches decoded round-robin "
+                   f"({NC * decode_bytes(wl, kb, kb, wl.context) / 1e6:.0f} MB > 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "decode_gbs": achieved,
+        "decode_us": dec_avg * 1e6,
+        "quantize_gbs": (qbytes / (sum(qtimes) / len(qtimes)) / 1e9) if qtimes else None,
+        "alloc_ms": alloc_ms,
+        "e2e": {"value": e2e_b_all / e2e_el_all / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": 2 * args.steps,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--copies", type=int, default=4)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

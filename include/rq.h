@@ -1,0 +1,210 @@
+/*
+ * rq.h -- mixed-precision, group-wise quantized KV cache and decode attention
+ * for NVIDIA B200 (sm_100a).  C ABI of librq.so.
+ *
+ * The operations follow three of the pages this library is built from:
+ *
+ *   RateQuant: Optimal Mixed-Precision KV Cache Quantization via
+ *   Rate-Distortion Theory (arXiv 2605.06675v2) -- per-head bit allocation
+ *   under an average-bit budget: distortion model D(b) = alpha*beta^-b (§3.1),
+ *   reverse waterfilling (§3.1, App. B.1), integer allocation (§3.3, App. U),
+ *   separate K and V budgets (§3.4).
+ *
+ *   InnerQ: Hardware-Aware Tuning-Free Quantization of KV Cache for Large
+ *   Language Models (arXiv 2602.23200) -- groups along the inner dimension of
+ *   the decode vector-matrix products (K: per token along head_dim; V: per
+ *   channel along tokens), asymmetric per-group quantization, high-precision
+ *   sink and recent windows, dequantization fused into decode attention
+ *   (abstract; "Core claim"; Algorithm 1, decode-phase attention).
+ *
+ *   Spend Bits Where Queries Look (NOVA-KV, arXiv 2608.04074, review page)
+ *   and Behavioral Capacity Certificates (arXiv 2609.37887, abstract) -- keys
+ *   need more precision than values, hence separate K and V bit widths.
+ *
+ * Conventions
+ *   - Every pointer named dev_* / k / v / q / out / workspace is DEVICE memory
+ *     owned by the caller.  The library never allocates or frees device memory.
+ *   - Device calls are asynchronous on the given stream; arguments are checked
+ *     on the host first and nothing is launched when a check fails.  After a
+ *     launch, a CUDA launch error is reported as RQ_ERR_CUDA.
+ *   - bf16 tensors are passed as raw 16-bit patterns (const void*), row-major
+ *     and contiguous; out is float32.
+ *   - Lengths are tracked on the host in the rq_cache handle, so no call reads
+ *     device memory back (except rq_cache_init and rq_decode_read_status,
+ *     which say so).
+ *   - A handle is not thread-safe; one handle per thread of control.
+ *
+ * Packed tile format (one record per 32-token tile of one (layer, batch,
+ * kv-head) stream; all offsets in bytes; the format is this library's own):
+ *   record = [K codes | K meta | V codes | V meta]
+ *   codes  : 32 lanes x W words, W = ceil(D / cpw), cpw = 16, 10, 8, 4 codes
+ *            per 32-bit word for b = 2, 3, 4, 8.  A word holds pairs of codes:
+ *            slot p keeps one code at bit b*p and the other at bit 16 + b*p.
+ *            Lane L = 4*gid + tig owns the elements of the 16x16 A-operand
+ *            fragments of the m16n8k16 tensor-core MMA, pair (mb, kb, r):
+ *              row = 16 mb + 8 (r&1) + gid, col = 16 kb + 8 (r>>1) + 2 tig + h
+ *            K: row = token, col = channel; V: row = channel, col = token.
+ *            Pairs are taken in quads (K: (mb, rr, group) over kb in the
+ *            group and r in {rr, rr+2}; V: (mb, rr) over kb and r) and quads
+ *            fill the lane's slots ordered by (class, word, slot) with
+ *            slot classes b=2: 0,1,2,3,4,0,1,2; b=4: 0,1,0,1; b=3,8: 0.
+ *            Word w of lane L lives at ((w/4)*32 + L)*16 + (w%4)*4 for
+ *            w < 4*floor(W/4), else floor(W/4)*512 + ((w - 4 floor(W/4))*32 + L)*4.
+ *   meta   : u32 = fp16 scale | bf16 zero << 16.  K: D/32 groups x 32 entries,
+ *            entry i = token 16((i>>1)&1) + 8(i&1) + (i>>2).  V: D entries,
+ *            entry i = channel 16*mb + 8*rr + gid, gid = i/(D/8),
+ *            mb = (i%(D/8))/2, rr = i%2.
+ *   Quantization rule per group (IEEE fp32, round to nearest even):
+ *     s = fp16(min((max - min) / (2^b - 1), 65504)), z = min (bf16),
+ *     c = clamp(rint((x - z) * (s > 0 ? 1/s : 0)), 0, 2^b - 1).
+ *   Windows per stream: sink K [S][D], sink V [S][D], recent ring K [R+32][D],
+ *   ring V [R+32][D] (bf16); token position P >= S sits in ring slot
+ *   (P - S) mod (R + 32).  With T tokens, Tq = 32*floor((T - S - R)/32) tokens
+ *   (0 when T < S + R) are quantized; the rest stay bf16.
+ */
+#ifndef RQ_H_
+#define RQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum {
+  RQ_OK = 0,
+  RQ_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad layer, ... */
+  RQ_ERR_UNSUPPORTED = 2,       /* head_dim not 64/128, group != 32, bits not in {2,3,4,8}, G not in {1,2,4,8} */
+  RQ_ERR_INFEASIBLE_BUDGET = 3, /* avg_bits outside [min S, max S] */
+  RQ_ERR_CAPACITY = 4,          /* tokens would exceed max_tokens, or buffer too small */
+  RQ_ERR_WORKSPACE = 5,         /* workspace too small */
+  RQ_ERR_CUDA = 6,              /* a CUDA runtime call failed */
+  RQ_ERR_DEVICE_TIMEOUT = 7     /* a kernel gave up waiting (see rq_decode_read_status) */
+} rq_status;
+
+/* Static, human-readable name of a status code.  Never NULL. */
+const char* rq_status_string(rq_status s);
+
+/* ---------------------------------------------------------------- allocation
+ * rq_allocate_bits -- RateQuant per-head bit allocation (host only, pure).
+ *   Continuous reverse waterfilling (§3.1, App. B.1): minimise
+ *   sum_h w_h alpha_h beta_h^-b_h subject to sum_h b_h = n * avg_bits and
+ *   min(S) <= b_h <= max(S); stationary point
+ *   b_h = clip(log_beta_h(w_h alpha_h ln(beta_h) / lambda)).
+ *   Integer allocation (§3.3, App. B.3, App. U): b_int[h] in S minimising the
+ *   same objective with sum_h b_int[h] <= floor(n * avg_bits); greedy
+ *   max-heap when S is contiguous, exact dynamic programme otherwise.  Among
+ *   allocations of equal distortion (relative 1e-12) the lexicographically
+ *   largest vector is returned.
+ * Arguments: n heads (n >= 1); w, alpha, beta host arrays [n] with w > 0,
+ *   alpha > 0, beta > 1; allowed host array [n_allowed] of distinct bit
+ *   widths in 1..16; b_cont [n] (nullable) receives the continuous solution,
+ *   b_int [n] the integer one; log_lambda (nullable) receives ln(lambda).
+ * Errors: RQ_ERR_INVALID_ARG, RQ_ERR_INFEASIBLE_BUDGET.  Outputs untouched on
+ *   error.  Memory: all host, caller-owned. */
+rq_status rq_allocate_bits(int n, const double* w, const double* alpha, const double* beta,
+                           double avg_bits, const int* allowed, int n_allowed,
+                           double* b_cont, int* b_int, double* log_lambda);
+
+/* --------------------------------------------------------------------- cache */
+typedef struct {
+  int n_layers;      /* L >= 1 */
+  int batch;         /* B >= 1 */
+  int n_q_heads;     /* Hq, multiple of n_kv_heads, Hq/Hkv in {1,2,4,8} */
+  int n_kv_heads;    /* Hkv >= 1 */
+  int head_dim;      /* D in {64, 128} */
+  int group;         /* must be 32 (tokens per V group = channels per K group) */
+  int n_sink;        /* S >= 0 bf16 sink tokens */
+  int n_recent;      /* R >= 0 minimum bf16 recent tokens */
+  int max_tokens;    /* capacity per sequence */
+  const int* k_bits; /* host [L*Hkv] in {2,3,4,8}, index l*Hkv + h (copied) */
+  const int* v_bits; /* host [L*Hkv] in {2,3,4,8} (copied) */
+} rq_cache_config;
+
+typedef struct rq_cache rq_cache; /* opaque host handle */
+
+/* Device buffer size needed for cfg (header + tile records + windows). */
+rq_status rq_cache_bytes(const rq_cache_config* cfg, size_t* bytes);
+
+/* Bind a caller-owned device buffer (>= rq_cache_bytes, 256-byte aligned) to
+ * a new host handle with length 0.  Writes the buffer's descriptor header with
+ * a synchronous cudaMemcpy on the current device (the only blocking call
+ * besides rq_decode_read_status).  *out receives the handle. */
+rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes, rq_cache** out);
+
+/* Free the host handle (never the device buffer).  NULL is ignored. */
+void rq_cache_destroy(rq_cache* cache);
+
+/* Current token count of a layer (all batch elements share it). */
+rq_status rq_cache_length(const rq_cache* cache, int layer, int* tokens);
+
+/* Where a stream's data lives inside the device buffer (byte offsets from the
+ * buffer start): tile records (tile i at tile_offset + i*record_bytes, valid
+ * for i < *n_tiles) and the window block (sink K, sink V, ring K, ring V). */
+rq_status rq_cache_stream_layout(const rq_cache* cache, int layer, int b, int kv_head,
+                                 size_t* tile_offset, int* record_bytes, int* n_tiles,
+                                 size_t* window_offset);
+
+/* ------------------------------------------------------------- quantize / pack
+ * rq_quantize_kv -- prefill: quantize and pack a T-token prefix of every
+ *   layer, replacing the cache contents (InnerQ groups, fp16 scale / bf16
+ *   zero, per-(layer, kv-head) bits).  k, v: device bf16
+ *   [L][B][Hkv][T][D] contiguous.  Tokens [0,S) go to the sink, Tq tokens to
+ *   tiles, the rest to the recent ring.  n_tokens in [0, max_tokens].
+ * Errors: RQ_ERR_INVALID_ARG, RQ_ERR_CAPACITY, RQ_ERR_CUDA. */
+rq_status rq_quantize_kv(rq_cache* cache, const void* k, const void* v, int n_tokens,
+                         cudaStream_t stream);
+
+/* rq_append_token -- add one token per (batch, kv-head) to one layer
+ *   (layer >= 0; k_new, v_new bf16 [B][Hkv][D]) or to all layers at once
+ *   (layer = -1; [L][B][Hkv][D]; every layer must have the same length).
+ *   The token enters the recent ring (or the sink while T < S); when the
+ *   recent window reaches R + 32 tokens its oldest 32 are quantized into the
+ *   next tile by the same rule as rq_quantize_kv.
+ * Errors: RQ_ERR_INVALID_ARG, RQ_ERR_CAPACITY (length would pass max_tokens),
+ *   RQ_ERR_CUDA. */
+rq_status rq_append_token(rq_cache* cache, int layer, const void* k_new, const void* v_new,
+                          cudaStream_t stream);
+
+/* ---------------------------------------------------------- decode attention
+ * Workspace (caller-owned device memory) holds split partials, per-stream
+ * completion counters and a status word.  Size it with
+ * rq_decode_workspace_bytes (valid for every layer argument and every split
+ * count <= n_splits) and zero it once with rq_decode_workspace_init; every
+ * successful rq_decode_attention leaves the counters at zero again.  Calls
+ * that share a workspace must not overlap on the GPU. */
+rq_status rq_decode_workspace_bytes(const rq_cache* cache, int n_splits, size_t* bytes);
+rq_status rq_decode_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* rq_decode_attention -- one decode step of grouped-query attention over the
+ *   packed cache (InnerQ Algorithm 1, decode phase; the page's listing is cut
+ *   off, so the standard softmax(q K^T * scale) V is computed).  Query head h
+ *   reads kv head h / (Hq/Hkv).  Reads every cached token: bf16 sink, packed
+ *   tiles (dequantized inside the dot products: per-group scale and zero
+ *   factored out of the inner sums), bf16 recent window.  Split-K over tiles
+ *   with a fused log-sum-exp combine.
+ * q: device bf16 [B][Hq][D] (layer >= 0) or [L][B][Hq][D] (layer = -1).
+ * out: device float32, same shape.  softmax_scale <= 0 selects 1/sqrt(D).
+ * n_splits: tile splits per stream, 0 = automatic; capped to the tile count.
+ * Errors: RQ_ERR_INVALID_ARG, RQ_ERR_WORKSPACE, RQ_ERR_CUDA. */
+rq_status rq_decode_attention(rq_cache* cache, int layer, const void* q, float* out,
+                              float softmax_scale, int n_splits, void* workspace,
+                              size_t ws_bytes, cudaStream_t stream);
+
+/* Blocking read of the workspace status word: 0 when every kernel that used
+ * this workspace completed normally, otherwise RQ_ERR_DEVICE_TIMEOUT in the
+ * low byte (a pipeline wait gave up after ~1 s and the kernel returned
+ * without writing its outputs). */
+rq_status rq_decode_read_status(const void* workspace, int* device_status);
+
+/* Library build description (static string). */
+const char* rq_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RQ_H_ */

@@ -68,9 +68,11 @@ class StreamCache:
         self.sink_k = [k[i].copy() for i in range(s)]
         self.sink_v = [v[i].copy() for i in range(s)]
         self.tiles = []
-        for i in range(tq // TILE):
-            a = s + TILE * i
-            self.tiles.append(qz.quantize_tile(k[a : a + TILE], v[a : a + TILE], self.kb, self.vb))
+        n = tq // TILE
+        if n:
+            d = self.d
+            qb = qz.quantize_tiles(k[s : s + tq].reshape(n, TILE, d), v[s : s + tq].reshape(n, TILE, d), self.kb, self.vb)
+            self.tiles = [{key: val[i] for key, val in qb.items()} for i in range(n)]
         self.recent = [(p, k[p].copy(), v[p].copy()) for p in range(s + tq, T)]
         self.T = T
 
@@ -103,10 +105,10 @@ class StreamCache:
         if self.sink_k:
             parts_k.append(np.stack(self.sink_k).astype(np.float64))
             parts_v.append(np.stack(self.sink_v).astype(np.float64))
-        for t in self.tiles:
-            kh, vh = qz.dequantize_tile(t)
-            parts_k.append(kh)
-            parts_v.append(vh)
+        if self.tiles:
+            kh, vh = qz.dequantize_tile({key: np.stack([t[key] for t in self.tiles]) for key in self.tiles[0]})
+            parts_k.append(kh.reshape(-1, self.d))
+            parts_v.append(vh.reshape(-1, self.d))
         if self.recent:
             parts_k.append(np.stack([r[1] for r in self.recent]).astype(np.float64))
             parts_v.append(np.stack([r[2] for r in self.recent]).astype(np.float64))
@@ -116,6 +118,13 @@ class StreamCache:
 
     def record(self, i: int) -> np.ndarray:
         return qz.pack_record(self.tiles[i], self.kb, self.vb)
+
+    def records(self) -> np.ndarray:
+        """All tile records, uint8 [n_tiles, record_bytes]."""
+        if not self.tiles:
+            return np.zeros((0, qz.record_bytes(self.kb, self.vb, self.d)), dtype=np.uint8)
+        qb = {key: np.stack([t[key] for t in self.tiles]) for key in self.tiles[0]}
+        return qz.pack_records(qb, self.kb, self.vb)
 
     def window_rows(self):
         """Expected window content as {('sink'|'ring', 'k'|'v', slot): bf16 bits}."""

@@ -124,30 +124,37 @@ def quantize_tile(k_tile: np.ndarray, v_tile: np.ndarray, kb: int, vb: int):
     tile's 32 tokens.  Returns dict with codes [32, D] (token-major) for K and
     V, K scale/zero [32, D/32], V scale/zero [D].
     """
-    t, d = k_tile.shape
+    q = quantize_tiles(k_tile[None], v_tile[None], kb, vb)
+    return {key: val[0] for key, val in q.items()}
+
+
+def quantize_tiles(k_tiles: np.ndarray, v_tiles: np.ndarray, kb: int, vb: int):
+    """The same rule applied to n tiles at once: inputs [n, 32, D]; outputs
+    carry a leading tile axis."""
+    n, t, d = k_tiles.shape
     assert t == TILE and d % 32 == 0
-    kx = k_tile.reshape(TILE, d // 32, 32)
-    kc, ks, kz = quantize_groups(kx, kb, axis=2)
-    vc, vs, vz = quantize_groups(v_tile, vb, axis=0)
+    kx = np.asarray(k_tiles, dtype=np.float32).reshape(n, TILE, d // 32, 32)
+    kc, ks, kz = quantize_groups(kx, kb, axis=3)
+    vc, vs, vz = quantize_groups(np.asarray(v_tiles, dtype=np.float32), vb, axis=1)
     return {
-        "k_codes": kc.reshape(TILE, d),
-        "k_s": ks,  # [32 tokens, D/32 groups]
+        "k_codes": kc.reshape(n, TILE, d),
+        "k_s": ks,  # [n, 32 tokens, D/32 groups]
         "k_z": kz,
-        "v_codes": vc,  # [32 tokens, D]
-        "v_s": vs,  # [D]
+        "v_codes": vc,  # [n, 32 tokens, D]
+        "v_s": vs,  # [n, D]
         "v_z": vz,
     }
 
 
 def dequantize_tile(q: dict) -> tuple[np.ndarray, np.ndarray]:
-    """fp64 x_hat = c * s + z for K and V of one tile."""
+    """fp64 x_hat = c * s + z for K and V of one tile (or of n tiles with a
+    leading tile axis)."""
     kc = q["k_codes"].astype(np.float64)
-    t, d = kc.shape
-    ks = np.repeat(q["k_s"].astype(np.float64), 32, axis=1)
-    kz = np.repeat(q["k_z"].astype(np.float64), 32, axis=1)
+    ks = np.repeat(q["k_s"].astype(np.float64), 32, axis=-1)
+    kz = np.repeat(q["k_z"].astype(np.float64), 32, axis=-1)
     vc = q["v_codes"].astype(np.float64)
-    vs = q["v_s"].astype(np.float64)[None, :]
-    vz = q["v_z"].astype(np.float64)[None, :]
+    vs = q["v_s"].astype(np.float64)[..., None, :]
+    vz = q["v_z"].astype(np.float64)[..., None, :]
     return kc * ks + kz, vc * vs + vz
 
 
@@ -220,15 +227,25 @@ def blob_bytes(b: int, head_dim: int) -> int:
 
 
 def pack_blob(codes_rc: np.ndarray, role: str, b: int) -> np.ndarray:
-    """codes_rc: uint8 [rows, cols] in fragment coordinates
-    (K: [token, channel]; V: [channel, token]).  Returns the blob as uint8."""
-    head_dim = codes_rc.shape[1] if role == "K" else codes_rc.shape[0]
+    """codes_rc: uint8 [rows, cols] (or [n, rows, cols]) in fragment
+    coordinates (K: [token, channel]; V: [channel, token]).  Returns the blob
+    bytes (uint8 [blob] or [n, blob])."""
+    single = codes_rc.ndim == 2
+    c = codes_rc[None] if single else codes_rc
+    head_dim = c.shape[2] if role == "K" else c.shape[1]
     rows, cols, wbyte, bit = pack_table(role, b, head_dim)
-    n_bytes = blob_bytes(b, head_dim)
-    words = np.zeros(n_bytes // 4, dtype=np.uint32)
-    vals = codes_rc[rows, cols].astype(np.uint32) << bit.astype(np.uint32)
-    np.bitwise_or.at(words, wbyte // 4, vals)
-    return words.view(np.uint8)
+    n_words = blob_bytes(b, head_dim) // 4
+    # codes never overlap inside a word, so OR == sum over the codes of a word
+    vals = c[:, rows, cols].astype(np.uint64) << bit.astype(np.uint64)
+    words = np.zeros((c.shape[0], n_words), dtype=np.uint64)
+    order = np.argsort(wbyte, kind="stable")
+    w_sorted = wbyte[order] // 4
+    starts = np.searchsorted(w_sorted, np.arange(n_words))
+    present = np.unique(w_sorted)
+    sums = np.add.reduceat(vals[:, order], starts[present], axis=1)
+    words[:, present] = sums
+    out = words.astype(np.uint32).view(np.uint8)
+    return out[0] if single else out
 
 
 def unpack_blob(blob: np.ndarray, role: str, b: int, head_dim: int) -> np.ndarray:
@@ -265,18 +282,26 @@ def record_bytes(kb: int, vb: int, head_dim: int) -> int:
 
 def pack_record(q: dict, kb: int, vb: int) -> np.ndarray:
     """Serialize one quantized tile into its record bytes."""
-    d = q["k_codes"].shape[1]
+    return pack_records({k: v[None] for k, v in q.items()}, kb, vb)[0]
+
+
+def pack_records(q: dict, kb: int, vb: int) -> np.ndarray:
+    """Serialize n quantized tiles (leading tile axis) -> uint8 [n, record]."""
+    n, _, d = q["k_codes"].shape
     kblob = pack_blob(q["k_codes"], "K", kb)
-    i = np.arange(32)
-    t_of_i = k_meta_token(i)
+    t_of_i = k_meta_token(np.arange(32))
     kmeta = np.concatenate(
-        [meta_word(q["k_s"][t_of_i, g], q["k_z"][t_of_i, g]) for g in range(d // 32)]
+        [meta_word(q["k_s"][:, t_of_i, g], q["k_z"][:, t_of_i, g]) for g in range(d // 32)], axis=1
     )
-    vblob = pack_blob(np.ascontiguousarray(q["v_codes"].T), "V", vb)
+    vblob = pack_blob(np.ascontiguousarray(np.swapaxes(q["v_codes"], 1, 2)), "V", vb)
     d_of_i = v_meta_channel(np.arange(d), d)
-    vmeta = meta_word(q["v_s"][d_of_i], q["v_z"][d_of_i])
-    out = np.concatenate([kblob, kmeta.view(np.uint8), vblob, vmeta.view(np.uint8)])
-    assert out.size == record_bytes(kb, vb, d)
+    vmeta = meta_word(q["v_s"][:, d_of_i], q["v_z"][:, d_of_i])
+    kmeta = np.ascontiguousarray(kmeta, dtype=np.uint32)
+    vmeta = np.ascontiguousarray(vmeta, dtype=np.uint32)
+    out = np.concatenate(
+        [kblob, kmeta.view(np.uint8).reshape(n, -1), vblob, vmeta.view(np.uint8).reshape(n, -1)], axis=1
+    )
+    assert out.shape[1] == record_bytes(kb, vb, d)
     return out
 
 

@@ -1,0 +1,307 @@
+// Host side of the C ABI: argument checks, the cache buffer layout, length
+// bookkeeping and kernel launches.  See include/rq.h for the contract.
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "rq.h"
+#include "rq_internal.h"
+
+using rq::HeadDesc;
+
+struct rq_cache {
+  rq::Geom g;
+  int max_tokens;
+  std::vector<int> k_bits, v_bits;
+  std::vector<HeadDesc> desc;  // host copy of the device header
+  uint8_t* buf;
+  size_t bytes;
+  std::vector<int> length;  // tokens per layer
+  int sm_count;
+};
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
+
+rq_status check_config(const rq_cache_config* c) {
+  if (!c || !c->k_bits || !c->v_bits) return RQ_ERR_INVALID_ARG;
+  if (c->n_layers < 1 || c->batch < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_sink < 0 ||
+      c->n_recent < 0 || c->max_tokens < 0)
+    return RQ_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128) return RQ_ERR_UNSUPPORTED;
+  if (c->group != rq::kTile) return RQ_ERR_UNSUPPORTED;
+  if (c->n_q_heads % c->n_kv_heads != 0) return RQ_ERR_UNSUPPORTED;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return RQ_ERR_UNSUPPORTED;
+  for (int i = 0; i < c->n_layers * c->n_kv_heads; ++i)
+    if (!valid_bits(c->k_bits[i]) || !valid_bits(c->v_bits[i])) return RQ_ERR_UNSUPPORTED;
+  return RQ_OK;
+}
+
+// Computes the geometry, the per-(layer, kv-head) descriptors and the total size.
+size_t layout(const rq_cache_config* c, rq::Geom& g, std::vector<HeadDesc>& desc) {
+  g.L = c->n_layers;
+  g.B = c->batch;
+  g.Hq = c->n_q_heads;
+  g.Hkv = c->n_kv_heads;
+  g.D = c->head_dim;
+  g.G = c->n_q_heads / c->n_kv_heads;
+  g.S = c->n_sink;
+  g.R = c->n_recent;
+  g.max_tiles = rq::quantized_tokens(c->max_tokens, g.S, g.R) / rq::kTile;
+  g.win_bytes = rq::window_bytes(g.S, g.R, g.D);
+  const int nh = g.L * g.Hkv;
+  desc.assign(nh, HeadDesc{});
+  size_t off = align_up((size_t)nh * sizeof(HeadDesc), rq::kHeaderAlign);
+  for (int i = 0; i < nh; ++i) {
+    HeadDesc& d = desc[i];
+    d.k_bits = c->k_bits[i];
+    d.v_bits = c->v_bits[i];
+    d.rec_bytes = rq::record_bytes(d.k_bits, d.v_bits, g.D);
+    d.tile_base = (int64_t)off;
+    d.tile_stride = (int64_t)g.max_tiles * d.rec_bytes;
+    off = align_up(off + (size_t)g.B * d.tile_stride, rq::kHeaderAlign);
+  }
+  for (int i = 0; i < nh; ++i) {
+    desc[i].win_base = (int64_t)off;
+    off = align_up(off + (size_t)g.B * g.win_bytes, rq::kHeaderAlign);
+  }
+  return off;
+}
+
+bool layer_range(const rq_cache* c, int layer, int& l0, int& nl) {
+  if (layer == -1) {
+    l0 = 0;
+    nl = c->g.L;
+    for (int l = 1; l < c->g.L; ++l)
+      if (c->length[l] != c->length[0]) return false;
+    return true;
+  }
+  if (layer < 0 || layer >= c->g.L) return false;
+  l0 = layer;
+  nl = 1;
+  return true;
+}
+
+int auto_splits(const rq_cache* c, int streams, int n_tiles) {
+  if (n_tiles <= 0) return 0;
+  const int target = c->sm_count * 4;  // about four resident CTAs per SM
+  int s = (target + streams - 1) / streams;
+  if (s < 1) s = 1;
+  // keep at least 8 tiles per split so a CTA's pipeline fills
+  const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;
+  if (s > max_by_work) s = max_by_work;
+  if (s > n_tiles) s = n_tiles;
+  return s;
+}
+
+rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* rq_status_string(rq_status s) {
+  switch (s) {
+    case RQ_OK: return "ok";
+    case RQ_ERR_INVALID_ARG: return "invalid argument";
+    case RQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RQ_ERR_INFEASIBLE_BUDGET: return "infeasible bit budget";
+    case RQ_ERR_CAPACITY: return "capacity exceeded";
+    case RQ_ERR_WORKSPACE: return "workspace too small";
+    case RQ_ERR_CUDA: return "CUDA error";
+    case RQ_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* rq_build_info(void) {
+  return "librq: sm_100a; quantize/pack, append/flush, split-K mma.sync decode with bulk-copy pipeline";
+}
+
+rq_status rq_cache_bytes(const rq_cache_config* cfg, size_t* bytes) {
+  if (!bytes) return RQ_ERR_INVALID_ARG;
+  const rq_status st = check_config(cfg);
+  if (st != RQ_OK) return st;
+  rq::Geom g;
+  std::vector<HeadDesc> desc;
+  *bytes = layout(cfg, g, desc);
+  return RQ_OK;
+}
+
+rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes, rq_cache** out) {
+  if (!out || !dev_buf) return RQ_ERR_INVALID_ARG;
+  const rq_status st = check_config(cfg);
+  if (st != RQ_OK) return st;
+  if (reinterpret_cast<uintptr_t>(dev_buf) % rq::kHeaderAlign != 0) return RQ_ERR_INVALID_ARG;
+  rq_cache* c = new (std::nothrow) rq_cache();
+  if (!c) return RQ_ERR_INVALID_ARG;
+  const size_t need = layout(cfg, c->g, c->desc);
+  if (bytes < need) {
+    delete c;
+    return RQ_ERR_CAPACITY;
+  }
+  c->max_tokens = cfg->max_tokens;
+  c->k_bits.assign(cfg->k_bits, cfg->k_bits + c->g.L * c->g.Hkv);
+  c->v_bits.assign(cfg->v_bits, cfg->v_bits + c->g.L * c->g.Hkv);
+  c->buf = static_cast<uint8_t*>(dev_buf);
+  c->bytes = bytes;
+  c->length.assign(c->g.L, 0);
+  int dev = 0;
+  c->sm_count = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) c->sm_count = n;
+  }
+  const cudaError_t e =
+      cudaMemcpy(c->buf, c->desc.data(), c->desc.size() * sizeof(HeadDesc), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    delete c;
+    return RQ_ERR_CUDA;
+  }
+  *out = c;
+  return RQ_OK;
+}
+
+void rq_cache_destroy(rq_cache* cache) { delete cache; }
+
+rq_status rq_cache_length(const rq_cache* c, int layer, int* tokens) {
+  if (!c || !tokens || layer < 0 || layer >= c->g.L) return RQ_ERR_INVALID_ARG;
+  *tokens = c->length[layer];
+  return RQ_OK;
+}
+
+rq_status rq_cache_stream_layout(const rq_cache* c, int layer, int b, int kv_head, size_t* tile_offset,
+                                 int* record_bytes, int* n_tiles, size_t* window_offset) {
+  if (!c || layer < 0 || layer >= c->g.L || b < 0 || b >= c->g.B || kv_head < 0 || kv_head >= c->g.Hkv)
+    return RQ_ERR_INVALID_ARG;
+  const HeadDesc& d = c->desc[layer * c->g.Hkv + kv_head];
+  if (tile_offset) *tile_offset = (size_t)(d.tile_base + (int64_t)b * d.tile_stride);
+  if (record_bytes) *record_bytes = d.rec_bytes;
+  if (n_tiles) *n_tiles = rq::quantized_tokens(c->length[layer], c->g.S, c->g.R) / rq::kTile;
+  if (window_offset) *window_offset = (size_t)(d.win_base + (int64_t)b * c->g.win_bytes);
+  return RQ_OK;
+}
+
+rq_status rq_quantize_kv(rq_cache* c, const void* k, const void* v, int n_tokens, cudaStream_t stream) {
+  if (!c || n_tokens < 0 || (n_tokens > 0 && (!k || !v))) return RQ_ERR_INVALID_ARG;
+  if (n_tokens > c->max_tokens) return RQ_ERR_CAPACITY;
+  rq::QuantizeArgs a;
+  a.g = c->g;
+  a.buf = c->buf;
+  a.desc = reinterpret_cast<const HeadDesc*>(c->buf);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.T = n_tokens;
+  a.Tq = rq::quantized_tokens(n_tokens, c->g.S, c->g.R);
+  if (n_tokens > 0) {
+    const rq_status st = cuda_status(rq::launch_quantize(a, stream));
+    if (st != RQ_OK) return st;
+  }
+  for (int l = 0; l < c->g.L; ++l) c->length[l] = n_tokens;
+  return RQ_OK;
+}
+
+rq_status rq_append_token(rq_cache* c, int layer, const void* k_new, const void* v_new, cudaStream_t stream) {
+  if (!c || !k_new || !v_new) return RQ_ERR_INVALID_ARG;
+  int l0, nl;
+  if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
+  const int T_old = c->length[l0];
+  if (T_old + 1 > c->max_tokens) return RQ_ERR_CAPACITY;
+  rq::AppendArgs a;
+  a.g = c->g;
+  a.buf = c->buf;
+  a.desc = reinterpret_cast<const HeadDesc*>(c->buf);
+  a.k_new = static_cast<const uint16_t*>(k_new);
+  a.v_new = static_cast<const uint16_t*>(v_new);
+  a.layer0 = l0;
+  a.n_layers = nl;
+  a.T_old = T_old;
+  const int S = c->g.S, R = c->g.R;
+  const int Tq_old = rq::quantized_tokens(T_old, S, R);
+  a.flush = (T_old >= S && (T_old - S - Tq_old) + 1 == R + rq::kTile) ? 1 : 0;
+  a.flush_pos = S + Tq_old;
+  a.flush_tile = Tq_old / rq::kTile;
+  const rq_status st = cuda_status(rq::launch_append(a, stream));
+  if (st != RQ_OK) return st;
+  for (int l = l0; l < l0 + nl; ++l) c->length[l] = T_old + 1;
+  return RQ_OK;
+}
+
+rq_status rq_decode_workspace_bytes(const rq_cache* c, int n_splits, size_t* bytes) {
+  if (!c || !bytes || n_splits < 0) return RQ_ERR_INVALID_ARG;
+  const int streams_layer = c->g.B * c->g.Hkv;
+  const int max_tiles = c->g.max_tiles;
+  int s = n_splits;
+  const int a1 = auto_splits(c, streams_layer, max_tiles);
+  const int a2 = auto_splits(c, streams_layer * c->g.L, max_tiles);
+  if (s < a1) s = a1;
+  if (s < a2) s = a2;
+  const int64_t all = (int64_t)streams_layer * c->g.L;
+  *bytes = rq::ws_total_bytes(all, all, s + 1, c->g.G, c->g.D);
+  return RQ_OK;
+}
+
+rq_status rq_decode_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!workspace || ws_bytes < rq::ws_counter_offset()) return RQ_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, ws_bytes, stream));
+}
+
+rq_status rq_decode_read_status(const void* workspace, int* device_status) {
+  if (!workspace || !device_status) return RQ_ERR_INVALID_ARG;
+  return cuda_status(cudaMemcpy(device_status, workspace, sizeof(int), cudaMemcpyDeviceToHost));
+}
+
+rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out, float softmax_scale, int n_splits,
+                              void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!c || !q || !out || !workspace || n_splits < 0) return RQ_ERR_INVALID_ARG;
+  int l0, nl;
+  if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
+  const int T = c->length[l0];
+  const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
+  const int n_tiles = Tq / rq::kTile;
+  const int streams = nl * c->g.B * c->g.Hkv;
+  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles) : n_splits;
+  if (splits > n_tiles) splits = n_tiles;
+  if (n_tiles > 0 && splits < 1) splits = 1;
+  const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
+  if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + 1, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
+  if (streams > 65535) return RQ_ERR_UNSUPPORTED;
+  int stage_bytes = 16;
+  for (int l = l0; l < l0 + nl; ++l)
+    for (int h = 0; h < c->g.Hkv; ++h) {
+      const int r = c->desc[l * c->g.Hkv + h].rec_bytes;
+      if (r > stage_bytes) stage_bytes = r;
+    }
+  rq::DecodeArgs a;
+  a.g = c->g;
+  a.buf = c->buf;
+  a.desc = reinterpret_cast<const HeadDesc*>(c->buf);
+  a.q = static_cast<const uint16_t*>(q);
+  a.out = out;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)c->g.D);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.layer0 = l0;
+  a.n_layers = nl;
+  a.T = T;
+  a.Tq = Tq;
+  a.n_tiles = n_tiles;
+  a.n_splits = splits;
+  a.stages = 8;
+  a.stage_bytes = stage_bytes;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.status = reinterpret_cast<int*>(ws);
+  a.counters = reinterpret_cast<uint32_t*>(ws + rq::ws_counter_offset());
+  a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
+  const int smem = rq::decode_smem_bytes(splits + 1, stage_bytes, c->g.G, c->g.D);
+  if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
+  return cuda_status(rq::launch_decode(a, smem, stream));
+}
+
+}  // extern "C"

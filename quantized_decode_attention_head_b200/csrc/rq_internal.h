@@ -1,0 +1,115 @@
+// Internal declarations shared by the host library and the CUDA kernels.
+// Not part of the public C ABI (include/rq.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace rq {
+
+constexpr int kTile = 32;          // tokens per packed tile == group size
+constexpr int kHeaderAlign = 256;  // alignment of every region of the cache buffer
+
+// One descriptor per (layer, kv-head), stored at the start of the device buffer.
+struct HeadDesc {
+  int32_t k_bits;
+  int32_t v_bits;
+  int32_t rec_bytes;   // bytes of one packed tile record
+  int32_t pad;
+  int64_t tile_base;   // byte offset of batch element 0's tile records
+  int64_t tile_stride; // bytes between batch elements (max_tiles * rec_bytes)
+  int64_t win_base;    // byte offset of batch element 0's window block
+};
+static_assert(sizeof(HeadDesc) == 40, "HeadDesc layout");
+
+struct Geom {
+  int L, B, Hq, Hkv, D, G, S, R;
+  int max_tiles;
+  int64_t win_bytes;   // bytes of one stream's window block
+};
+
+// codes per 32-bit word for a bit width
+__host__ __device__ constexpr int codes_per_word(int b) { return b == 2 ? 16 : b == 3 ? 10 : b == 4 ? 8 : 4; }
+__host__ __device__ constexpr int words_per_lane(int b, int d) { return (d + codes_per_word(b) - 1) / codes_per_word(b); }
+__host__ __device__ constexpr int blob_bytes(int b, int d) { return words_per_lane(b, d) * 128; }
+__host__ __device__ constexpr int record_bytes(int kb, int vb, int d) {
+  return blob_bytes(kb, d) + 4 * d + blob_bytes(vb, d) + 4 * d;
+}
+
+// Window block of one stream: [sink K][sink V][ring K][ring V], bf16 rows of D.
+__host__ __device__ inline int64_t window_bytes(int S, int R, int D) {
+  return (int64_t)(2 * S + 2 * (R + kTile)) * D * 2;
+}
+
+// Quantized token count for T tokens (multiple of 32; recent window in [R, R+32)).
+__host__ __device__ inline int quantized_tokens(int T, int S, int R) {
+  return T >= S + R ? ((T - S - R) / kTile) * kTile : 0;
+}
+
+struct QuantizeArgs {
+  Geom g;
+  uint8_t* buf;
+  const HeadDesc* desc;
+  const uint16_t* k;   // [L][B][Hkv][T][D]
+  const uint16_t* v;
+  int T;
+  int Tq;
+};
+
+struct AppendArgs {
+  Geom g;
+  uint8_t* buf;
+  const HeadDesc* desc;
+  const uint16_t* k_new;  // [nL][B][Hkv][D]
+  const uint16_t* v_new;
+  int layer0, n_layers;
+  int T_old;              // length before the append
+  int flush;              // 1: quantize ring positions [flush_pos, flush_pos+32) into tile flush_tile
+  int flush_pos;
+  int flush_tile;
+};
+
+struct DecodeArgs {
+  Geom g;
+  const uint8_t* buf;
+  const HeadDesc* desc;
+  const uint16_t* q;      // [nL][B][Hq][D]
+  float* out;             // [nL][B][Hq][D]
+  float scale_log2;       // softmax scale * log2(e)
+  int layer0, n_layers;
+  int T, Tq, n_tiles;
+  int n_splits;           // tile splits; item n_splits is the bf16 window
+  int stages;             // pipeline depth (multiple of the consumer warp count)
+  int stage_bytes;        // bytes per stage (max record size in the call)
+  float* partials;        // [streams][n_splits+1][G*D + 2G]
+  uint32_t* counters;     // [streams]
+  int* status;            // workspace status word
+};
+
+// Workspace layout (bytes): [status int32, pad to 256][one u32 counter per
+// stream of the whole cache (L*B*Hkv), pad to 256][partials of one call].
+// The counter region is sized for every stream so calls with different layer
+// arguments never overlap each other's counters.
+inline size_t ws_counter_offset() { return 256; }
+inline size_t ws_partial_offset(int64_t all_streams) {
+  size_t c = ws_counter_offset() + (size_t)all_streams * 4;
+  return (c + 255) / 256 * 256;
+}
+inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int items, int G, int D) {
+  return ws_partial_offset(all_streams) + (size_t)call_streams * items * (size_t)(G * D + 2 * G) * 4;
+}
+
+// Kernel launchers (rq_kernels.cu).  Return cudaGetLastError() after launch.
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, int smem_bytes, cudaStream_t s);
+int decode_smem_bytes(int n_items, int stage_bytes, int G, int D);
+cudaError_t decode_set_smem_limit(int smem_bytes);
+
+constexpr int kDecodeConsumerWarps = 4;
+constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
+constexpr int kDeviceTimeout = 7;  // == RQ_ERR_DEVICE_TIMEOUT
+
+}  // namespace rq

@@ -1,0 +1,190 @@
+"""GPU parity on small caches: packed bytes bit-exact against the oracle,
+decode attention within max-abs 2e-3 / rel-L2 1e-3 of the fp64 oracle.
+
+Sizes span several tiles with a ragged recent window; every bit width for K
+and V, head_dim 64 and 128, GQA groups 1/2/4/8, split counts from 1 to one
+split per tile, the all-layers call, and the short-cache edge cases."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import (all_streams, assert_close, check_stream_bytes, make_cache, oracle_decode, oracle_streams,
+                         to_f32, workload_bits)
+from oracle import cache as ca
+from quantized_decode_attention_head_b200 import workloads
+from quantized_decode_attention_head_b200.api import QuantizedKVCache
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(**kw):
+    base = dict(name="small", n_layers=2, batch=2, n_q_heads=8, n_kv_heads=4, head_dim=128, context=4 + 32 * 6 + 32 + 13,
+                n_sink=4, n_recent=32, k_sigma=1.5, allowed=(2, 3, 4, 8), avg_bits=3.0, seed=7)
+    base.update(kw)
+    return workloads.Workload(**base)
+
+
+def _bits_grid(L, H):
+    kb = np.array([[[2, 3, 4, 8][(l + h) % 4] for h in range(H)] for l in range(L)])
+    vb = np.array([[[8, 2, 3, 4][(l + 2 * h) % 4] for h in range(H)] for l in range(L)])
+    return kb, vb
+
+
+def _build(wl, kb, vb, extra=64):
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, wl.context + extra)
+    cache.rq_quantize_kv(k, v)
+    torch.cuda.synchronize()
+    st = oracle_streams(wl, kb, vb, to_f32(k), to_f32(v), all_streams(wl))
+    return cache, st, (k, v, f)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_quantize_all_bit_pairs_bitexact(d):
+    wl = _small(head_dim=d)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    cache, st, _ = _build(wl, kb, vb)
+    assert cache.length(0) == wl.context
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+
+
+@pytest.mark.parametrize("d,g", [(64, 1), (64, 2), (64, 4), (64, 8), (128, 1), (128, 2), (128, 4), (128, 8)])
+def test_decode_matches_oracle(d, g):
+    wl = _small(head_dim=d, n_q_heads=4 * g, n_kv_heads=4, context=4 + 32 * 9 + 32 + 21)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    cache, st, (k, v, f) = _build(wl, kb, vb)
+    q, _, _ = workloads.step_inputs(wl, 1, f, "cuda")
+    ws = cache.make_workspace(n_splits=16)
+    for layer in range(wl.n_layers):
+        exp = oracle_decode(wl, st, to_f32(q[0]).astype(np.float64), [(layer, b) for b in range(wl.batch)])
+        for splits in [1, 2, 5, 9, 0]:
+            out = cache.rq_decode_attention(layer, q[0, layer].contiguous(), n_splits=splits, workspace=ws)
+            got = out.cpu().numpy()
+            for b in range(wl.batch):
+                assert_close(got[b], exp[(layer, b)], f"layer {layer} b {b} splits {splits}")
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+
+
+def test_decode_all_layers_call():
+    wl = _small(n_layers=3, context=4 + 32 * 5 + 32 + 3)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    cache, st, (k, v, f) = _build(wl, kb, vb)
+    q, _, _ = workloads.step_inputs(wl, 1, f, "cuda")
+    out = cache.rq_decode_attention(-1, q[0].contiguous(), n_splits=3)
+    exp = oracle_decode(wl, st, to_f32(q[0]).astype(np.float64),
+                        [(l, b) for l in range(wl.n_layers) for b in range(wl.batch)])
+    got = out.cpu().numpy()
+    for (l, b), e in exp.items():
+        assert_close(got[l, b], e, f"layer {l} b {b}")
+
+
+@pytest.mark.parametrize("T", [0, 1, 3, 4, 20, 36, 67, 68, 69, 100])
+def test_short_caches(T):
+    # T < S, T < S + R (no tiles), exactly one tile, ragged windows
+    wl = _small(n_layers=1, batch=1, context=T)
+    kb, vb = _bits_grid(1, wl.n_kv_heads)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, 200)
+    cache.rq_quantize_kv(k, v)
+    st = oracle_streams(wl, kb, vb, to_f32(k), to_f32(v), all_streams(wl))
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    q, _, _ = workloads.step_inputs(wl, 1, f, "cuda")
+    out = cache.rq_decode_attention(0, q[0, 0].contiguous()).cpu().numpy()
+    exp = oracle_decode(wl, st, to_f32(q[0]).astype(np.float64), [(0, 0)])[(0, 0)]
+    if T == 0:
+        assert np.all(out == 0)
+    else:
+        assert_close(out[0], exp, f"T={T}")
+
+
+@pytest.mark.parametrize("S,R", [(4, 32), (0, 16), (2, 0), (6, 40)])
+def test_append_across_flushes(S, R):
+    wl = _small(n_layers=2, batch=2, n_sink=S, n_recent=R, context=S + R + 32 * 2 + 5)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    steps = 75
+    cache, st, (k, v, f) = _build(wl, kb, vb, extra=steps)
+    q, kn, vn = workloads.step_inputs(wl, steps, f, "cuda")
+    knp, vnp, qnp = to_f32(kn), to_f32(vn), to_f32(q).astype(np.float64)
+    ws = cache.make_workspace()
+    flushes = 0
+    for t in range(steps):
+        layer_mode = t % 3 == 0  # alternate all-layers and per-layer appends
+        if layer_mode:
+            cache.rq_append_token(-1, kn[t].contiguous(), vn[t].contiguous())
+        else:
+            for l in range(wl.n_layers):
+                cache.rq_append_token(l, kn[t, l].contiguous(), vn[t, l].contiguous())
+        for (l, b, h), s in st.items():
+            flushes += s.append(knp[t, l, b, h], vnp[t, l, b, h])
+        if t in (0, 3, 30, 31, 32, 33, 50, steps - 1):
+            out = cache.rq_decode_attention(-1, q[t].contiguous(), workspace=ws).cpu().numpy()
+            exp = oracle_decode(wl, st, qnp[t], [(l, b) for l in range(wl.n_layers) for b in range(wl.batch)])
+            for (l, b), e in exp.items():
+                assert_close(out[l, b], e, f"step {t} layer {l} b {b}")
+    assert flushes > 0
+    assert cache.length(0) == wl.context + steps
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+
+
+def test_append_from_empty_fills_sink_then_ring():
+    wl = _small(n_layers=1, batch=1, context=0)
+    kb, vb = _bits_grid(1, wl.n_kv_heads)
+    steps = 4 + 32 + 32 + 7
+    k, v, f = workloads.kv_inputs(wl, "cuda", n_tokens=0)
+    cache = make_cache(wl, kb, vb, steps)
+    cache.rq_quantize_kv(k, v)
+    q, kn, vn = workloads.step_inputs(wl, steps, f, "cuda")
+    st = {(0, 0, h): ca.StreamCache(wl.head_dim, int(kb[0, h]), int(vb[0, h]), wl.n_sink, wl.n_recent)
+          for h in range(wl.n_kv_heads)}
+    knp, vnp = to_f32(kn), to_f32(vn)
+    for t in range(steps):
+        cache.rq_append_token(0, kn[t, 0].contiguous(), vn[t, 0].contiguous())
+        for (l, b, h), s in st.items():
+            s.append(knp[t, l, b, h], vnp[t, l, b, h])
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    out = cache.rq_decode_attention(0, q[-1, 0].contiguous()).cpu().numpy()
+    exp = oracle_decode(wl, st, to_f32(q[-1]).astype(np.float64), [(0, 0)])[(0, 0)]
+    assert_close(out[0], exp)
+    # capacity is checked on the host
+    from quantized_decode_attention_head_b200._lib import RQError
+
+    with pytest.raises(RQError) as e:
+        cache.rq_append_token(0, kn[0, 0].contiguous(), vn[0, 0].contiguous())
+    assert e.value.status == "RQ_ERR_CAPACITY"
+
+
+def test_workspace_too_small_is_rejected():
+    wl = _small(n_layers=1)
+    kb, vb = _bits_grid(1, wl.n_kv_heads)
+    cache, st, (k, v, f) = _build(wl, kb, vb)
+    q, _, _ = workloads.step_inputs(wl, 1, f, "cuda")
+    from quantized_decode_attention_head_b200._lib import RQError
+
+    ws = torch.zeros(512, dtype=torch.uint8, device="cuda")
+    with pytest.raises(RQError) as e:
+        cache.rq_decode_attention(0, q[0, 0].contiguous(), n_splits=4, workspace=ws)
+    assert e.value.status == "RQ_ERR_WORKSPACE"
+
+
+def test_tiny_workload_end_to_end():
+    wl = workloads.CONFIGS["tiny"]
+    (kb, vb), (okb, ovb) = workload_bits(wl)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, wl.context + wl.decode_steps)
+    cache.rq_quantize_kv(k, v)
+    st = oracle_streams(wl, okb, ovb, to_f32(k), to_f32(v), all_streams(wl))
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    q, kn, vn = workloads.step_inputs(wl, 1, f, "cuda")
+    cache.rq_append_token(0, kn[0, 0].contiguous(), vn[0, 0].contiguous())
+    for (l, b, h), s in st.items():
+        s.append(to_f32(kn[0, l, b, h]), to_f32(vn[0, l, b, h]))
+    out = cache.rq_decode_attention(0, q[0, 0].contiguous()).cpu().numpy()
+    exp = oracle_decode(wl, st, to_f32(q[0]).astype(np.float64), [(0, 0)])[(0, 0)]
+    assert_close(out[0], exp, "tiny")

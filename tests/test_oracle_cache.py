@@ -79,3 +79,23 @@ def test_ring_slots_never_collide_with_live_tokens():
         s, tq, r = ca.split_lengths(T, S, R)
         slots = [ca.ring_slot(p, S, R) for p in range(S + tq, T)]
         assert len(set(slots)) == len(slots)
+
+
+@pytest.mark.parametrize("kb,vb,d", [(2, 2, 128), (3, 8, 64), (4, 3, 128), (8, 4, 64)])
+def test_batched_records_equal_single_tile_records(kb, vb, d):
+    rng = np.random.default_rng(kb * 100 + vb + d)
+    T = 4 + 32 * 5 + 32 + 9
+    k = qz.bf16_bits_to_f32(rng.integers(0x3C00, 0x4100, size=(T, d), dtype=np.uint16))
+    v = qz.bf16_bits_to_f32(rng.integers(0xBC00, 0xC100, size=(T, d), dtype=np.uint16))
+    st = ca.StreamCache(d, kb, vb, 4, 32)
+    st.prefill(k, v)
+    recs = st.records()
+    assert recs.shape == (st.n_tiles, qz.record_bytes(kb, vb, d)) and st.n_tiles == 5
+    for i in range(st.n_tiles):
+        assert np.array_equal(recs[i], st.record(i))
+        # and each record decodes back to the tile's own quantization
+        back = qz.unpack_record(recs[i], kb, vb, d)
+        a = 4 + 32 * i
+        ref = qz.quantize_tile(k[a : a + 32], v[a : a + 32], kb, vb)
+        for key in ref:
+            assert np.array_equal(back[key], ref[key]), key
