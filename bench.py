@@ -256,7 +256,9 @@ def run_gpu(args):
     kb = alloc["b_int"].reshape(wl.n_layers, wl.n_kv_heads)
 
     total_steps = args.warmup + args.steps
-    steps_per_copy = (total_steps + NC - 1) // NC + 1
+    e2e_steps = args.steps
+    j0 = (total_steps + NC - 1) // NC  # first per-copy step index of the e2e loop
+    steps_per_copy = j0 + (e2e_steps + NC - 1) // NC + 1
     max_tokens = wl.context + steps_per_copy + 32
     caches, step_in = [], []
     qbytes, qtimes = 0, []
@@ -337,7 +339,6 @@ def run_gpu(args):
     dk = [torch.empty_like(step_in[c][1][0, 0]) for c in range(NC)]
     dv = [torch.empty_like(step_in[c][2][0, 0]) for c in range(NC)]
     host_out = torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=torch.float32).pin_memory()
-    e2e_steps = min(args.steps, max(1, (steps_per_copy - (total_steps + NC - 1) // NC - 1) * NC))
     base_len = [caches[c].length(0) for c in range(NC)]
     e2e_bytes = 0
     for i in range(e2e_steps):
@@ -347,7 +348,6 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    j0 = (total_steps + NC - 1) // NC
     s2.record(stream)
     for i in range(e2e_steps):
         c = i % NC

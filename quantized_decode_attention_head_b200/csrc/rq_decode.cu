@@ -32,8 +32,7 @@ namespace rq {
 namespace {
 
 constexpr int NW = kDecodeConsumerWarps;
-constexpr int kStages = 8;  // multiple of NW: stage s is always consumed by warp s % NW
-static_assert(kStages % NW == 0, "stage ownership");
+constexpr int kMaxStages = 8;  // per-warp ring depth limit
 
 template <int D, int G>
 struct Cfg {
@@ -45,11 +44,12 @@ struct Cfg {
 
 template <int D, int G>
 struct WarpState {
-  uint32_t qb[D / 16][2];          // q B-fragments (fp16, scaled by 2^kq)
-  float kscale;                    // 2^(24 - kq)
-  float qsum[Cfg<D, G>::NSET][2];  // sum of q over the thread's (group, head) columns
-  float m[2], l[2];                // running max (log2 units) / sum per column parity
-  float o[D / 16][4];              // P.V accumulators, out^T fragment layout
+  static constexpr int KE = G == 1 ? 2 : 1;  // column parities with distinct K groups
+  uint32_t qb[D / 16][2];                    // q B-fragments (fp16, scaled by 2^kq)
+  float ksf[2][2][Cfg<D, G>::NSET][KE];      // 2^(24 - kq - b*class) * softmax scale * log2(e)
+  float qsum[Cfg<D, G>::NSET][2];            // softmax-scaled sum of q over (group, head) columns
+  float m[2], l[2];                          // running max (log2 units) / sum per column parity
+  float o[D / 16][4];                        // P.V accumulators (x 2^-24), out^T fragment layout
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -63,9 +63,12 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int D, int G>
-__device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, int lane) {
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
+template <int D, int G, int KB>
+__device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, float scale_log2, int lane) {
   using C = Cfg<D, G>;
+  constexpr int WK = words_per_lane(KB, D);
   const int gid = lane >> 2, tig = lane & 3;
   const int bh = gid % G;          // head of B column n = gid
   const int bgl = gid / G;         // group slot of B column n = gid
@@ -85,8 +88,7 @@ __device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, int lane) {
     kq = 15 - e;
     kq = kq > 100 ? 100 : (kq < -100 ? -100 : kq);
   }
-  const float up = __int_as_float((kq + 127) << 23);
-  st.kscale = __int_as_float((24 - kq + 127) << 23);
+  const float up = pow2i(kq);
 #pragma unroll
   for (int kb = 0; kb < D / 16; ++kb) {
     const bool valid = ((kb / 2) % C::GPS) == bgl;
@@ -114,7 +116,16 @@ __device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, int lane) {
           for (int k = 0; k < 4; ++k) acc += bf16_bits_to_float(w[k] & 0xFFFFu) + bf16_bits_to_float(w[k] >> 16);
         }
       }
-      st.qsum[s][e] = acc;
+      st.qsum[s][e] = acc * scale_log2;
+#pragma unroll
+      for (int mb = 0; mb < 2; ++mb)
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          if (e < WarpState<D, G>::KE) {
+            const int q = (mb * 2 + rr) * C::NG + (grp < C::NG ? grp : 0);
+            st.ksf[mb][rr][s][e] = pow2i(24 - kq - KB * quad_class(KB, WK, q)) * scale_log2;
+          }
+        }
     }
   st.m[0] = st.m[1] = -INFINITY;
   st.l[0] = st.l[1] = 0.0f;
@@ -138,11 +149,14 @@ __device__ __forceinline__ void load_words(uint32_t (&w)[W], const uint8_t* blob
   for (int k = 4 * (W / 4); k < W; ++k) w[k] = *reinterpret_cast<const uint32_t*>(blob + word_offset(W, lane, k));
 }
 
-// q.K^T of one tile -> logits x[mb][rr][e] (log2 units) for tokens
-// 16mb + 8rr + gid and heads (2 tig + e) % G.
+__device__ __forceinline__ float half_lo_to_float(uint32_t m) {
+  return __half2float(__ushort_as_half((unsigned short)(m & 0xFFFFu)));
+}
+
+// q.K^T of one tile -> logits x[mb][rr][e] (log2 units, softmax scale applied)
+// for tokens 16mb + 8rr + gid and heads (2 tig + e) % G.
 template <int D, int G, int KB>
-__device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G>& st, float scale_log2,
-                                        float (&x)[2][2][2], int lane) {
+__device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G>& st, float (&x)[2][2][2], int lane) {
   using C = Cfg<D, G>;
   constexpr int W = words_per_lane(KB, D);
   const int gid = lane >> 2, tig = lane & 3;
@@ -163,7 +177,7 @@ __device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int idx = k_pair_index(D, mb, kb, r);
-        a[r] = extract_pair<KB>(kw[slot_word(KB, W, idx)], slot_pos(KB, W, idx));
+        a[r] = extract_pair<KB>(kw, slot_word(KB, W, idx), slot_pos(KB, W, idx));
       }
       mma_f16(acc[(kb / 2) / C::GPS][mb], a, st.qb[kb][0], st.qb[kb][1]);
     }
@@ -176,7 +190,8 @@ __device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G
 #pragma unroll
   for (int s = 0; s < C::NSET; ++s)
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
+    for (int e = 0; e < WarpState<D, G>::KE; ++e) {
+      // for G >= 2 both column parities of a thread share one K group
       const int grp = s * C::GPS + (2 * tig + e) / G;
       if (grp < C::NG) {
         const uint4 mv = *reinterpret_cast<const uint4*>(kmeta + grp * 32 + gid * 4);
@@ -186,9 +201,14 @@ __device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G
 #pragma unroll
           for (int rr = 0; rr < 2; ++rr) {
             const uint32_t m = mw[mb * 2 + rr];
-            const float sk = __half2float(__ushort_as_half((unsigned short)(m & 0xFFFFu))) * st.kscale;
+            const float sk = half_lo_to_float(m) * st.ksf[mb][rr][s][e];
             const float z = __uint_as_float(m & 0xFFFF0000u);
-            sc[mb][rr][e] = fmaf(sk, acc[s][mb][rr * 2 + e], fmaf(z, st.qsum[s][e], sc[mb][rr][e]));
+            if (G == 1) {
+              sc[mb][rr][e] = fmaf(sk, acc[s][mb][rr * 2 + e], fmaf(z, st.qsum[s][e], sc[mb][rr][e]));
+            } else {
+              sc[mb][rr][0] = fmaf(sk, acc[s][mb][rr * 2], fmaf(z, st.qsum[s][0], sc[mb][rr][0]));
+              sc[mb][rr][1] = fmaf(sk, acc[s][mb][rr * 2 + 1], fmaf(z, st.qsum[s][1], sc[mb][rr][1]));
+            }
           }
       }
     }
@@ -212,8 +232,8 @@ __device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G
         v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
         v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
       }
-      x[mb][rr][0] = v0 * scale_log2;
-      x[mb][rr][1] = v1 * scale_log2;
+      x[mb][rr][0] = v0;
+      x[mb][rr][1] = v1;
     }
 }
 
@@ -267,17 +287,18 @@ __device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int idx = v_pair_index(mb, kb, r);
-        a[r] = extract_pair<VB>(vw[slot_word(VB, W, idx)], slot_pos(VB, W, idx));
+        a[r] = extract_pair<VB>(vw, slot_word(VB, W, idx), slot_pos(VB, W, idx));
       }
       mma_f16(acc[mb], a, pb[kb][0], pb[kb][1]);
     }
   }
+  // sum_t p_t * 2^-24 per column: A = the fp16 subnormal 2^-24, so every
+  // accumulator below carries the same 2^-24 as the unpacked codes
   float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  const uint32_t ones[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};
-  mma_f16(ps, ones, pb[0][0], pb[0][1]);
-  mma_f16(ps, ones, pb[1][0], pb[1][1]);
+  const uint32_t tiny[4] = {0x00010001u, 0x00010001u, 0x00010001u, 0x00010001u};
+  mma_f16(ps, tiny, pb[0][0], pb[0][1]);
+  mma_f16(ps, tiny, pb[1][0], pb[1][1]);
   const uint32_t* vmeta = reinterpret_cast<const uint32_t*>(vrec + blob_bytes(VB, D)) + gid * (D / 8);
-  constexpr float k2p24 = 16777216.0f;
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
     const uint4 mv = *reinterpret_cast<const uint4*>(vmeta + 4 * c);
@@ -285,7 +306,9 @@ __device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int mb = 2 * c + j / 2, rr = j % 2;
-      const float sv = __half2float(__ushort_as_half((unsigned short)(mw[j] & 0xFFFFu))) * k2p24;
+      const int cls = quad_class(VB, W, mb * 2 + rr);
+      float sv = half_lo_to_float(mw[j]);
+      if (cls) sv *= 1.0f / (float)(1 << (VB * cls));
       const float z = __uint_as_float(mw[j] & 0xFFFF0000u);
 #pragma unroll
       for (int e = 0; e < 2; ++e)
@@ -297,23 +320,72 @@ __device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st
 }
 
 template <int D, int G, int KB, int VB>
-__device__ __forceinline__ void process_tile(const uint8_t* rec, WarpState<D, G>& st, float scale_log2, int lane) {
+__device__ __forceinline__ void process_tile(const uint8_t* rec, WarpState<D, G>& st, int lane) {
   float x[2][2][2];
-  qk_tile<D, G, KB>(rec, st, scale_log2, x, lane);
+  qk_tile<D, G, KB>(rec, st, x, lane);
   uint32_t pb[2][2];
   softmax_tile<D, G>(st, x, pb);
   pv_tile<D, G, VB>(rec + blob_bytes(KB, D) + 4 * D, st, pb, lane);
 }
 
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
+  *abort_flag = 1;
+  atomicCAS(status, 0, kDeviceTimeout);
+}
+
+// Consumer warp w owns tiles w, w + NW, w + 2 NW, ... of the CTA's range and a
+// private ring of `stages` shared-memory slots.  Lane 0 streams the warp's
+// own tile records into the ring with 1-D bulk copies (TMA) and re-arms a
+// slot as soon as the warp has read it, so the warp never waits on another
+// warp and every warp keeps `stages` records in flight.
+template <int D, int G, int KB, int VB>
+__device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log2, uint8_t* ring, int stages,
+                        int stage_bytes, uint64_t* bars, const uint8_t* src, int rec, int n_my, int warp, int lane,
+                        volatile int* abort_flag, int* status) {
+  const int n_w = n_my > warp ? (n_my - warp + NW - 1) / NW : 0;
+  if (lane == 0) {
+    for (int j = 0; j < stages && j < n_w; ++j) {
+      mbar_arrive_expect_tx(&bars[j], (uint32_t)rec);
+      bulk_g2s(ring + (size_t)j * stage_bytes, src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec, &bars[j]);
+    }
+  }
+  setup_query<D, G, KB>(st, qh, scale_log2, lane);
+  int j = 0;
+  for (; j < n_w; ++j) {
+    const int s = j % stages;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (j / stages) & 1));
+    if (!ok) {
+      if (lane == 0) raise_abort(abort_flag, status);
+      break;
+    }
+    process_tile<D, G, KB, VB>(ring + (size_t)s * stage_bytes, st, lane);
+    __syncwarp();
+    if (lane == 0 && j + stages < n_w) {
+      fence_proxy_async_smem();  // the generic-proxy reads of this slot precede the async refill
+      mbar_arrive_expect_tx(&bars[s], (uint32_t)rec);
+      bulk_g2s(ring + (size_t)s * stage_bytes, src + (int64_t)(warp + (j + stages) * NW) * rec, (uint32_t)rec,
+               &bars[s]);
+    }
+  }
+  if (j < n_w && lane == 0) {  // aborted: let the copies in flight land before the CTA exits
+    for (int k = j; k < n_w && k < j + stages; ++k) (void)mbar_wait_bounded(&bars[k % stages], (k / stages) & 1);
+  }
+}
+
 template <int D, int G>
-__device__ __forceinline__ void process_tile_dispatch(int kb, int vb, const uint8_t* rec, WarpState<D, G>& st,
-                                                      float sl2, int lane) {
-#define RQ_V(KBV)                                                         \
-  switch (vb) {                                                           \
-    case 2: process_tile<D, G, KBV, 2>(rec, st, sl2, lane); break;        \
-    case 3: process_tile<D, G, KBV, 3>(rec, st, sl2, lane); break;        \
-    case 4: process_tile<D, G, KBV, 4>(rec, st, sl2, lane); break;        \
-    default: process_tile<D, G, KBV, 8>(rec, st, sl2, lane); break;       \
+__device__ __forceinline__ void consume_dispatch(int kb, int vb, WarpState<D, G>& st, const uint16_t* qh,
+                                                 float scale_log2, uint8_t* ring, int stages, int stage_bytes,
+                                                 uint64_t* bars, const uint8_t* src, int rec, int n_my, int warp,
+                                                 int lane, volatile int* abort_flag, int* status) {
+#define RQ_C(KBV, VBV)                                                                                           \
+  consume<D, G, KBV, VBV>(st, qh, scale_log2, ring, stages, stage_bytes, bars, src, rec, n_my, warp, lane, abort_flag, \
+                          status)
+#define RQ_V(KBV)                  \
+  switch (vb) {                    \
+    case 2: RQ_C(KBV, 2); break;   \
+    case 3: RQ_C(KBV, 3); break;   \
+    case 4: RQ_C(KBV, 4); break;   \
+    default: RQ_C(KBV, 8); break;  \
   }
   switch (kb) {
     case 2: RQ_V(2) break;
@@ -322,6 +394,7 @@ __device__ __forceinline__ void process_tile_dispatch(int kb, int vb, const uint
     default: RQ_V(8) break;
   }
 #undef RQ_V
+#undef RQ_C
 }
 
 // Canonical partial of one warp in shared memory: o[G][D], m[G], l[G].
@@ -335,84 +408,133 @@ __device__ void dump_tile_state(const WarpState<D, G>& st, float* slot, int lane
 #pragma unroll
       for (int mb = 0; mb < D / 16; ++mb)
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) slot[n * D + 16 * mb + 8 * rr + gid] = st.o[mb][rr * 2 + e];
+        for (int rr = 0; rr < 2; ++rr) slot[n * D + 16 * mb + 8 * rr + gid] = st.o[mb][rr * 2 + e] * 16777216.0f;
       if (gid == 0) {
         slot[G * D + n] = st.m[e];
-        slot[G * D + G + n] = st.l[e];
+        slot[G * D + G + n] = st.l[e] * 16777216.0f;
       }
     }
   }
 }
 
-// bf16 sink + recent window on CUDA cores; lane = token for q.k, lane = channel for p.v.
-template <int D, int G>
-__device__ void window_warp(const DecodeArgs& a, const uint8_t* win, const float* qs, float* slot, int warp, int lane) {
+// bf16 sink + recent window on CUDA cores.  Warp w takes the window's
+// 32-token chunks w, w + 4, ...: lane 0 stages the chunk's K and V rows in
+// the warp's own shared buffer with at most six 1-D bulk copies (the rows of
+// a chunk form at most three contiguous runs: sink, ring, ring after wrap),
+// then the warp scores all G heads (lane = token; K row words read in a
+// lane-rotated order so the 32 rows hit 32 banks) and accumulates P.V
+// (lane = channel).  Only warp-level synchronisation inside the loop.
+constexpr int kWinChunk = 32;
+
+template <int D>
+__device__ __forceinline__ int window_issue_chunk(const DecodeArgs& a, const uint8_t* win, uint32_t* kbuf,
+                                                  uint32_t* vbuf, uint64_t* bar, int j0, int cnt) {
   const int S = a.g.S, ring = a.g.R + kTile;
   const int n_sink = a.T < S ? a.T : S;
+  mbar_arrive_expect_tx(bar, (uint32_t)(cnt * D * 2 * 2));
+  int t = 0;
+  while (t < cnt) {
+    const int j = j0 + t;
+    size_t row;  // row index inside the K half of the window block
+    int run;
+    if (j < n_sink) {
+      row = j;
+      run = min(cnt - t, n_sink - j);
+    } else {
+      const int slot = (a.Tq + (j - n_sink)) % ring;
+      row = (size_t)2 * S + slot;
+      run = min(cnt - t, ring - slot);
+    }
+    const size_t v_off = (j < n_sink) ? (size_t)S : (size_t)ring;  // V rows follow the K rows of their block
+    bulk_g2s(kbuf + (size_t)t * (D / 2), win + row * D * 2, (uint32_t)(run * D * 2), bar);
+    bulk_g2s(vbuf + (size_t)t * (D / 2), win + (row + v_off) * D * 2, (uint32_t)(run * D * 2), bar);
+    t += run;
+  }
+  return 0;
+}
+
+template <int D, int G>
+__device__ void window_warp(const DecodeArgs& a, const uint8_t* win, const float2* q2, uint32_t* kbuf,
+                            uint32_t* vbuf, uint64_t* bar, float* slot, int warp, int lane,
+                            volatile int* abort_flag) {
+  constexpr int RW = D / 2;  // words per bf16 row
+  const int S = a.g.S;
+  const int n_sink = a.T < S ? a.T : S;
   const int n_tok = n_sink + (a.T - n_sink - a.Tq);
+  const int n_chunks = (n_tok + kWinChunk - 1) / kWinChunk;
   float m[G], l[G], o[G][D / 32];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.0f;
 #pragma unroll
-    for (int j = 0; j < D / 32; ++j) o[h][j] = 0.0f;
+    for (int c = 0; c < D / 32; ++c) o[h][c] = 0.0f;
   }
-  auto row_of = [&](int j, int kv) -> const uint16_t* {
-    if (j < n_sink) return reinterpret_cast<const uint16_t*>(win + ((size_t)kv * S + j) * D * 2);
-    const int slot_i = (a.Tq + (j - n_sink)) % ring;  // position S + Tq + (j - n_sink)
-    return reinterpret_cast<const uint16_t*>(win + ((size_t)2 * S + (size_t)kv * ring + slot_i) * D * 2);
-  };
-  for (int c0 = warp * 32; c0 < n_tok; c0 += NW * 32) {
-    const int j = c0 + lane;
-    const bool valid = j < n_tok;
+  int k = 0;
+  for (int c = warp; c < n_chunks; c += NW, ++k) {
+    const int j0 = c * kWinChunk;
+    const int cnt = min(kWinChunk, n_tok - j0);
+    if (k > 0) __syncwarp();  // the previous chunk is fully read
+    if (lane == 0) {
+      if (k > 0) fence_proxy_async_smem();
+      window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt);
+    }
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar, k & 1))) {
+      if (lane == 0) {
+        raise_abort(abort_flag, a.status);
+        (void)mbar_wait_bounded(bar, k & 1);  // let this warp's copies land before the CTA exits
+      }
+      return;
+    }
+    // scores of token `lane` for all heads
     float sc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) sc[h] = 0.0f;
-    if (valid) {
-      const uint4* kr = reinterpret_cast<const uint4*>(row_of(j, 0));
+    if (lane < cnt) {
 #pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 u = __ldg(kr + c);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      for (int w = 0; w < RW; ++w) {
+        const int wr = (w + lane) & (RW - 1);
+        const uint32_t kk = kbuf[lane * RW + wr];
+        const float k0 = bf16_bits_to_float(kk & 0xFFFFu), k1 = bf16_bits_to_float(kk >> 16);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float k0 = bf16_bits_to_float(w[k] & 0xFFFFu), k1 = bf16_bits_to_float(w[k] >> 16);
-#pragma unroll
-          for (int h = 0; h < G; ++h) sc[h] = fmaf(qs[h * D + 8 * c + 2 * k], k0, fmaf(qs[h * D + 8 * c + 2 * k + 1], k1, sc[h]));
+        for (int h = 0; h < G; ++h) {
+          const float2 qq = q2[h * RW + wr];
+          sc[h] = fmaf(qq.x, k0, fmaf(qq.y, k1, sc[h]));
         }
       }
     }
     float p[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float xv = valid ? sc[h] * a.scale_log2 : -INFINITY;
-      const float mn = fmaxf(m[h], warp_max(xv));
+      const float x = lane < cnt ? sc[h] * a.scale_log2 : -INFINITY;
+      const float mn = fmaxf(m[h], warp_max(x));
       const float alpha = ex2(m[h] - mn);
-      p[h] = valid ? ex2(xv - mn) : 0.0f;
+      p[h] = ex2(x - mn);
       l[h] = l[h] * alpha + warp_sum(p[h]);
       m[h] = mn;
 #pragma unroll
-      for (int jj = 0; jj < D / 32; ++jj) o[h][jj] *= alpha;
+      for (int cc = 0; cc < D / 32; ++cc) o[h][cc] *= alpha;
     }
-    const int cnt = min(32, n_tok - c0);
     for (int t = 0; t < cnt; ++t) {
-      const uint16_t* vr = row_of(c0 + t, 1);
-      float vv[D / 32];
+      float v[D / 32];
 #pragma unroll
-      for (int jj = 0; jj < D / 32; ++jj) vv[jj] = bf16_bits_to_float(__ldg(vr + lane + 32 * jj));
+      for (int cc = 0; cc < D / 32; ++cc) {
+        const int d = lane + 32 * cc;
+        const uint32_t vv = vbuf[t * RW + d / 2];
+        v[cc] = (d & 1) ? bf16_bits_to_float(vv >> 16) : bf16_bits_to_float(vv & 0xFFFFu);
+      }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float pt = __shfl_sync(0xffffffffu, p[h], t);
 #pragma unroll
-        for (int jj = 0; jj < D / 32; ++jj) o[h][jj] = fmaf(pt, vv[jj], o[h][jj]);
+        for (int cc = 0; cc < D / 32; ++cc) o[h][cc] = fmaf(pt, v[cc], o[h][cc]);
       }
     }
   }
 #pragma unroll
   for (int h = 0; h < G; ++h) {
 #pragma unroll
-    for (int jj = 0; jj < D / 32; ++jj) slot[h * D + lane + 32 * jj] = o[h][jj];
+    for (int cc = 0; cc < D / 32; ++cc) slot[h * D + lane + 32 * cc] = o[h][cc];
     if (lane == 0) {
       slot[G * D + h] = m[h];
       slot[G * D + G + h] = l[h];
@@ -420,16 +542,11 @@ __device__ void window_warp(const DecodeArgs& a, const uint8_t* win, const float
   }
 }
 
-__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
-  *abort_flag = 1;
-  atomicCAS(status, 0, kDeviceTimeout);
-}
-
 template <int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a) {
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ uint64_t bars[NW * kMaxStages];
   __shared__ volatile int abort_flag;
   __shared__ int is_last;
 
@@ -444,11 +561,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
 
   if (tid == 0) {
     abort_flag = 0;
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
+    for (int s = 0; s < NW * kMaxStages; ++s) mbar_init(&bars[s], 1);
     mbar_fence_init();
   }
   __syncthreads();
@@ -461,51 +574,23 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
     const int n_my = t1 - t0;
     const int rec = hd.rec_bytes;
     const uint8_t* src = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)t0 * rec;
-    if (warp == NW) {
-      if (lane == 0) {
-        int last_issue[kStages];
-#pragma unroll
-        for (int s = 0; s < kStages; ++s) last_issue[s] = -1;
-        for (int i = 0; i < n_my; ++i) {
-          const int s = i % kStages;
-          if (i >= kStages && !mbar_wait_bounded(&empty_bar[s], ((i / kStages) - 1) & 1)) {
-            raise_abort(&abort_flag, a.status);
-            break;
-          }
-          if (abort_flag) break;
-          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)rec);
-          bulk_g2s(smem + (size_t)s * a.stage_bytes, src + (int64_t)i * rec, (uint32_t)rec, &full_bar[s]);
-          last_issue[s] = i;
-        }
-        if (abort_flag) {  // let copies in flight land before the CTA exits
-          for (int s = 0; s < kStages; ++s)
-            if (last_issue[s] >= 0) (void)mbar_wait_bounded(&full_bar[s], (last_issue[s] / kStages) & 1);
-        }
-      }
-    } else {
-      setup_query<D, G>(st, qh, lane);
-      for (int i = warp; i < n_my; i += NW) {
-        const int s = i % kStages;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[s], (i / kStages) & 1));
-        if (!ok) {
-          if (lane == 0) raise_abort(&abort_flag, a.status);
-          break;
-        }
-        process_tile_dispatch<D, G>(hd.k_bits, hd.v_bits, smem + (size_t)s * a.stage_bytes, st, a.scale_log2, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[s]);
-        if (abort_flag) break;
-      }
-    }
+    if (warp < NW)
+      consume_dispatch<D, G>(hd.k_bits, hd.v_bits, st, qh, a.scale_log2,
+                             smem + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
+                             bars + warp * kMaxStages, src, rec, n_my, warp, lane, &abort_flag, a.status);
   } else {
-    // bf16 sink + recent window on CUDA cores
-    float* qs = merge + NW * C::PART;
-    for (int i = tid; i < G * D; i += blockDim.x) qs[i] = bf16_bits_to_float(qh[i]);
-    __syncthreads();
-    if (warp < NW) {
-      const uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
-      window_warp<D, G>(a, win, qs, merge + warp * C::PART, warp, lane);
+    // bf16 sink + recent window: q (fp32 pairs) after the merge slots, then
+    // one K and one V chunk buffer per warp
+    const uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
+    float2* q2 = reinterpret_cast<float2*>(merge + NW * C::PART);
+    for (int i = tid; i < G * D / 2; i += blockDim.x) {
+      const uint32_t w = reinterpret_cast<const uint32_t*>(qh)[i];
+      q2[i] = make_float2(bf16_bits_to_float(w & 0xFFFFu), bf16_bits_to_float(w >> 16));
     }
+    __syncthreads();
+    uint32_t* kbuf = reinterpret_cast<uint32_t*>(q2 + G * D / 2) + (size_t)warp * 2 * kWinChunk * (D / 2);
+    window_warp<D, G>(a, win, q2, kbuf, kbuf + kWinChunk * (D / 2), &bars[warp * kMaxStages], merge + warp * C::PART,
+                      warp, lane, &abort_flag);
   }
   __syncthreads();  // every stage read has completed; merge may now alias the stages
   if (tiles_item && warp < NW && !abort_flag) dump_tile_state<D, G>(st, merge + warp * C::PART, lane);
@@ -560,11 +645,34 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
   }
   __syncthreads();
   float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  for (int idx = tid; idx < G * D; idx += blockDim.x) {
-    const int hh = idx / D;
-    float O = 0.0f;
-    for (int i = 0; i < NI; ++i) O = fmaf(__ldcg(base + (size_t)i * C::PART + idx), wts[i * G + hh], O);
-    outp[idx] = O * wts[NI * G + hh];
+  // each thread owns OPT outputs; U items per round -> OPT * U loads in flight
+  constexpr int OPT = (G * D + kDecodeThreads - 1) / kDecodeThreads;
+  constexpr int U = OPT >= 64 ? 1 : 64 / OPT;
+  float acc[OPT];
+#pragma unroll
+  for (int k = 0; k < OPT; ++k) acc[k] = 0.0f;
+  for (int i0 = 0; i0 < NI; i0 += U) {
+    float v[OPT][U];
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+      const int idx = tid + k * kDecodeThreads;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        v[k][u] = (idx < G * D && i0 + u < NI) ? __ldcg(base + (size_t)(i0 + u) * C::PART + idx) : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+      const int idx = tid + k * kDecodeThreads;
+      const int hh = idx < G * D ? idx / D : 0;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + u < NI) acc[k] = fmaf(v[k][u], wts[(i0 + u) * G + hh], acc[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < OPT; ++k) {
+    const int idx = tid + k * kDecodeThreads;
+    if (idx < G * D) outp[idx] = acc[k] * wts[NI * G + idx / D];
   }
   if (tid == 0) a.counters[srel] = 0u;
 }
@@ -581,14 +689,34 @@ cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
 
 }  // namespace
 
-int decode_smem_bytes(int n_items, int stage_bytes, int G, int D) {
+int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   const int part = G * D + 2 * G;
-  int merge = (NW * part + G * D) * 4;
+  // merge slots + window scratch (q, one K and one V chunk per warp)
+  int merge = (NW * part + G * D) * 4 + NW * 2 * kWinChunk * D * 2;
   const int wts = (n_items + 1) * G * 4;
   merge = merge > wts ? merge : wts;
-  const int ring = kStages * stage_bytes;
+  const int ring = NW * stages * stage_bytes;
   int need = ring > merge ? ring : merge;
   return (need + 127) / 128 * 128;
+}
+
+template <int D, int G>
+int occupancy_dg(int smem) {
+  if (cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<D, G>, kDecodeThreads, smem) != cudaSuccess)
+    return 1;
+  return n > 0 ? n : 1;
+}
+
+int decode_occupancy(int D, int G, int smem) {
+#define RQ_DG(DD, GG) \
+  if (D == DD && G == GG) return occupancy_dg<DD, GG>(smem);
+  RQ_DG(128, 1) RQ_DG(128, 2) RQ_DG(128, 4) RQ_DG(128, 8)
+  RQ_DG(64, 1) RQ_DG(64, 2) RQ_DG(64, 4) RQ_DG(64, 8)
+#undef RQ_DG
+  return 1;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int smem, cudaStream_t st) {

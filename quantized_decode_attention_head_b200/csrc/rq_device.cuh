@@ -38,12 +38,29 @@ __host__ __device__ constexpr int word_offset(int W, int lane, int w) {
                          : (W / 4) * 512 + ((w - 4 * (W / 4)) * 32 + lane) * 4;
 }
 
-// Pair of b-bit codes of slot p as an fp16x2 of subnormals c * 2^-24
-// (exact: the code bits become the fp16 mantissa, exponent field zero).
+// Class of a slot: how many b-bit steps its codes sit above the lowest
+// position from which they are read in place (fp16 mantissa = bits 0..9 of a
+// 16-bit half).  b=2: slots 0..4 in place, 5..7 after a 10-bit shift;
+// b=4: slots 0,1 in place, 2,3 after an 8-bit shift; b=3, 8: every slot is
+// shifted down to bit 0 (class 0).
+__host__ __device__ constexpr int slot_class(int b, int p) {
+  return b == 2 ? (p < 5 ? p : p - 5) : b == 4 ? (p & 1) : 0;
+}
+// Class shared by the four pairs of quad q of a blob with W words per lane.
+__host__ __device__ constexpr int quad_class(int b, int W, int q) { return slot_class(b, slot_pos(b, W, 4 * q)); }
+
+// Pair of b-bit codes of slot p of word w as an fp16x2 of subnormals
+// c * 2^(b*class - 24): the code bits become the fp16 mantissa with a zero
+// exponent field, so the values are exact and need no offset removal.  The
+// 2^(b*class) factor is undone by the per-quad scale.
 template <int B>
-__device__ __forceinline__ uint32_t extract_pair(uint32_t word, int p) {
+__device__ __forceinline__ uint32_t extract_pair(const uint32_t* words, int w, int p) {
   constexpr uint32_t m = (1u << B) - 1u;
-  return (word >> (B * p)) & (m | (m << 16));
+  constexpr uint32_t mm = m | (m << 16);
+  if (B == 2) return p < 5 ? (words[w] & (mm << (2 * p))) : ((words[w] >> 10) & (mm << (2 * (p - 5))));
+  if (B == 4) return p < 2 ? (words[w] & (mm << (4 * p))) : ((words[w] >> 8) & (mm << (4 * (p - 2))));
+  if (B == 8) return p == 0 ? (words[w] & mm) : ((words[w] >> 8) & mm);
+  return (words[w] >> (B * p)) & mm;
 }
 
 // ------------------------------------------------------------ tensor cores
@@ -115,6 +132,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 > 1000000000ull) return false;
   }
+}
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 // 1-D bulk copy global -> shared, completion counted on an mbarrier (bytes).
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

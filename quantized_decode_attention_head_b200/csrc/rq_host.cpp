@@ -89,16 +89,27 @@ bool layer_range(const rq_cache* c, int layer, int& l0, int& nl) {
   return true;
 }
 
-int auto_splits(const rq_cache* c, int streams, int n_tiles) {
+// Largest record among the heads of layers [l0, l0 + nl).
+int max_record(const rq_cache* c, int l0, int nl) {
+  int r = 16;
+  for (int l = l0; l < l0 + nl; ++l)
+    for (int h = 0; h < c->g.Hkv; ++h) r = c->desc[l * c->g.Hkv + h].rec_bytes > r ? c->desc[l * c->g.Hkv + h].rec_bytes : r;
+  return r;
+}
+
+// Tile splits per stream so that all work items of the call (splits + one
+// window item per stream) fill the resident CTA slots of the GPU once.
+int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes) {
   if (n_tiles <= 0) return 0;
-  const int target = c->sm_count * 4;  // about four resident CTAs per SM
-  int s = (target + streams - 1) / streams;
+  const int occ = rq::decode_occupancy(
+      c->g.D, c->g.G, rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes), stage_bytes, c->g.G, c->g.D));
+  const long slots = (long)occ * c->sm_count;
+  long s = slots / streams - 1;
   if (s < 1) s = 1;
-  // keep at least 8 tiles per split so a CTA's pipeline fills
-  const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;
+  const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;  // keep a CTA's pipeline busy
   if (s > max_by_work) s = max_by_work;
   if (s > n_tiles) s = n_tiles;
-  return s;
+  return (int)s;
 }
 
 rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
@@ -239,8 +250,9 @@ rq_status rq_decode_workspace_bytes(const rq_cache* c, int n_splits, size_t* byt
   const int streams_layer = c->g.B * c->g.Hkv;
   const int max_tiles = c->g.max_tiles;
   int s = n_splits;
-  const int a1 = auto_splits(c, streams_layer, max_tiles);
-  const int a2 = auto_splits(c, streams_layer * c->g.L, max_tiles);
+  const int rec = max_record(c, 0, c->g.L);
+  const int a1 = auto_splits(c, streams_layer, max_tiles, rec);
+  const int a2 = auto_splits(c, streams_layer * c->g.L, max_tiles, rec);
   if (s < a1) s = a1;
   if (s < a2) s = a2;
   const int64_t all = (int64_t)streams_layer * c->g.L;
@@ -267,18 +279,13 @@ rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out,
   const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
   const int n_tiles = Tq / rq::kTile;
   const int streams = nl * c->g.B * c->g.Hkv;
-  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles) : n_splits;
+  const int stage_bytes = max_record(c, l0, nl);
+  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes) : n_splits;
   if (splits > n_tiles) splits = n_tiles;
   if (n_tiles > 0 && splits < 1) splits = 1;
   const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
   if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + 1, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
   if (streams > 65535) return RQ_ERR_UNSUPPORTED;
-  int stage_bytes = 16;
-  for (int l = l0; l < l0 + nl; ++l)
-    for (int h = 0; h < c->g.Hkv; ++h) {
-      const int r = c->desc[l * c->g.Hkv + h].rec_bytes;
-      if (r > stage_bytes) stage_bytes = r;
-    }
   rq::DecodeArgs a;
   a.g = c->g;
   a.buf = c->buf;
@@ -293,13 +300,13 @@ rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out,
   a.Tq = Tq;
   a.n_tiles = n_tiles;
   a.n_splits = splits;
-  a.stages = 8;
+  a.stages = rq::decode_stages(stage_bytes);
   a.stage_bytes = stage_bytes;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.status = reinterpret_cast<int*>(ws);
   a.counters = reinterpret_cast<uint32_t*>(ws + rq::ws_counter_offset());
   a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
-  const int smem = rq::decode_smem_bytes(splits + 1, stage_bytes, c->g.G, c->g.D);
+  const int smem = rq::decode_smem_bytes(splits + 1, a.stages, stage_bytes, c->g.G, c->g.D);
   if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
   return cuda_status(rq::launch_decode(a, smem, stream));
 }

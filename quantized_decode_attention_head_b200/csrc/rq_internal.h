@@ -81,7 +81,7 @@ struct DecodeArgs {
   int layer0, n_layers;
   int T, Tq, n_tiles;
   int n_splits;           // tile splits; item n_splits is the bf16 window
-  int stages;             // pipeline depth (multiple of the consumer warp count)
+  int stages;             // per-warp ring depth (2..8)
   int stage_bytes;        // bytes per stage (max record size in the call)
   float* partials;        // [streams][n_splits+1][G*D + 2G]
   uint32_t* counters;     // [streams]
@@ -105,11 +105,16 @@ inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int item
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int smem_bytes, cudaStream_t s);
-int decode_smem_bytes(int n_items, int stage_bytes, int G, int D);
-cudaError_t decode_set_smem_limit(int smem_bytes);
+int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D);
+int decode_occupancy(int D, int G, int smem_bytes);  // resident CTAs per SM
 
 constexpr int kDecodeConsumerWarps = 4;
-constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
+constexpr int kDecodeThreads = kDecodeConsumerWarps * 32;
+// per-warp ring depth: about 64 KB of records in flight per CTA
+inline int decode_stages(int stage_bytes) {
+  int p = 65536 / (kDecodeConsumerWarps * stage_bytes);
+  return p < 2 ? 2 : (p > 8 ? 8 : p);
+}
 constexpr int kDeviceTimeout = 7;  // == RQ_ERR_DEVICE_TIMEOUT
 
 }  // namespace rq
