@@ -200,6 +200,31 @@ rq_status rq_decode_attention(rq_cache* cache, int layer, const void* q, float* 
  * without writing its outputs). */
 rq_status rq_decode_read_status(const void* workspace, int* device_status);
 
+/* rq_decode_attention_noalloc -- the same decode step as rq_decode_attention,
+ *   for callers that cannot allocate device memory: code running where
+ *   cudaMalloc is unavailable or forbidden (inside a custom allocator or
+ *   memory pool that must not re-enter the CUDA allocator, a host runtime
+ *   whose device memory is fully pre-reserved, or a plugin that may only use
+ *   buffers handed to it).  The pages define no such call; it has no
+ *   counterpart there.
+ * Scratch: a fixed 32 MiB device array inside this library (status word,
+ *   per-stream completion counters, split partials), held by every device
+ *   that loads the library until the process exits.  The first call on a
+ *   device looks the array's address up (cudaGetSymbolAddress) with that
+ *   device current; make that first call before any stream capture.  Each
+ *   call clears the status word and counters (cudaMemsetAsync on the given
+ *   stream) before the kernel; no memory is allocated or freed.
+ * All calls share the one array, which keeps the last call's contents: calls
+ *   that overlap on the GPU (other streams, other threads, other handles)
+ *   race and corrupt each other's results; serialise them.
+ * Arguments as rq_decode_attention, minus the workspace.  The device status
+ *   word is not readable through the C ABI for this variant.
+ * Errors: RQ_ERR_INVALID_ARG; RQ_ERR_WORKSPACE when the split partials of the
+ *   call (about (n_splits + 1) * streams * (G*D + 2G) * 4 bytes) exceed the
+ *   array -- reduce n_splits or decode fewer layers per call; RQ_ERR_CUDA. */
+rq_status rq_decode_attention_noalloc(rq_cache* cache, int layer, const void* q, float* out,
+                                      float softmax_scale, int n_splits, cudaStream_t stream);
+
 /* Library build description (static string). */
 const char* rq_build_info(void);
 

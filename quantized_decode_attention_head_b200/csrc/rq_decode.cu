@@ -24,6 +24,7 @@
 #include <cuda_fp16.h>
 
 #include <cfloat>
+#include <mutex>
 
 #include "rq_device.cuh"
 #include "rq_internal.h"
@@ -729,4 +730,36 @@ cudaError_t launch_decode(const DecodeArgs& a, int smem, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
+}  // namespace rq
+
+// ---------------------------------------------------------------------------
+// Scratch for rq_decode_attention_noalloc: a file-scope device array, so that
+// callers that must not allocate device memory (see include/rq.h) can still
+// run the split-K decode.  Every device that loads this library holds it
+// until the process exits.  Host code may only use the address returned by
+// cudaGetSymbolAddress for the current device, never the array's name.
+namespace rq {
+namespace {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+cudaError_t noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // once per device, with that device current
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
 }  // namespace rq

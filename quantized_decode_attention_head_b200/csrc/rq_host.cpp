@@ -312,3 +312,52 @@ rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out,
 }
 
 }  // extern "C"
+
+// Decode without a caller-supplied workspace (see include/rq.h).  Uses the
+// library's own device scratch array; allocates nothing.
+extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const void* q, float* out,
+                                                  float softmax_scale, int n_splits, cudaStream_t stream) {
+  if (!c || !q || !out || n_splits < 0) return RQ_ERR_INVALID_ARG;
+  int l0, nl;
+  if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
+  const int T = c->length[l0];
+  const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
+  const int n_tiles = Tq / rq::kTile;
+  const int streams = nl * c->g.B * c->g.Hkv;
+  if (streams > 65535) return RQ_ERR_UNSUPPORTED;
+  const int stage_bytes = max_record(c, l0, nl);
+  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes) : n_splits;
+  if (splits > n_tiles) splits = n_tiles;
+  if (n_tiles > 0 && splits < 1) splits = 1;
+  const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
+  if (rq::ws_total_bytes(all_streams, streams, splits + 1, c->g.G, c->g.D) > rq::kNoAllocScratchBytes)
+    return RQ_ERR_WORKSPACE;  // more split partials than the fixed scratch array holds
+  void* scratch = nullptr;
+  if (rq::noalloc_scratch(&scratch) != cudaSuccess) return RQ_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  // status word and completion counters must start at zero; the array keeps
+  // whatever the previous call (on any stream) left in it
+  if (cudaMemsetAsync(ws, 0, rq::ws_partial_offset(all_streams), stream) != cudaSuccess) return RQ_ERR_CUDA;
+  rq::DecodeArgs a;
+  a.g = c->g;
+  a.buf = c->buf;
+  a.desc = reinterpret_cast<const HeadDesc*>(c->buf);
+  a.q = static_cast<const uint16_t*>(q);
+  a.out = out;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)c->g.D);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.layer0 = l0;
+  a.n_layers = nl;
+  a.T = T;
+  a.Tq = Tq;
+  a.n_tiles = n_tiles;
+  a.n_splits = splits;
+  a.stages = rq::decode_stages(stage_bytes);
+  a.stage_bytes = stage_bytes;
+  a.status = reinterpret_cast<int*>(ws);
+  a.counters = reinterpret_cast<uint32_t*>(ws + rq::ws_counter_offset());
+  a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
+  const int smem = rq::decode_smem_bytes(splits + 1, a.stages, stage_bytes, c->g.G, c->g.D);
+  if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
+  return cuda_status(rq::launch_decode(a, smem, stream));
+}

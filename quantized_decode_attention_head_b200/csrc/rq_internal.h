@@ -108,6 +108,11 @@ cudaError_t launch_decode(const DecodeArgs& a, int smem_bytes, cudaStream_t s);
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D);
 int decode_occupancy(int D, int G, int smem_bytes);  // resident CTAs per SM
 
+// Size of the device array behind rq_decode_attention_noalloc (bytes).
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+// Address of that array on the current device (looked up once per device).
+cudaError_t noalloc_scratch(void** ptr);
+
 constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeThreads = kDecodeConsumerWarps * 32;
 // per-warp ring depth: about 64 KB of records in flight per CTA
