@@ -34,6 +34,7 @@ namespace {
 
 constexpr int NW = kDecodeConsumerWarps;
 constexpr int kMaxStages = 8;  // per-warp ring depth limit
+constexpr float kRescaleSlack = 8.0f;
 
 template <int D, int G>
 struct Cfg {
@@ -250,7 +251,10 @@ __device__ __forceinline__ void softmax_tile(WarpState<D, G>& st, const float (&
     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
     tmax[e] = v;
   }
-  const bool grow = tmax[0] > st.m[0] || tmax[1] > st.m[1];
+  // Lazy rescale: the reference max only moves when a score exceeds it by
+  // more than kRescaleSlack (log2 units), so P <= 2^kRescaleSlack stays well
+  // inside fp16 and o is rescaled only a handful of times per work item.
+  const bool grow = tmax[0] > st.m[0] + kRescaleSlack || tmax[1] > st.m[1] + kRescaleSlack;
   if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -276,57 +280,55 @@ template <int D, int G, int VB>
 __device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st, const uint32_t (&pb)[2][2], int lane) {
   constexpr int W = words_per_lane(VB, D);
   const int gid = lane >> 2;
-  uint32_t vw[W];
-  load_words<W>(vw, vrec, lane);
-  float acc[D / 16][4];
-#pragma unroll
-  for (int mb = 0; mb < D / 16; ++mb) {
-    acc[mb][0] = acc[mb][1] = acc[mb][2] = acc[mb][3] = 0.0f;
-#pragma unroll
-    for (int kb = 0; kb < 2; ++kb) {
-      uint32_t a[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int idx = v_pair_index(mb, kb, r);
-        a[r] = extract_pair<VB>(vw, slot_word(VB, W, idx), slot_pos(VB, W, idx));
-      }
-      mma_f16(acc[mb], a, pb[kb][0], pb[kb][1]);
-    }
-  }
   // sum_t p_t * 2^-24 per column: A = the fp16 subnormal 2^-24, so every
   // accumulator below carries the same 2^-24 as the unpacked codes
   float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   const uint32_t tiny[4] = {0x00010001u, 0x00010001u, 0x00010001u, 0x00010001u};
   mma_f16(ps, tiny, pb[0][0], pb[0][1]);
   mma_f16(ps, tiny, pb[1][0], pb[1][1]);
+  uint32_t vw[W];
+  load_words<W>(vw, vrec, lane);
   const uint32_t* vmeta = reinterpret_cast<const uint32_t*>(vrec + blob_bytes(VB, D)) + gid * (D / 8);
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
     const uint4 mv = *reinterpret_cast<const uint4*>(vmeta + 4 * c);
     const uint32_t mw[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int mb = 2 * c + j / 2, rr = j % 2;
-      const int cls = quad_class(VB, W, mb * 2 + rr);
-      float sv = half_lo_to_float(mw[j]);
-      if (cls) sv *= 1.0f / (float)(1 << (VB * cls));
-      const float z = __uint_as_float(mw[j] & 0xFFFF0000u);
+    for (int half = 0; half < 2; ++half) {
+      const int mb = 2 * c + half;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int e = 0; e < 2; ++e)
-        st.o[mb][rr * 2 + e] = fmaf(sv, acc[mb][rr * 2 + e], fmaf(z, ps[e], st.o[mb][rr * 2 + e]));
+      for (int kb = 0; kb < 2; ++kb) {
+        uint32_t a[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int idx = v_pair_index(mb, kb, r);
+          a[r] = extract_pair<VB>(vw, slot_word(VB, W, idx), slot_pos(VB, W, idx));
+        }
+        mma_f16(acc, a, pb[kb][0], pb[kb][1]);
+      }
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const uint32_t m = mw[half * 2 + rr];
+        const int cls = quad_class(VB, W, mb * 2 + rr);
+        float sv = half_lo_to_float(m);
+        if (cls) sv *= 1.0f / (float)(1 << (VB * cls));
+        const float z = __uint_as_float(m & 0xFFFF0000u);
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          st.o[mb][rr * 2 + e] = fmaf(sv, acc[rr * 2 + e], fmaf(z, ps[e], st.o[mb][rr * 2 + e]));
+      }
     }
   }
   st.l[0] += ps[0];
   st.l[1] += ps[1];
 }
 
-template <int D, int G, int KB, int VB>
-__device__ __forceinline__ void process_tile(const uint8_t* rec, WarpState<D, G>& st, int lane) {
+template <int D, int G, int KB>
+__device__ __forceinline__ void score_tile(const uint8_t* rec, WarpState<D, G>& st, uint32_t (&pb)[2][2], int lane) {
   float x[2][2][2];
   qk_tile<D, G, KB>(rec, st, x, lane);
-  uint32_t pb[2][2];
   softmax_tile<D, G>(st, x, pb);
-  pv_tile<D, G, VB>(rec + blob_bytes(KB, D) + 4 * D, st, pb, lane);
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
@@ -351,25 +353,55 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
     }
   }
   setup_query<D, G, KB>(st, qh, scale_log2, lane);
-  int j = 0;
-  for (; j < n_w; ++j) {
-    const int s = j % stages;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (j / stages) & 1));
-    if (!ok) {
-      if (lane == 0) raise_abort(abort_flag, status);
-      break;
-    }
-    process_tile<D, G, KB, VB>(ring + (size_t)s * stage_bytes, st, lane);
-    __syncwarp();
+  auto wait_tile = [&](int j) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait_bounded(&bars[j % stages], (j / stages) & 1));
+  };
+  auto refill = [&](int j) {  // the warp has finished reading tile j's slot
     if (lane == 0 && j + stages < n_w) {
-      fence_proxy_async_smem();  // the generic-proxy reads of this slot precede the async refill
+      fence_proxy_async_smem();  // generic-proxy reads of the slot precede the async refill
+      const int s = j % stages;
       mbar_arrive_expect_tx(&bars[s], (uint32_t)rec);
       bulk_g2s(ring + (size_t)s * stage_bytes, src + (int64_t)(warp + (j + stages) * NW) * rec, (uint32_t)rec,
                &bars[s]);
     }
+  };
+  const int VOFF = blob_bytes(KB, D) + 4 * D;
+  int j = 0;
+  bool ok = true;
+  if (n_w > 0) {
+    // software pipeline: the scores of tile j + 1 are computed in the same
+    // block as the P.V of tile j, so their MMA chains interleave
+    uint32_t pb[2][2];
+    ok = wait_tile(0);
+    if (ok) score_tile<D, G, KB>(ring, st, pb, lane);
+    for (; ok && j + 1 < n_w; ++j) {
+      ok = wait_tile(j + 1);
+      if (!ok) break;
+      const uint8_t* cur = ring + (size_t)(j % stages) * stage_bytes;
+      const uint8_t* nxt = ring + (size_t)((j + 1) % stages) * stage_bytes;
+      float x[2][2][2];
+      qk_tile<D, G, KB>(nxt, st, x, lane);
+      pv_tile<D, G, VB>(cur + VOFF, st, pb, lane);
+      softmax_tile<D, G>(st, x, pb);
+      __syncwarp();
+      refill(j);
+      if (*abort_flag) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok) {
+      pv_tile<D, G, VB>(ring + (size_t)(j % stages) * stage_bytes + VOFF, st, pb, lane);
+      __syncwarp();
+      ++j;
+    }
   }
-  if (j < n_w && lane == 0) {  // aborted: let the copies in flight land before the CTA exits
-    for (int k = j; k < n_w && k < j + stages; ++k) (void)mbar_wait_bounded(&bars[k % stages], (k / stages) & 1);
+  if (!ok) {
+    if (lane == 0) {
+      raise_abort(abort_flag, status);
+      // let the copies in flight land before the CTA exits
+      for (int k = j; k < n_w && k < j + stages; ++k) (void)mbar_wait_bounded(&bars[k % stages], (k / stages) & 1);
+    }
   }
 }
 
@@ -418,127 +450,179 @@ __device__ void dump_tile_state(const WarpState<D, G>& st, float* slot, int lane
   }
 }
 
-// bf16 sink + recent window on CUDA cores.  Warp w takes the window's
-// 32-token chunks w, w + 4, ...: lane 0 stages the chunk's K and V rows in
-// the warp's own shared buffer with at most six 1-D bulk copies (the rows of
-// a chunk form at most three contiguous runs: sink, ring, ring after wrap),
-// then the warp scores all G heads (lane = token; K row words read in a
-// lane-rotated order so the 32 rows hit 32 banks) and accumulates P.V
-// (lane = channel).  Only warp-level synchronisation inside the loop.
+// bf16 sink + recent window on CUDA cores.  The window is split into work
+// items of 32 tokens.  Thread 0 stages the item's K and V rows in shared
+// memory with at most six 1-D bulk copies (the rows of a chunk form at most
+// three contiguous runs: sink, ring, ring after wrap); warp w then takes heads
+// w, w + 4, ...: lane = token for q.k (K row words read in a lane-rotated
+// order so the 32 rows hit 32 banks), lane = channel for p.v.
 constexpr int kWinChunk = 32;
 
+__host__ __device__ inline int window_tokens(int T, int S, int Tq) { return (T < S ? T : S) + (T - (T < S ? T : S) - Tq); }
+
 template <int D>
-__device__ __forceinline__ int window_issue_chunk(const DecodeArgs& a, const uint8_t* win, uint32_t* kbuf,
-                                                  uint32_t* vbuf, uint64_t* bar, int j0, int cnt) {
+__device__ __forceinline__ void window_issue_chunk(const DecodeArgs& a, const uint8_t* win, uint32_t* kbuf,
+                                                   uint32_t* vbuf, uint64_t* bar, int j0, int cnt) {
   const int S = a.g.S, ring = a.g.R + kTile;
   const int n_sink = a.T < S ? a.T : S;
   mbar_arrive_expect_tx(bar, (uint32_t)(cnt * D * 2 * 2));
   int t = 0;
   while (t < cnt) {
     const int j = j0 + t;
-    size_t row;  // row index inside the K half of the window block
+    size_t row;  // K row inside the window block; its V row follows its block's K rows
     int run;
+    size_t v_off;
     if (j < n_sink) {
       row = j;
       run = min(cnt - t, n_sink - j);
+      v_off = S;
     } else {
       const int slot = (a.Tq + (j - n_sink)) % ring;
       row = (size_t)2 * S + slot;
       run = min(cnt - t, ring - slot);
+      v_off = ring;
     }
-    const size_t v_off = (j < n_sink) ? (size_t)S : (size_t)ring;  // V rows follow the K rows of their block
     bulk_g2s(kbuf + (size_t)t * (D / 2), win + row * D * 2, (uint32_t)(run * D * 2), bar);
     bulk_g2s(vbuf + (size_t)t * (D / 2), win + (row + v_off) * D * 2, (uint32_t)(run * D * 2), bar);
     t += run;
   }
-  return 0;
 }
 
 template <int D, int G>
-__device__ void window_warp(const DecodeArgs& a, const uint8_t* win, const float2* q2, uint32_t* kbuf,
-                            uint32_t* vbuf, uint64_t* bar, float* slot, int warp, int lane,
-                            volatile int* abort_flag) {
+__device__ void window_item(const DecodeArgs& a, const uint8_t* win, const uint16_t* qh, int chunk, float* scratch,
+                            uint64_t* bar, float* slot, int warp, int lane, volatile int* abort_flag) {
   constexpr int RW = D / 2;  // words per bf16 row
-  const int S = a.g.S;
-  const int n_sink = a.T < S ? a.T : S;
-  const int n_tok = n_sink + (a.T - n_sink - a.Tq);
-  const int n_chunks = (n_tok + kWinChunk - 1) / kWinChunk;
-  float m[G], l[G], o[G][D / 32];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.0f;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) o[h][c] = 0.0f;
+  constexpr int HW = (G + NW - 1) / NW;
+  const int tid = warp * 32 + lane;
+  const int n_tok = window_tokens(a.T, a.g.S, a.Tq);
+  const int j0 = chunk * kWinChunk;
+  const int cnt = max(0, min(kWinChunk, n_tok - j0));
+  float* qs = scratch;                                              // [G][D]
+  uint32_t* kbuf = reinterpret_cast<uint32_t*>(qs + G * D);         // [32][RW]
+  uint32_t* vbuf = kbuf + kWinChunk * RW;                           // [32][RW]
+  if (tid == 0 && cnt > 0) window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt);
+  for (int i = tid; i < G * D; i += NW * 32) qs[i] = bf16_bits_to_float(qh[i]);
+  const bool ok = cnt == 0 || __all_sync(0xffffffffu, mbar_wait_bounded(bar, 0));
+  if (!__syncthreads_and(ok)) {
+    if (tid == 0) {
+      raise_abort(abort_flag, a.status);
+      (void)mbar_wait_bounded(bar, 0);  // let the copies land before the CTA exits
+    }
+    return;
   }
-  int k = 0;
-  for (int c = warp; c < n_chunks; c += NW, ++k) {
-    const int j0 = c * kWinChunk;
-    const int cnt = min(kWinChunk, n_tok - j0);
-    if (k > 0) __syncwarp();  // the previous chunk is fully read
-    if (lane == 0) {
-      if (k > 0) fence_proxy_async_smem();
-      window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt);
-    }
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar, k & 1))) {
-      if (lane == 0) {
-        raise_abort(abort_flag, a.status);
-        (void)mbar_wait_bounded(bar, k & 1);  // let this warp's copies land before the CTA exits
+#pragma unroll
+  for (int j = 0; j < HW; ++j) {
+    const int h = warp + NW * j;
+    float m = -INFINITY, l = 0.0f, o[D / 32];
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) o[c] = 0.0f;
+    if (h < G && cnt > 0) {
+      float acc = 0.0f;
+      if (lane < cnt) {
+#pragma unroll 8
+        for (int w = 0; w < RW; ++w) {
+          const int wr = (w + lane) & (RW - 1);
+          const uint32_t kk = kbuf[lane * RW + wr];
+          acc = fmaf(qs[h * D + 2 * wr], bf16_bits_to_float(kk & 0xFFFFu),
+                     fmaf(qs[h * D + 2 * wr + 1], bf16_bits_to_float(kk >> 16), acc));
+        }
       }
-      return;
-    }
-    // scores of token `lane` for all heads
-    float sc[G];
+      const float x = lane < cnt ? acc * a.scale_log2 : -INFINITY;
+      m = warp_max(x);
+      const float p = ex2(x - m);
+      l = warp_sum(p);
+      for (int t = 0; t < cnt; ++t) {
+        const float pt = __shfl_sync(0xffffffffu, p, t);
 #pragma unroll
-    for (int h = 0; h < G; ++h) sc[h] = 0.0f;
-    if (lane < cnt) {
-#pragma unroll 4
-      for (int w = 0; w < RW; ++w) {
-        const int wr = (w + lane) & (RW - 1);
-        const uint32_t kk = kbuf[lane * RW + wr];
-        const float k0 = bf16_bits_to_float(kk & 0xFFFFu), k1 = bf16_bits_to_float(kk >> 16);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float2 qq = q2[h * RW + wr];
-          sc[h] = fmaf(qq.x, k0, fmaf(qq.y, k1, sc[h]));
+        for (int c = 0; c < D / 32; ++c) {
+          const int d = lane + 32 * c;
+          const uint32_t vv = vbuf[t * RW + d / 2];
+          o[c] = fmaf(pt, (d & 1) ? bf16_bits_to_float(vv >> 16) : bf16_bits_to_float(vv & 0xFFFFu), o[c]);
         }
       }
     }
-    float p[G];
+    if (h < G) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float x = lane < cnt ? sc[h] * a.scale_log2 : -INFINITY;
-      const float mn = fmaxf(m[h], warp_max(x));
-      const float alpha = ex2(m[h] - mn);
-      p[h] = ex2(x - mn);
-      l[h] = l[h] * alpha + warp_sum(p[h]);
-      m[h] = mn;
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) o[h][cc] *= alpha;
-    }
-    for (int t = 0; t < cnt; ++t) {
-      float v[D / 32];
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        const int d = lane + 32 * cc;
-        const uint32_t vv = vbuf[t * RW + d / 2];
-        v[cc] = (d & 1) ? bf16_bits_to_float(vv >> 16) : bf16_bits_to_float(vv & 0xFFFFu);
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float pt = __shfl_sync(0xffffffffu, p[h], t);
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) o[h][cc] = fmaf(pt, v[cc], o[h][cc]);
+      for (int c = 0; c < D / 32; ++c) slot[h * D + lane + 32 * c] = o[c];
+      if (lane == 0) {
+        slot[G * D + h] = m;
+        slot[G * D + G + h] = l;
       }
     }
   }
-#pragma unroll
+  // heads of the other warps: empty partial states
   for (int h = 0; h < G; ++h) {
+    if (h % NW == warp) continue;
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) slot[h * D + lane + 32 * cc] = o[h][cc];
+    for (int c = 0; c < D / 32; ++c) slot[h * D + lane + 32 * c] = 0.0f;
     if (lane == 0) {
-      slot[G * D + h] = m[h];
-      slot[G * D + G + h] = l[h];
+      slot[G * D + h] = -INFINITY;
+      slot[G * D + G + h] = 0.0f;
+    }
+  }
+}
+
+// Log-sum-exp merge of n partial states (stride PART floats from `base`)
+// into one: written to `dst` as a partial, or normalised into `outp`.  Each
+// thread owns OPT outputs and loads the o, m and l of up to U partials for
+// all of them at once (one round of independent loads per U partials).
+template <int D, int G>
+__device__ void combine_partials(const float* base, int n, float* dst, float* outp, int tid) {
+  using C = Cfg<D, G>;
+  constexpr int OPT = (G * D + kDecodeThreads - 1) / kDecodeThreads;
+  constexpr int U = OPT >= 32 ? 1 : 32 / OPT;  // at most 96 values in flight per thread
+  float M[OPT], L[OPT], O[OPT];
+#pragma unroll
+  for (int k = 0; k < OPT; ++k) {
+    M[k] = -INFINITY;
+    L[k] = 0.0f;
+    O[k] = 0.0f;
+  }
+  for (int i0 = 0; i0 < n; i0 += U) {
+    float ov[OPT][U], mv[OPT][U], lv[OPT][U];
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+      const int idx = tid + k * kDecodeThreads;
+      const int hh = idx < G * D ? idx / D : 0;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const bool ok = idx < G * D && i0 + u < n;
+        const float* pp = base + (size_t)(i0 + u) * C::PART;
+        ov[k][u] = ok ? __ldcg(pp + idx) : 0.0f;
+        mv[k][u] = ok ? __ldcg(pp + G * D + hh) : -INFINITY;
+        lv[k][u] = ok ? __ldcg(pp + G * D + G + hh) : 0.0f;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+      float nm = M[k];
+#pragma unroll
+      for (int u = 0; u < U; ++u) nm = fmaxf(nm, mv[k][u]);
+      if (nm == -INFINITY) continue;
+      const float a = ex2(M[k] - nm);  // 0 when M was -inf
+      O[k] *= a;
+      L[k] *= a;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float f = ex2(mv[k][u] - nm);
+        O[k] = fmaf(ov[k][u], f, O[k]);
+        L[k] = fmaf(lv[k][u], f, L[k]);
+      }
+      M[k] = nm;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < OPT; ++k) {
+    const int idx = tid + k * kDecodeThreads;
+    if (idx >= G * D) continue;
+    if (outp) {
+      outp[idx] = L[k] > 0.0f ? O[k] / L[k] : 0.0f;
+    } else {
+      dst[idx] = O[k];
+      if (idx % D == 0) {
+        dst[G * D + idx / D] = M[k];
+        dst[G * D + G + idx / D] = L[k];
+      }
     }
   }
 }
@@ -553,7 +637,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int srel = blockIdx.y, item = blockIdx.x;
-  const int NI = a.n_splits + 1;
+  const int NI = a.n_splits + a.n_win;  // work items of this stream
+  const int NG = (NI + kGroup - 1) / kGroup;
   const int h = srel % a.g.Hkv, b = (srel / a.g.Hkv) % a.g.B, lrel = srel / (a.g.Hkv * a.g.B);
   const int l = a.layer0 + lrel;
   const HeadDesc hd = a.desc[l * a.g.Hkv + h];
@@ -580,18 +665,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a)
                              smem + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
                              bars + warp * kMaxStages, src, rec, n_my, warp, lane, &abort_flag, a.status);
   } else {
-    // bf16 sink + recent window: q (fp32 pairs) after the merge slots, then
-    // one K and one V chunk buffer per warp
+    // one 32-token chunk of the bf16 sink + recent window
     const uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
-    float2* q2 = reinterpret_cast<float2*>(merge + NW * C::PART);
-    for (int i = tid; i < G * D / 2; i += blockDim.x) {
-      const uint32_t w = reinterpret_cast<const uint32_t*>(qh)[i];
-      q2[i] = make_float2(bf16_bits_to_float(w & 0xFFFFu), bf16_bits_to_float(w >> 16));
-    }
-    __syncthreads();
-    uint32_t* kbuf = reinterpret_cast<uint32_t*>(q2 + G * D / 2) + (size_t)warp * 2 * kWinChunk * (D / 2);
-    window_warp<D, G>(a, win, q2, kbuf, kbuf + kWinChunk * (D / 2), &bars[warp * kMaxStages], merge + warp * C::PART,
-                      warp, lane, &abort_flag);
+    window_item<D, G>(a, win, qh, item - a.n_splits, merge + NW * C::PART, &bars[0], merge + warp * C::PART, warp,
+                      lane, &abort_flag);
   }
   __syncthreads();  // every stage read has completed; merge may now alias the stages
   if (tiles_item && warp < NW && !abort_flag) dump_tile_state<D, G>(st, merge + warp * C::PART, lane);
@@ -620,62 +697,32 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a)
       part[G * D + G + hh] = L;
     }
   }
+  // two-level log-sum-exp combine: the last item of each group of kGroup
+  // merges the group; the last group merges the group results into out.
+  uint32_t* cnt = a.counters + (size_t)srel * kCountersPerStream;
+  const int g = item / kGroup;
+  const int gsize = min(kGroup, NI - g * kGroup);
+  float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
+  float* gpart = a.partials + (size_t)a.n_streams * NI * C::PART + ((size_t)srel * NG + g) * C::PART;
   __threadfence();
   __syncthreads();
-  if (tid == 0) is_last = (atomicAdd(&a.counters[srel], 1u) == (unsigned)(NI - 1));
+  if (tid == 0) is_last = (atomicAdd(&cnt[1 + g], 1u) == (unsigned)(gsize - 1));
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-
-  // last CTA of the stream: log-sum-exp combine over all items
-  float* wts = merge;  // [NI][G] weights, then [G] 1/L
-  const float* base = a.partials + (size_t)srel * NI * C::PART;
-  for (int hh = warp; hh < G; hh += blockDim.x / 32) {
-    float M = -INFINITY;
-    for (int i = lane; i < NI; i += 32) M = fmaxf(M, __ldcg(base + (size_t)i * C::PART + G * D + hh));
-    M = warp_max(M);
-    float L = 0.0f;
-    for (int i = lane; i < NI; i += 32) {
-      const float mi = __ldcg(base + (size_t)i * C::PART + G * D + hh);
-      const float f = (M == -INFINITY) ? 0.0f : ex2(mi - M);
-      wts[i * G + hh] = f;
-      L = fmaf(__ldcg(base + (size_t)i * C::PART + G * D + G + hh), f, L);
-    }
-    L = warp_sum(L);
-    if (lane == 0) wts[NI * G + hh] = L > 0.0f ? 1.0f / L : 0.0f;
-  }
+  combine_partials<D, G>(a.partials + ((size_t)srel * NI + g * kGroup) * C::PART, gsize, gpart,
+                         NG == 1 ? outp : nullptr, tid);
+  if (tid == 0) cnt[1 + g] = 0u;
+  if (NG == 1) return;
+  __threadfence();
   __syncthreads();
-  float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  // each thread owns OPT outputs; U items per round -> OPT * U loads in flight
-  constexpr int OPT = (G * D + kDecodeThreads - 1) / kDecodeThreads;
-  constexpr int U = OPT >= 64 ? 1 : 64 / OPT;
-  float acc[OPT];
-#pragma unroll
-  for (int k = 0; k < OPT; ++k) acc[k] = 0.0f;
-  for (int i0 = 0; i0 < NI; i0 += U) {
-    float v[OPT][U];
-#pragma unroll
-    for (int k = 0; k < OPT; ++k) {
-      const int idx = tid + k * kDecodeThreads;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        v[k][u] = (idx < G * D && i0 + u < NI) ? __ldcg(base + (size_t)(i0 + u) * C::PART + idx) : 0.0f;
-    }
-#pragma unroll
-    for (int k = 0; k < OPT; ++k) {
-      const int idx = tid + k * kDecodeThreads;
-      const int hh = idx < G * D ? idx / D : 0;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (i0 + u < NI) acc[k] = fmaf(v[k][u], wts[(i0 + u) * G + hh], acc[k]);
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < OPT; ++k) {
-    const int idx = tid + k * kDecodeThreads;
-    if (idx < G * D) outp[idx] = acc[k] * wts[NI * G + idx / D];
-  }
-  if (tid == 0) a.counters[srel] = 0u;
+  if (tid == 0) is_last = (atomicAdd(&cnt[0], 1u) == (unsigned)(NG - 1));
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  combine_partials<D, G>(a.partials + (size_t)a.n_streams * NI * C::PART + (size_t)srel * NG * C::PART, NG,
+                         nullptr, outp, tid);
+  if (tid == 0) cnt[0] = 0u;
 }
 
 template <int D, int G>
@@ -683,7 +730,7 @@ cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int streams = a.n_layers * a.g.B * a.g.Hkv;
-  dim3 grid(a.n_splits + 1, streams);
+  dim3 grid(a.n_splits + a.n_win, streams);
   decode_kernel<D, G><<<grid, kDecodeThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
@@ -692,10 +739,8 @@ cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
 
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   const int part = G * D + 2 * G;
-  // merge slots + window scratch (q, one K and one V chunk per warp)
-  int merge = (NW * part + G * D) * 4 + NW * 2 * kWinChunk * D * 2;
-  const int wts = (n_items + 1) * G * 4;
-  merge = merge > wts ? merge : wts;
+  // merge slots + window scratch (q, one K and one V chunk)
+  int merge = (NW * part + G * D) * 4 + 2 * kWinChunk * D * 2;
   const int ring = NW * stages * stage_bytes;
   int need = ring > merge ? ring : merge;
   return (need + 127) / 128 * 128;

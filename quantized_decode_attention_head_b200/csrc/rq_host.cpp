@@ -99,16 +99,17 @@ int max_record(const rq_cache* c, int l0, int nl) {
 
 // Tile splits per stream so that all work items of the call (splits + one
 // window item per stream) fill the resident CTA slots of the GPU once.
-int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes) {
+int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win) {
   if (n_tiles <= 0) return 0;
   const int occ = rq::decode_occupancy(
       c->g.D, c->g.G, rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes), stage_bytes, c->g.G, c->g.D));
   const long slots = (long)occ * c->sm_count;
-  long s = slots / streams - 1;
+  long s = slots / streams - n_win;
   if (s < 1) s = 1;
   const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;  // keep a CTA's pipeline busy
   if (s > max_by_work) s = max_by_work;
   if (s > n_tiles) s = n_tiles;
+  if (s > rq::kMaxItems - n_win) s = rq::kMaxItems - n_win;
   return (int)s;
 }
 
@@ -251,12 +252,14 @@ rq_status rq_decode_workspace_bytes(const rq_cache* c, int n_splits, size_t* byt
   const int max_tiles = c->g.max_tiles;
   int s = n_splits;
   const int rec = max_record(c, 0, c->g.L);
-  const int a1 = auto_splits(c, streams_layer, max_tiles, rec);
-  const int a2 = auto_splits(c, streams_layer * c->g.L, max_tiles, rec);
+  const int nw = (c->g.S + c->g.R + 2 * rq::kTile - 1) / rq::kTile;  // most window items any length can need
+  const int a1 = auto_splits(c, streams_layer, max_tiles, rec, 1);
+  const int a2 = auto_splits(c, streams_layer * c->g.L, max_tiles, rec, 1);
   if (s < a1) s = a1;
   if (s < a2) s = a2;
+  if (s > rq::kMaxItems - nw) s = rq::kMaxItems - nw;
   const int64_t all = (int64_t)streams_layer * c->g.L;
-  *bytes = rq::ws_total_bytes(all, all, s + 1, c->g.G, c->g.D);
+  *bytes = rq::ws_total_bytes(all, all, s + nw, c->g.G, c->g.D);
   return RQ_OK;
 }
 
@@ -280,11 +283,13 @@ rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out,
   const int n_tiles = Tq / rq::kTile;
   const int streams = nl * c->g.B * c->g.Hkv;
   const int stage_bytes = max_record(c, l0, nl);
-  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes) : n_splits;
+  const int n_win = rq::window_items(T, c->g.S, c->g.R);
+  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win) : n_splits;
   if (splits > n_tiles) splits = n_tiles;
   if (n_tiles > 0 && splits < 1) splits = 1;
+  if (splits + n_win > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
   const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
-  if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + 1, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
+  if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + n_win, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
   if (streams > 65535) return RQ_ERR_UNSUPPORTED;
   rq::DecodeArgs a;
   a.g = c->g;
@@ -300,13 +305,15 @@ rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out,
   a.Tq = Tq;
   a.n_tiles = n_tiles;
   a.n_splits = splits;
+  a.n_win = n_win;
+  a.n_streams = streams;
   a.stages = rq::decode_stages(stage_bytes);
   a.stage_bytes = stage_bytes;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.status = reinterpret_cast<int*>(ws);
   a.counters = reinterpret_cast<uint32_t*>(ws + rq::ws_counter_offset());
   a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
-  const int smem = rq::decode_smem_bytes(splits + 1, a.stages, stage_bytes, c->g.G, c->g.D);
+  const int smem = rq::decode_smem_bytes(splits + n_win, a.stages, stage_bytes, c->g.G, c->g.D);
   if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
   return cuda_status(rq::launch_decode(a, smem, stream));
 }
@@ -326,11 +333,13 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
   const int streams = nl * c->g.B * c->g.Hkv;
   if (streams > 65535) return RQ_ERR_UNSUPPORTED;
   const int stage_bytes = max_record(c, l0, nl);
-  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes) : n_splits;
+  const int n_win = rq::window_items(T, c->g.S, c->g.R);
+  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win) : n_splits;
   if (splits > n_tiles) splits = n_tiles;
   if (n_tiles > 0 && splits < 1) splits = 1;
+  if (splits + n_win > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
   const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
-  if (rq::ws_total_bytes(all_streams, streams, splits + 1, c->g.G, c->g.D) > rq::kNoAllocScratchBytes)
+  if (rq::ws_total_bytes(all_streams, streams, splits + n_win, c->g.G, c->g.D) > rq::kNoAllocScratchBytes)
     return RQ_ERR_WORKSPACE;  // more split partials than the fixed scratch array holds
   void* scratch = nullptr;
   if (rq::noalloc_scratch(&scratch) != cudaSuccess) return RQ_ERR_CUDA;
@@ -352,12 +361,14 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
   a.Tq = Tq;
   a.n_tiles = n_tiles;
   a.n_splits = splits;
+  a.n_win = n_win;
+  a.n_streams = streams;
   a.stages = rq::decode_stages(stage_bytes);
   a.stage_bytes = stage_bytes;
   a.status = reinterpret_cast<int*>(ws);
   a.counters = reinterpret_cast<uint32_t*>(ws + rq::ws_counter_offset());
   a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
-  const int smem = rq::decode_smem_bytes(splits + 1, a.stages, stage_bytes, c->g.G, c->g.D);
+  const int smem = rq::decode_smem_bytes(splits + n_win, a.stages, stage_bytes, c->g.G, c->g.D);
   if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
   return cuda_status(rq::launch_decode(a, smem, stream));
 }

@@ -80,7 +80,9 @@ struct DecodeArgs {
   float scale_log2;       // softmax scale * log2(e)
   int layer0, n_layers;
   int T, Tq, n_tiles;
-  int n_splits;           // tile splits; item n_splits is the bf16 window
+  int n_splits;           // tile splits: items [0, n_splits)
+  int n_win;              // bf16 window items (32 tokens each): items [n_splits, n_splits + n_win)
+  int n_streams;          // streams of this call
   int stages;             // per-warp ring depth (2..8)
   int stage_bytes;        // bytes per stage (max record size in the call)
   float* partials;        // [streams][n_splits+1][G*D + 2G]
@@ -88,17 +90,31 @@ struct DecodeArgs {
   int* status;            // workspace status word
 };
 
-// Workspace layout (bytes): [status int32, pad to 256][one u32 counter per
-// stream of the whole cache (L*B*Hkv), pad to 256][partials of one call].
-// The counter region is sized for every stream so calls with different layer
-// arguments never overlap each other's counters.
+// Split-K combine: work items are merged in groups of kGroup, then groups.
+constexpr int kGroup = 8;
+constexpr int kCountersPerStream = 64;  // [0] group counter, [1 + g] item counters of group g
+constexpr int kMaxItems = kGroup * (kCountersPerStream - 1);
+inline int group_count(int items) { return (items + kGroup - 1) / kGroup; }
+
+// Workspace layout (bytes): [status int32, pad to 256][kCountersPerStream u32
+// counters per stream of the whole cache (L*B*Hkv)][item partials of one
+// call][group partials of one call].  The counter region is sized for every
+// stream so calls with different layer arguments never overlap.
 inline size_t ws_counter_offset() { return 256; }
 inline size_t ws_partial_offset(int64_t all_streams) {
-  size_t c = ws_counter_offset() + (size_t)all_streams * 4;
-  return (c + 255) / 256 * 256;
+  return ws_counter_offset() + (size_t)all_streams * kCountersPerStream * 4;
 }
 inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int items, int G, int D) {
-  return ws_partial_offset(all_streams) + (size_t)call_streams * items * (size_t)(G * D + 2 * G) * 4;
+  return ws_partial_offset(all_streams) +
+         (size_t)call_streams * (items + group_count(items)) * (size_t)(G * D + 2 * G) * 4;
+}
+// bf16 window tokens of a T-token cache and the number of 32-token window items
+inline int window_items(int T, int S, int R) {
+  const int n_sink = T < S ? T : S;
+  const int n_tok = T - quantized_tokens(T, S, R);
+  (void)n_sink;
+  const int n = (n_tok + kTile - 1) / kTile;
+  return n > 0 ? n : 1;
 }
 
 // Kernel launchers (rq_kernels.cu).  Return cudaGetLastError() after launch.
