@@ -52,27 +52,30 @@ def _peaks():
 
 
 # --------------------------------------------------------------- byte counts
-def decode_bytes(wl, k_bits, v_bits, T):
-    """Algorithmic bytes of one decode over a cache of T tokens (all streams)."""
-    from oracle.cache import split_lengths  # pure arithmetic on lengths
-    from oracle.quantize import record_bytes
+def split_lengths(T, n_sink, n_recent):
+    """(sink, quantized, recent) token counts of a stream of T tokens: tiles of
+    32 are quantized once more than n_recent tokens follow the sink."""
+    s = min(T, n_sink)
+    tq = ((T - n_sink - n_recent) // 32) * 32 if T >= n_sink + n_recent else 0
+    return s, tq, T - s - tq
 
+
+def decode_bytes(wl, rec, T):
+    """Algorithmic bytes of one decode over a cache of T tokens (all streams);
+    rec[l][h] = bytes of one packed 32-token tile record of (layer, kv-head)."""
     s, tq, r = split_lengths(T, wl.n_sink, wl.n_recent)
     n_tiles = tq // 32
     D, G = wl.head_dim, wl.group
     total = 0
     for l in range(wl.n_layers):
         for h in range(wl.n_kv_heads):
-            per_stream = n_tiles * record_bytes(int(k_bits[l, h]), int(v_bits[l, h]), D)
+            per_stream = n_tiles * int(rec[l][h])
             per_stream += (s + r) * D * 2 * 2 + G * D * 2 + G * D * 4
             total += per_stream * wl.batch
     return total
 
 
-def append_bytes(wl, k_bits, v_bits, T_old):
-    from oracle.cache import split_lengths
-    from oracle.quantize import record_bytes
-
+def append_bytes(wl, rec, T_old):
     D = wl.head_dim
     s, tq, r = split_lengths(T_old, wl.n_sink, wl.n_recent)
     flush = T_old >= wl.n_sink and r + 1 == wl.n_recent + 32
@@ -81,7 +84,7 @@ def append_bytes(wl, k_bits, v_bits, T_old):
         for h in range(wl.n_kv_heads):
             b = 2 * D * 2 * 2  # read new rows, write them to the ring
             if flush:
-                b += 32 * D * 2 * 2 + record_bytes(int(k_bits[l, h]), int(v_bits[l, h]), D)
+                b += 32 * D * 2 * 2 + int(rec[l][h])
             total += b * wl.batch
     return total
 
@@ -177,8 +180,8 @@ def oracle_sample(wl, seconds=12.0):
         if time.perf_counter() - t0 >= seconds:
             break
     t_dec = (time.perf_counter() - t0) / runs
-    kb = np.full((1, 1), 2)
-    bytes_dec = decode_bytes(one, kb, kb, wl.context)
+    rec = [[qz.record_bytes(2, 2, wl.head_dim)]]
+    bytes_dec = decode_bytes(one, rec, wl.context)
     bytes_q = wl.context * wl.head_dim * 2 * 2 + bytes_dec
     return {
         "decode_gbs": bytes_dec / t_dec / 1e9,
@@ -276,11 +279,14 @@ def run_gpu(args):
         torch.cuda.synchronize()
         if c > 0:  # the first call pays one-time set-up
             qtimes.append(e0.elapsed_time(e1) / 1e3)
-            qbytes = k.numel() * 2 * 2 + decode_bytes(wl, kb, kb, wl.context)
+            qbytes = k.numel() * 2 * 2 + decode_bytes(wl, rec, wl.context)
         del k, v
         q, kn, vn = workloads.step_inputs(wl, steps_per_copy, f, "cuda", seed=seed)
         caches.append(cache)
         step_in.append((q, kn, vn))
+        if c == 0:  # packed record size of every (layer, kv-head), from the library's own layout
+            rec = [[cache.stream_layout(l, 0, h)["record_bytes"] for h in range(wl.n_kv_heads)]
+                   for l in range(wl.n_layers)]
     ws = caches[0].make_workspace(n_splits=args.splits)
     outs = [torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=torch.float32, device="cuda") for _ in range(NC)]
     torch.cuda.synchronize()
@@ -305,8 +311,8 @@ def run_gpu(args):
     for i in range(args.warmup, total_steps):
         c = i % NC
         T_old = caches[c].length(0) + (i - args.warmup) // NC  # length before this step's append
-        ab = append_bytes(wl, kb, kb, T_old)
-        db = decode_bytes(wl, kb, kb, T_old + 1)
+        ab = append_bytes(wl, rec, T_old)
+        db = decode_bytes(wl, rec, T_old + 1)
         step_bytes += ab + db
         dec_bytes_steps.append(db)
     if world > 1:
@@ -343,7 +349,7 @@ def run_gpu(args):
     e2e_bytes = 0
     for i in range(e2e_steps):
         c = i % NC
-        e2e_bytes += append_bytes(wl, kb, kb, base_len[c] + i // NC) + decode_bytes(wl, kb, kb, base_len[c] + i // NC + 1)
+        e2e_bytes += append_bytes(wl, rec, base_len[c] + i // NC) + decode_bytes(wl, rec, base_len[c] + i // NC + 1)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -411,7 +417,7 @@ def run_gpu(args):
         "config": {"workload": WORKLOAD, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
                    "head_dim": wl.head_dim, "context": wl.context, "bits": "K=V=2 on every head (avg 2 over {2,3,4})",
                    "splits": args.splits or "auto", "l2": f"{NC} caches decoded round-robin "
-                   f"({NC * decode_bytes(wl, kb, kb, wl.context) / 1e6:.0f} MB > 126 MB L2)",
+                   f"({NC * decode_bytes(wl, rec, wl.context) / 1e6:.0f} MB > 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
         "decode_gbs": achieved,
         "decode_us": dec_avg * 1e6,

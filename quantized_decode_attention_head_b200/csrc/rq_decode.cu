@@ -2,9 +2,10 @@
 //
 // One CTA = one work item of one (layer, batch, kv-head) stream: either a
 // contiguous range of packed tiles (items 0..n_splits-1) or the bf16 sink +
-// recent window (item n_splits).  Four consumer warps process tiles; a fifth
-// warp streams tile records into a ring of shared-memory stages with 1-D bulk
-// copies (cp.async.bulk, TMA engine) completing on mbarriers.  The last CTA
+// recent window (items n_splits..).  Four warps process tiles; lane 0 of each
+// streams the warp's own tile records into a private ring of shared-memory
+// stages with 1-D bulk copies (cp.async.bulk, TMA engine) completing on
+// mbarriers.  The last CTA
 // of a stream to finish merges all items' partial softmax states
 // (log-sum-exp) and writes the output -- no second launch.
 //
@@ -353,16 +354,17 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
     }
   }
   setup_query<D, G, KB>(st, qh, scale_log2, lane);
-  auto wait_tile = [&](int j) -> bool {
-    return __all_sync(0xffffffffu, mbar_wait_bounded(&bars[j % stages], (j / stages) & 1));
+  // ring position of a tile: slot = j mod stages, parity = (j / stages) & 1,
+  // advanced incrementally (no integer division in the loop)
+  auto wait_slot = [&](int slot, int parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], (uint32_t)parity));
   };
-  auto refill = [&](int j) {  // the warp has finished reading tile j's slot
+  auto refill = [&](int j, int slot) {  // the warp has finished reading tile j's slot
     if (lane == 0 && j + stages < n_w) {
       fence_proxy_async_smem();  // generic-proxy reads of the slot precede the async refill
-      const int s = j % stages;
-      mbar_arrive_expect_tx(&bars[s], (uint32_t)rec);
-      bulk_g2s(ring + (size_t)s * stage_bytes, src + (int64_t)(warp + (j + stages) * NW) * rec, (uint32_t)rec,
-               &bars[s]);
+      mbar_arrive_expect_tx(&bars[slot], (uint32_t)rec);
+      bulk_g2s(ring + (size_t)slot * stage_bytes, src + (int64_t)(warp + (j + stages) * NW) * rec, (uint32_t)rec,
+               &bars[slot]);
     }
   };
   const int VOFF = blob_bytes(KB, D) + 4 * D;
@@ -372,26 +374,37 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
     // software pipeline: the scores of tile j + 1 are computed in the same
     // block as the P.V of tile j, so their MMA chains interleave
     uint32_t pb[2][2];
-    ok = wait_tile(0);
+    int cs = 0;             // slot of tile j
+    int ns = 1, nph = 0;    // slot and parity of tile j + 1
+    if (ns == stages) {
+      ns = 0;
+      nph = 1;
+    }
+    ok = wait_slot(0, 0);
     if (ok) score_tile<D, G, KB>(ring, st, pb, lane);
     for (; ok && j + 1 < n_w; ++j) {
-      ok = wait_tile(j + 1);
+      ok = wait_slot(ns, nph);
       if (!ok) break;
-      const uint8_t* cur = ring + (size_t)(j % stages) * stage_bytes;
-      const uint8_t* nxt = ring + (size_t)((j + 1) % stages) * stage_bytes;
+      const uint8_t* cur = ring + (size_t)cs * stage_bytes;
+      const uint8_t* nxt = ring + (size_t)ns * stage_bytes;
       float x[2][2][2];
       qk_tile<D, G, KB>(nxt, st, x, lane);
       pv_tile<D, G, VB>(cur + VOFF, st, pb, lane);
       softmax_tile<D, G>(st, x, pb);
       __syncwarp();
-      refill(j);
+      refill(j, cs);
+      cs = ns;
+      if (++ns == stages) {
+        ns = 0;
+        nph ^= 1;
+      }
       if (*abort_flag) {
         ok = false;
         break;
       }
     }
     if (ok) {
-      pv_tile<D, G, VB>(ring + (size_t)(j % stages) * stage_bytes + VOFF, st, pb, lane);
+      pv_tile<D, G, VB>(ring + (size_t)cs * stage_bytes + VOFF, st, pb, lane);
       __syncwarp();
       ++j;
     }
