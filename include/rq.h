@@ -38,16 +38,20 @@
  * kv-head) stream; all offsets in bytes; the format is this library's own):
  *   record = [K codes | K meta | V codes | V meta]
  *   codes  : 32 lanes x W words, W = ceil(D / cpw), cpw = 16, 10, 8, 4 codes
- *            per 32-bit word for b = 2, 3, 4, 8.  A word holds pairs of codes:
- *            slot p keeps one code at bit b*p and the other at bit 16 + b*p.
- *            Lane L = 4*gid + tig owns the elements of the 16x16 A-operand
- *            fragments of the m16n8k16 tensor-core MMA, pair (mb, kb, r):
- *              row = 16 mb + 8 (r&1) + gid, col = 16 kb + 8 (r>>1) + 2 tig + h
- *            K: row = token, col = channel; V: row = channel, col = token.
- *            Pairs are taken in quads (K: (mb, rr, group) over kb in the
- *            group and r in {rr, rr+2}; V: (mb, rr) over kb and r) and quads
- *            fill the lane's slots ordered by (class, word, slot) with
- *            slot classes b=2: 0,1,2,3,4,0,1,2; b=4: 0,1,0,1; b=3,8: 0.
+ *            per 32-bit word for b = 2, 3, 4, 8.  Lane L = 4*gid + tig owns
+ *            D/4 registers of four bytes e = 0..3: the 8-bit A-operand
+ *            fragments of the m16n8k32 integer tensor-core MMA.  Register
+ *            (rho, kh), rho in 0..D/8-1, kh in 0..1, byte e holds the code of
+ *              K: token gid + 8i, channel 32g + 16kh + 4tig + e, rho = i*D/32 + g
+ *              V: channel 16mb + 8rh + gid, token 4kh + tig + 8e,  rho = 2mb + rh
+ *            Row group rho has class j = rho mod C (C = 4, 2, 2, 1 for
+ *            b = 2, 3, 4, 8) and source sigma = 2*(rho / C) + kh: the code
+ *            sits at bits 8e + b*j .. 8e + b*j + b - 1 of word sigma, so the
+ *            word masked to those bits of every byte reads code * 2^(b*j).
+ *            b = 3, sigma >= W: source W + q is the top bit pair (bits 6, 7 of
+ *            each byte) of words 3q, 3q+1, 3q+2; code bit k of class j, byte e
+ *            is bit 8e + 6 + (f%2) of word 3q + f/2, f = 3j + k; unused top
+ *            bits are zero.
  *            Word w of lane L lives at ((w/4)*32 + L)*16 + (w%4)*4 for
  *            w < 4*floor(W/4), else floor(W/4)*512 + ((w - 4 floor(W/4))*32 + L)*4.
  *   meta   : u32 = fp16 scale | bf16 zero << 16.  K: D/32 groups x 32 entries,

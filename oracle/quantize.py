@@ -29,32 +29,38 @@ stream), byte layout:
 
     [K code blob][K meta][V code blob][V meta]
 
-Code blobs.  Each of the 32 lanes of a blob owns D/2 *pairs* of codes; a pair
-is two codes that share a 32-bit word, the first at bit b*p, the second at bit
-16 + b*p (slot p of the word).  The pairs a lane owns are the elements of the
-16x16 "A" operand fragments of an m16n8k16 tensor-core multiply-accumulate:
+Code blobs.  Each of the 32 lanes (lane = 4*gid + tig) of a blob owns D/4
+registers of four byte lanes e = 0..3, laid out as the 8-bit "A" operand
+fragments of the m16n8k32 integer tensor-core multiply-accumulate.  Register
+(rho, kh) -- row group rho in 0..D/8-1, half kh in 0..1 -- holds in byte e:
 
-    lane = 4*gid + tig;   pair (mb, kb, r), r in 0..3
-    row = 16*mb + 8*(r & 1) + gid
-    col = 16*kb + 8*(r >> 1) + 2*tig + h    (h = 0 first code, h = 1 second)
+    K blob: rho = i*(D/32) + g            code of token t = gid + 8*i,
+                                          channel d = 32*g + 16*kh + 4*tig + e
+    V blob: rho = 2*mb + rh               code of channel d = 16*mb + 8*rh + gid,
+                                          token t = 4*kh + tig + 8*e
 
-    K blob: row = token (mb in 0..1),  col = channel (kb in 0..D/16-1)
-    V blob: row = channel (mb in 0..D/16-1), col = token (kb in 0..1)
+(the V token order is the order in which the softmax probabilities of a tile
+arrive in the "B" fragment of the P.V product).  Row group rho has class
+j = rho mod C and both its registers come from source sigma = 2*(rho // C) + kh,
+with C = 4, 2, 2, 1 classes for b = 2, 3, 4, 8.  A register of class j is the
+source word masked to the bits [b*j, b*j + b) of each of its four bytes, so
+every byte reads as code * 2^(b*j) and one factor 2^(-b*j) per row group
+undoes the position.
 
-Pairs are grouped in quads of four.  K quad Q = (mb*2 + rr)*(D/32) + grp holds
-the pairs (mb, 2grp + kk, rr + 2ch) for u = 2kk + ch; V quad Q = mb*2 + rr
-holds (mb, kb, rr + 2ch) for u = 2kb + ch.  Quad Q occupies entries
-4Q .. 4Q+3 of the lane's slot list, which orders the W = ceil(D / cpw) words'
-slots by (class, word, slot) with the per-slot class
+    b = 2, 4, 8: source sigma is word sigma; the code of byte e occupies bits
+                 8e + b*j .. 8e + b*j + b - 1.
+    b = 3:       W = ceil(D/10) words (ten codes per word, as dense as 10 per
+                 u32).  Source sigma < W is word sigma, code at bits
+                 8e + 3j .. 8e + 3j + 2.  Source sigma = W + q is assembled
+                 from the two top bits (6, 7) of each byte of words 3q, 3q+1,
+                 3q+2: bit k of the class-j code of byte e is bit
+                 8e + 6 + (f mod 2) of word 3q + f // 2, f = 3j + k.  The top
+                 bits of the remaining words are zero.
 
-    b = 2: [0,1,2,3,4,0,1,2]   b = 4: [0,1,0,1]   b = 3, 8: all 0
-
-(cpw = codes per word = 16, 10, 8, 4 for b = 2, 3, 4, 8).  The class is the
-number of b-bit steps a code sits above the lowest position it can be read
-from in place inside an fp16 mantissa; grouping equal classes into a quad lets
-one scale factor per quad undo the position.  Unused slots (b = 3) are zero.
-Word w of lane L is stored at byte ((w // 4) * 32 + L) * 16 + (w % 4) * 4 for
-w < 4*floor(W/4), else at floor(W/4)*512 + ((w - 4*floor(W/4)) * 32 + L) * 4.
+A blob has W = ceil(D / cpw) words per lane (cpw = 16, 10, 8, 4 codes per word
+for b = 2, 3, 4, 8).  Word w of lane L is stored at byte
+((w // 4) * 32 + L) * 16 + (w % 4) * 4 for w < 4*floor(W/4), else at
+floor(W/4)*512 + ((w - 4*floor(W/4)) * 32 + L) * 4.
 
 Metadata entries are u32 = fp16 bits of s | bf16 bits of z << 16.
     K meta: D/32 groups x 32 entries; entry i of group grp is token
@@ -71,7 +77,6 @@ import numpy as np
 
 TILE = 32  # tokens per quantized tile == group size g
 CPW = {2: 16, 3: 10, 4: 8, 8: 4}
-SLOT_CLASS = {2: [0, 1, 2, 3, 4, 0, 1, 2], 3: [0] * 5, 4: [0, 1, 0, 1], 8: [0, 0]}
 
 
 # ---------------------------------------------------------------- bf16 helpers
@@ -159,66 +164,70 @@ def dequantize_tile(q: dict) -> tuple[np.ndarray, np.ndarray]:
 
 
 # --------------------------------------------------------------- pack format
+CLASSES = {2: 4, 3: 2, 4: 2, 8: 1}
+
+
 def words_per_lane(b: int, head_dim: int) -> int:
     return -(-head_dim // CPW[b])
 
 
-def _sorted_slots(b: int, n_words: int):
-    slots = [(SLOT_CLASS[b][p], w, p) for w in range(n_words) for p in range(CPW[b] // 2)]
-    slots.sort()
-    return [(w, p) for _, w, p in slots]
+def word_byte(n_words: int, lane: int, w: int) -> int:
+    full4 = 4 * (n_words // 4)
+    if w < full4:
+        return ((w // 4) * 32 + lane) * 16 + (w % 4) * 4
+    return (n_words // 4) * 512 + ((w - full4) * 32 + lane) * 4
 
 
-def _lane_pairs(role: str, head_dim: int):
-    """The lane-independent list of (mb, kb, r) in quad order (quad-major)."""
+def code_bit_positions(b: int, head_dim: int, rho: int, kh: int, e: int):
+    """(word, bit) of bits 0..b-1 of the code in byte e of register (rho, kh)."""
+    n_words = words_per_lane(b, head_dim)
+    c = CLASSES[b]
+    j, sigma = rho % c, 2 * (rho // c) + kh
+    if b != 3 or sigma < n_words:
+        return [(sigma, 8 * e + b * j + k) for k in range(b)]
+    q = sigma - n_words
     out = []
-    if role == "K":
-        for mb in range(2):
-            for rr in range(2):
-                for grp in range(head_dim // 32):
-                    for kk in range(2):
-                        for ch in range(2):
-                            out.append((mb, 2 * grp + kk, rr + 2 * ch))
-    elif role == "V":
-        for mb in range(head_dim // 16):
-            for rr in range(2):
-                for kb in range(2):
-                    for ch in range(2):
-                        out.append((mb, kb, rr + 2 * ch))
-    else:
-        raise ValueError(role)
+    for k in range(3):
+        f = 3 * j + k
+        out.append((3 * q + f // 2, 8 * e + 6 + f % 2))
     return out
+
+
+def fragment_coords(role: str, head_dim: int, lane: int, rho: int, kh: int, e: int):
+    """(row, col) of the code in byte e of register (rho, kh) of a lane.
+    K: (token, channel); V: (channel, token)."""
+    gid, tig = lane >> 2, lane & 3
+    if role == "K":
+        ng = head_dim // 32
+        i, g = rho // ng, rho % ng
+        return gid + 8 * i, 32 * g + 16 * kh + 4 * tig + e
+    if role == "V":
+        mb, rh = rho // 2, rho % 2
+        return 16 * mb + 8 * rh + gid, 4 * kh + tig + 8 * e
+    raise ValueError(role)
 
 
 @lru_cache(maxsize=None)
 def pack_table(role: str, b: int, head_dim: int):
     """Scatter table for one code blob.
 
-    Returns (rows, cols, word_byte, bit) arrays of length 32 * head_dim * 32 / 32
-    = 32 * D: for every code of the tile, the fragment row/col it holds, the
-    byte offset of its 32-bit word inside the blob and its bit offset.
+    Returns (rows, cols, word_byte, bit): rows/cols [32 * D] give the fragment
+    coordinates of every code of the tile; word_byte/bit [32 * D, b] give, for
+    each bit k of that code, the byte offset of its 32-bit word inside the
+    blob and the bit offset inside the word.
     """
     n_words = words_per_lane(b, head_dim)
-    slots = _sorted_slots(b, n_words)
-    pairs = _lane_pairs(role, head_dim)
-    assert len(pairs) == head_dim // 2 and len(slots) >= len(pairs)
-    full4 = 4 * (n_words // 4)
     rows, cols, wbyte, bit = [], [], [], []
     for lane in range(32):
-        gid, tig = lane >> 2, lane & 3
-        for j, (mb, kb, r) in enumerate(pairs):
-            w, p = slots[j]
-            if w < full4:
-                off = ((w // 4) * 32 + lane) * 16 + (w % 4) * 4
-            else:
-                off = (n_words // 4) * 512 + ((w - full4) * 32 + lane) * 4
-            row = 16 * mb + 8 * (r & 1) + gid
-            for h in range(2):
-                col = 16 * kb + 8 * (r >> 1) + 2 * tig + h
-                rows.append(row)
-                cols.append(col)
-                wbyte.append(off)
-                bit.append(16 * h + b * p)
+        for rho in range(head_dim // 8):
+            for kh in range(2):
+                for e in range(4):
+                    r, c = fragment_coords(role, head_dim, lane, rho, kh, e)
+                    pos = code_bit_positions(b, head_dim, rho, kh, e)
+                    rows.append(r)
+                    cols.append(c)
+                    wbyte.append([word_byte(n_words, lane, w) for w, _ in pos])
+                    bit.append([bt for _, bt in pos])
     return (np.array(rows), np.array(cols), np.array(wbyte), np.array(bit))
 
 
@@ -235,15 +244,18 @@ def pack_blob(codes_rc: np.ndarray, role: str, b: int) -> np.ndarray:
     head_dim = c.shape[2] if role == "K" else c.shape[1]
     rows, cols, wbyte, bit = pack_table(role, b, head_dim)
     n_words = blob_bytes(b, head_dim) // 4
-    # codes never overlap inside a word, so OR == sum over the codes of a word
-    vals = c[:, rows, cols].astype(np.uint64) << bit.astype(np.uint64)
-    words = np.zeros((c.shape[0], n_words), dtype=np.uint64)
-    order = np.argsort(wbyte, kind="stable")
-    w_sorted = wbyte[order] // 4
-    starts = np.searchsorted(w_sorted, np.arange(n_words))
+    codes = c[:, rows, cols].astype(np.uint64)  # [n, codes]
+    # every code bit lands on its own (word, bit): OR == sum over a word
+    ks = np.arange(b, dtype=np.uint64)
+    vals = ((codes[:, :, None] >> ks) & np.uint64(1)) << bit.astype(np.uint64)[None]  # [n, codes, b]
+    widx = (wbyte // 4).reshape(-1)
+    vals = vals.reshape(c.shape[0], -1)
+    order = np.argsort(widx, kind="stable")
+    w_sorted = widx[order]
     present = np.unique(w_sorted)
-    sums = np.add.reduceat(vals[:, order], starts[present], axis=1)
-    words[:, present] = sums
+    starts = np.searchsorted(w_sorted, present)
+    words = np.zeros((c.shape[0], n_words), dtype=np.uint64)
+    words[:, present] = np.add.reduceat(vals[:, order], starts, axis=1)
     out = words.astype(np.uint32).view(np.uint8)
     return out[0] if single else out
 
@@ -252,9 +264,11 @@ def unpack_blob(blob: np.ndarray, role: str, b: int, head_dim: int) -> np.ndarra
     """Inverse of pack_blob: returns codes in fragment coordinates."""
     rows, cols, wbyte, bit = pack_table(role, b, head_dim)
     words = np.asarray(blob, dtype=np.uint8).view(np.uint32)
+    bits = (words[wbyte // 4] >> bit.astype(np.uint32)) & np.uint32(1)  # [codes, b]
+    vals = (bits << np.arange(b, dtype=np.uint32)[None]).sum(axis=1)
     shape = (TILE, head_dim) if role == "K" else (head_dim, TILE)
     out = np.zeros(shape, dtype=np.uint8)
-    out[rows, cols] = ((words[wbyte // 4] >> bit.astype(np.uint32)) & ((1 << b) - 1)).astype(np.uint8)
+    out[rows, cols] = vals.astype(np.uint8)
     return out
 
 

@@ -115,23 +115,92 @@ def test_pack_table_is_a_bijection(role, b, d):
     seen = np.zeros(shape, dtype=np.int64)
     np.add.at(seen, (rows, cols), 1)
     assert np.all(seen == 1)
-    # no two codes share bits of a word
-    occ = set()
-    for wb, bt in zip(wbyte.tolist(), bit.tolist()):
-        for k in range(b):
-            key = (wb, bt + k)
-            assert key not in occ
-            occ.add(key)
-        assert (bt % 16) + b <= 16
-    assert wbyte.max() < qz.blob_bytes(b, d)
-    # slots of one quad share one class (4 pairs = 8 codes per quad per lane)
-    cls = qz.SLOT_CLASS[b]
-    per_lane = d  # codes per lane
+    # no two code bits share a bit of a word; every bit stays inside the blob
+    keys = set(zip(wbyte.reshape(-1).tolist(), bit.reshape(-1).tolist()))
+    assert len(keys) == wbyte.size
+    assert wbyte.max() < qz.blob_bytes(b, d) and bit.min() >= 0 and bit.max() < 32
+    # the blob has no more room than its codes need, up to the 3-bit padding
+    assert qz.blob_bytes(b, d) * 8 - 32 * d * b == (0 if b != 3 else 32 * (32 * qz.words_per_lane(3, d) - 3 * d))
+
+
+def _extract_registers(blob, b, d):
+    """Model of the decode-side unpacking: for every lane and register
+    (rho, kh), mask the source word to the class bits of each byte (3-bit top
+    sources are first assembled from the top bits of three words).  Returns
+    uint8 [32, D/8, 2, 4] byte values."""
+    words = np.asarray(blob, dtype=np.uint8).view(np.uint32).astype(np.int64)
+    nw = qz.words_per_lane(b, d)
+    c = qz.CLASSES[b]
+    out = np.zeros((32, d // 8, 2, 4), dtype=np.int64)
     for lane in range(32):
-        sl = slice(lane * per_lane, (lane + 1) * per_lane)
-        p = (bit[sl] % 16) // b
-        for qd in range(per_lane // 8):
-            assert len({cls[x] for x in p[qd * 8 : (qd + 1) * 8]}) == 1
+        wl = [int(words[qz.word_byte(nw, lane, w) // 4]) for w in range(nw)]
+        for rho in range(d // 8):
+            for kh in range(2):
+                j, sigma = rho % c, 2 * (rho // c) + kh
+                if b == 3 and sigma >= nw:
+                    q = sigma - nw
+                    src = ((wl[3 * q] >> 6) & 0x03030303) | ((wl[3 * q + 1] >> 4) & 0x0C0C0C0C) | (
+                        (wl[3 * q + 2] >> 2) & 0x30303030)
+                else:
+                    src = wl[sigma]
+                mask = (((1 << b) - 1) * 0x01010101) & 0xFFFFFFFF
+                reg = src & ((mask << (b * j)) & 0xFFFFFFFF)
+                for e in range(4):
+                    out[lane, rho, kh, e] = (reg >> (8 * e)) & 0xFF
+    return out
+
+
+@pytest.mark.parametrize("role", ["K", "V"])
+@pytest.mark.parametrize("b", BITS)
+@pytest.mark.parametrize("d", [64, 128])
+def test_masked_registers_read_code_times_class_factor(role, b, d):
+    """Each byte of a masked register equals code * 2^(b*j) of the code the
+    table places there (fits a u8), and every row group's two registers share
+    one class -- the property the integer tensor-core path relies on."""
+    rng = np.random.default_rng(b * 1000 + d + (role == "V"))
+    shape = (32, d) if role == "K" else (d, 32)
+    codes = rng.integers(0, 1 << b, size=shape, dtype=np.uint8)
+    regs = _extract_registers(qz.pack_blob(codes, role, b), b, d)
+    c = qz.CLASSES[b]
+    for lane in range(32):
+        for rho in range(d // 8):
+            f = 1 << (b * (rho % c))
+            for kh in range(2):
+                for e in range(4):
+                    r, col = qz.fragment_coords(role, d, lane, rho, kh, e)
+                    assert regs[lane, rho, kh, e] == int(codes[r, col]) * f
+                    assert regs[lane, rho, kh, e] <= 255
+
+
+def test_fragment_products_reproduce_the_dot_products():
+    """Integer model of one tile's two MMAs built from the registers alone:
+    sum over fragments of (register byte / class factor) * operand equals the
+    plain q.K^T and P.V products of the codes (K: token x channel, V: channel
+    x token, P in the V token order of the format)."""
+    rng = np.random.default_rng(7)
+    d, b = 128, 2
+    kc = rng.integers(0, 4, size=(32, d), dtype=np.uint8)
+    vc = rng.integers(0, 4, size=(d, 32), dtype=np.uint8)
+    q = rng.integers(-127, 128, size=d).astype(np.int64)
+    p = rng.integers(0, 256, size=32).astype(np.int64)
+    kr = _extract_registers(qz.pack_blob(kc, "K", b), b, d)
+    vr = _extract_registers(qz.pack_blob(vc, "V", b), b, d)
+    c = qz.CLASSES[b]
+    s_k = np.zeros(32, dtype=np.int64)
+    o_v = np.zeros(d, dtype=np.int64)
+    for lane in range(32):
+        gid, tig = lane >> 2, lane & 3
+        for rho in range(d // 8):
+            f = 1 << (b * (rho % c))
+            for kh in range(2):
+                for e in range(4):
+                    # K: B operand of byte e of a k32 fragment is channel 32g + 16kh + 4tig + e
+                    g = rho % (d // 32)
+                    s_k[gid + 8 * (rho // (d // 32))] += (kr[lane, rho, kh, e] // f) * q[32 * g + 16 * kh + 4 * tig + e]
+                    # V: B operand k = 16kh + 4tig + e holds token 4kh + tig + 8e
+                    o_v[16 * (rho // 2) + 8 * (rho % 2) + gid] += (vr[lane, rho, kh, e] // f) * p[4 * kh + tig + 8 * e]
+    assert np.array_equal(s_k, kc.astype(np.int64) @ q)
+    assert np.array_equal(o_v, vc.astype(np.int64) @ p)
 
 
 def test_pack_positions_golden():
@@ -140,7 +209,8 @@ def test_pack_positions_golden():
         rows, cols, wbyte, bit = qz.pack_table(c["role"], c["bits"], c["head_dim"])
         idx = np.nonzero((rows == c["row"]) & (cols == c["col"]))[0]
         assert idx.size == 1
-        assert (int(wbyte[idx[0]]), int(bit[idx[0]])) == (c["byte"], c["bit"]), c["why"]
+        got = [[int(a), int(t)] for a, t in zip(wbyte[idx[0]], bit[idx[0]])]
+        assert got == c["positions"], c["why"]
 
 
 def test_meta_permutations():
