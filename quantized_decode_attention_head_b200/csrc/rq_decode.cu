@@ -34,25 +34,36 @@ namespace rq {
 namespace {
 
 constexpr int NW = kDecodeConsumerWarps;
-constexpr int kMaxStages = 8;  // per-warp ring depth limit
-constexpr float kRescaleSlack = 8.0f;
+constexpr int kMaxStages = 8;                // per-warp ring depth limit
+constexpr uint32_t kBiasBits = 0x4B400000u;  // bits of 1.5 * 2^23
+constexpr float kBias = 12582912.0f;         // 1.5 * 2^23
+constexpr float kPScale = 65535.0f;          // P in 16-bit fixed point: p_int = rint(p * 65535)
+constexpr float kQMax = 32639.0f;            // q_int in [-32639, 32639] = 256 * q1 + q2, q1, q2 in s8
 
 template <int D, int G>
 struct Cfg {
-  static constexpr int NG = D / 32;      // K groups per token
-  static constexpr int GPS = 8 / G;      // groups sharing one 8-column accumulator
-  static constexpr int NSET = (NG + GPS - 1) / GPS;
-  static constexpr int PART = G * D + 2 * G;  // floats per partial state
+  static constexpr int NG = D / 32;                  // K groups per token (one k32 MMA each)
+  static constexpr int NB = (G + 3) / 4;             // 8-column blocks: 4 heads x 2 terms
+  static constexpr int HB = G < 4 ? G : 4;           // heads per block
+  static constexpr int PART = G * D + 2 * G;         // floats per partial state
+  static constexpr int KMW = NG;                     // K meta words converted per lane
+  static constexpr int VMW = D / 32;                 // V meta words converted per lane
+  static constexpr int KSTR = NG * 8 + 4;            // floats per gid row of the K scale scratch
+  static constexpr int VSTR = (D / 8) * 2 + 4;       // floats per gid row of the V scale scratch
+  static constexpr int SCRATCH = 8 * (KSTR + VSTR);  // floats per warp
 };
 
+// Per-warp state.  Thread (gid, tig) owns, in block nb, head 4nb + tig of the
+// MMA results (columns 2 tig, 2 tig + 1 = the two terms of that head).
 template <int D, int G>
 struct WarpState {
-  static constexpr int KE = G == 1 ? 2 : 1;  // column parities with distinct K groups
-  uint32_t qb[D / 16][2];                    // q B-fragments (fp16, scaled by 2^kq)
-  float ksf[2][2][Cfg<D, G>::NSET][KE];      // 2^(24 - kq - b*class) * softmax scale * log2(e)
-  float qsum[Cfg<D, G>::NSET][2];            // softmax-scaled sum of q over (group, head) columns
-  float m[2], l[2];                          // running max (log2 units) / sum per column parity
-  float o[D / 16][4];                        // P.V accumulators (x 2^-24), out^T fragment layout
+  using C = Cfg<D, G>;
+  uint32_t qb[C::NB][C::NG][2];  // q B-fragments: column n = 2 h + term, bytes = s8 terms
+  float qz[C::NB][C::NG];        // sum of q_int over group g -- zero-point term
+  float xs[C::NB];               // sq * softmax scale * log2(e)
+  float m[C::NB], l[C::NB];      // running max (log2 units) and sum of p (x 65535)
+  float o[C::NB][D / 16][2];     // channel 16 mb + 8 rh + gid (x 65535)
+  float kf[C::KMW], vf[C::VMW];  // class factors 2^(-b j) of the meta words this lane converts
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -68,74 +79,87 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 
-template <int D, int G, int KB>
+// q of the G heads -> per-head 16-bit fixed point (sq = max|q_h| / 32639)
+// split into two s8 terms q_int = 256 q1 + q2, laid out as the k32 x n8
+// B-fragments of the q.K^T MMA (column n = 2 * head + term).
+template <int D, int G, int KB, int VB>
 __device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, float scale_log2, int lane) {
   using C = Cfg<D, G>;
-  constexpr int WK = words_per_lane(KB, D);
   const int gid = lane >> 2, tig = lane & 3;
-  const int bh = gid % G;          // head of B column n = gid
-  const int bgl = gid / G;         // group slot of B column n = gid
-  uint32_t raw[D / 16][2];
-  float mx = 0.0f;
+  const int hl = gid >> 1, tau = gid & 1;
 #pragma unroll
-  for (int kb = 0; kb < D / 16; ++kb)
+  for (int nb = 0; nb < C::NB; ++nb) {
+    const bool hv = hl < C::HB;
+    const uint16_t* qp = qh + (size_t)(4 * nb + hl) * D;
+    float qv[C::NG][8];
+    float mx = 0.0f, ps[C::NG];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      raw[kb][j] = __ldg(reinterpret_cast<const uint32_t*>(qh + bh * D + 16 * kb + 8 * j + 2 * tig));
-      mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_float(raw[kb][j] & 0xFFFFu)), fabsf(bf16_bits_to_float(raw[kb][j] >> 16))));
-    }
-  mx = warp_max(mx);
-  int kq = 0;
-  if (mx > 0.0f) {
-    const int e = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126;  // mx < 2^e
-    kq = 15 - e;
-    kq = kq > 100 ? 100 : (kq < -100 ? -100 : kq);
-  }
-  const float up = pow2i(kq);
+    for (int g = 0; g < C::NG; ++g) {
+      ps[g] = 0.0f;
 #pragma unroll
-  for (int kb = 0; kb < D / 16; ++kb) {
-    const bool valid = ((kb / 2) % C::GPS) == bgl;
+      for (int kh = 0; kh < 2; ++kh) {
+        uint2 u = make_uint2(0u, 0u);
+        if (hv) u = __ldg(reinterpret_cast<const uint2*>(qp + 32 * g + 16 * kh + 4 * tig));
+        const uint32_t w[2] = {u.x, u.y};
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float lo = bf16_bits_to_float(raw[kb][j] & 0xFFFFu) * up;
-      const float hi = bf16_bits_to_float(raw[kb][j] >> 16) * up;
-      st.qb[kb][j] = valid ? pack_half2(lo, hi) : 0u;
-    }
-  }
-#pragma unroll
-  for (int s = 0; s < C::NSET; ++s)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int n = 2 * tig + e;
-      const int grp = s * C::GPS + n / G, h = n % G;
-      float acc = 0.0f;
-      if (grp < C::NG) {
-        const uint4* p = reinterpret_cast<const uint4*>(qh + h * D + grp * 32);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 u = __ldg(p + c);
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc += bf16_bits_to_float(w[k] & 0xFFFFu) + bf16_bits_to_float(w[k] >> 16);
+        for (int e = 0; e < 4; ++e) {
+          const float x = bf16_bits_to_float(e & 1 ? w[e >> 1] >> 16 : w[e >> 1] & 0xFFFFu);
+          qv[g][4 * kh + e] = x;
+          mx = fmaxf(mx, fabsf(x));
         }
       }
-      st.qsum[s][e] = acc * scale_log2;
-#pragma unroll
-      for (int mb = 0; mb < 2; ++mb)
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          if (e < WarpState<D, G>::KE) {
-            const int q = (mb * 2 + rr) * C::NG + (grp < C::NG ? grp : 0);
-            st.ksf[mb][rr][s][e] = pow2i(24 - kq - KB * quad_class(KB, WK, q)) * scale_log2;
-          }
-        }
     }
-  st.m[0] = st.m[1] = -INFINITY;
-  st.l[0] = st.l[1] = 0.0f;
+    // the four lanes of a quad hold all D channels of one head
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float inv = mx > 0.0f ? kQMax / mx : 0.0f;
+    const float sq = mx * (1.0f / kQMax);
 #pragma unroll
-  for (int mb = 0; mb < D / 16; ++mb)
+    for (int g = 0; g < C::NG; ++g)
 #pragma unroll
-    for (int r = 0; r < 4; ++r) st.o[mb][r] = 0.0f;
+      for (int kh = 0; kh < 2; ++kh) {
+        uint32_t packed = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          int qi = __float2int_rn(qv[g][4 * kh + e] * inv);
+          qi = qi > 32639 ? 32639 : (qi < -32639 ? -32639 : qi);
+          const int q1 = (qi + 128) >> 8;  // floor((qi + 128) / 256)
+          const int q2 = qi - (q1 << 8);   // in [-128, 127]
+          packed |= ((uint32_t)(tau ? q2 : q1) & 0xFFu) << (8 * e);
+          ps[g] += (float)qi;
+        }
+        st.qb[nb][g][kh] = hv ? packed : 0u;
+      }
+    // zero-point term: sum of the SAME rounded q_int over each group, so the
+    // code and zero terms together are exactly (s c + z) . q_int and the large
+    // cancellation between them (z = group minimum) leaves no rounding residue
+#pragma unroll
+    for (int g = 0; g < C::NG; ++g) {
+      ps[g] += __shfl_xor_sync(0xffffffffu, ps[g], 1);
+      ps[g] += __shfl_xor_sync(0xffffffffu, ps[g], 2);
+    }
+    // the result columns of thread (gid, tig) belong to head 4nb + tig, whose
+    // statistics live in lane 8 tig (gid = 2 tig, term 0)
+    const float sq_c = __shfl_sync(0xffffffffu, sq, 8 * tig);
+#pragma unroll
+    for (int g = 0; g < C::NG; ++g) st.qz[nb][g] = __shfl_sync(0xffffffffu, ps[g], 8 * tig);
+    st.xs[nb] = sq_c * scale_log2;
+    st.m[nb] = -INFINITY;
+    st.l[nb] = 0.0f;
+#pragma unroll
+    for (int mb = 0; mb < D / 16; ++mb) st.o[nb][mb][0] = st.o[nb][mb][1] = 0.0f;
+  }
+  // class factors of the metadata words this lane converts (see convert_meta)
+#pragma unroll
+  for (int k = 0; k < C::KMW; ++k) {
+    const int w = C::KMW * lane + k, g = w / 32, i = (w % 32) % 4;
+    st.kf[k] = pow2i(-KB * reg_class(KB, i * C::NG + g));
+  }
+#pragma unroll
+  for (int k = 0; k < C::VMW; ++k) {
+    const int w = C::VMW * lane + k, rho = w % (D / 8);
+    st.vf[k] = pow2i(-VB * reg_class(VB, rho));
+  }
 }
 
 template <int W>
@@ -156,180 +180,192 @@ __device__ __forceinline__ float half_lo_to_float(uint32_t m) {
   return __half2float(__ushort_as_half((unsigned short)(m & 0xFFFFu)));
 }
 
-// q.K^T of one tile -> logits x[mb][rr][e] (log2 units, softmax scale applied)
-// for tokens 16mb + 8rr + gid and heads (2 tig + e) % G.
+// Metadata of one tile -> (scale * 2^(-b j), zero) float pairs in the warp's
+// scratch, each entry converted once.  K: scratch[gid][g][i] for token
+// gid + 8 i; V: scratch[gid][rho] for channel 16 (rho/2) + 8 (rho%2) + gid.
+template <int D, int G, int KB, int VB>
+__device__ __forceinline__ void convert_meta(const uint8_t* rec, const WarpState<D, G>& st, float* ks, float* vs,
+                                             int lane) {
+  using C = Cfg<D, G>;
+  const uint32_t* kmeta = reinterpret_cast<const uint32_t*>(rec + blob_bytes(KB, D));
+  const uint32_t* vmeta = reinterpret_cast<const uint32_t*>(rec + blob_bytes(KB, D) + 4 * D + blob_bytes(VB, D));
+  uint32_t km[C::KMW], vm[C::VMW];
+  if constexpr (C::KMW == 4) {
+    const uint4 u = *reinterpret_cast<const uint4*>(kmeta + 4 * lane);
+    km[0] = u.x, km[1] = u.y, km[2] = u.z, km[3] = u.w;
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(kmeta + 2 * lane);
+    km[0] = u.x, km[1] = u.y;
+  }
+  if constexpr (C::VMW == 4) {
+    const uint4 u = *reinterpret_cast<const uint4*>(vmeta + 4 * lane);
+    vm[0] = u.x, vm[1] = u.y, vm[2] = u.z, vm[3] = u.w;
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(vmeta + 2 * lane);
+    vm[0] = u.x, vm[1] = u.y;
+  }
+  float kv[2 * C::KMW], vv[2 * C::VMW];
+#pragma unroll
+  for (int k = 0; k < C::KMW; ++k) {
+    kv[2 * k] = half_lo_to_float(km[k]) * st.kf[k];
+    kv[2 * k + 1] = __uint_as_float(km[k] & 0xFFFF0000u);
+  }
+#pragma unroll
+  for (int k = 0; k < C::VMW; ++k) {
+    vv[2 * k] = half_lo_to_float(vm[k]) * st.vf[k];
+    vv[2 * k + 1] = __uint_as_float(vm[k] & 0xFFFF0000u);
+  }
+  // word w = KMW * lane + k: group w / 32, gid (w % 32) / 4, i = w % 4
+  {
+    const int w0 = C::KMW * lane;
+    float* dst = ks + ((w0 % 32) / 4) * C::KSTR + ((w0 / 32) * 4 + (w0 % 4)) * 2;
+#pragma unroll
+    for (int c = 0; c < C::KMW / 2; ++c)
+      *reinterpret_cast<float4*>(dst + 4 * c) = make_float4(kv[4 * c], kv[4 * c + 1], kv[4 * c + 2], kv[4 * c + 3]);
+  }
+  // word w = VMW * lane + k: gid w / (D/8), rho = w % (D/8)
+  {
+    const int w0 = C::VMW * lane;
+    float* dst = vs + (w0 / (D / 8)) * C::VSTR + (w0 % (D / 8)) * 2;
+#pragma unroll
+    for (int c = 0; c < C::VMW / 2; ++c)
+      *reinterpret_cast<float4*>(dst + 4 * c) = make_float4(vv[4 * c], vv[4 * c + 1], vv[4 * c + 2], vv[4 * c + 3]);
+  }
+}
+
+// q.K^T of one tile: raw scores acc[nb][i] (units sq, without the softmax
+// scale) for token gid + 8 i and head 4 nb + tig.  One k32 MMA per (token
+// half, group); its two term columns combine exactly in int32, and the
+// group's scale/zero apply to that exact integer sum.
 template <int D, int G, int KB>
-__device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G>& st, float (&x)[2][2][2], int lane) {
+__device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G>& st, const float* ks,
+                                        float (&acc)[Cfg<D, G>::NB][4], int lane) {
   using C = Cfg<D, G>;
   constexpr int W = words_per_lane(KB, D);
-  const int gid = lane >> 2, tig = lane & 3;
+  const int gid = lane >> 2;
   uint32_t kw[W];
   load_words<W>(kw, rec, lane);
-  float acc[C::NSET][2][4];
 #pragma unroll
-  for (int s = 0; s < C::NSET; ++s)
+  for (int nb = 0; nb < C::NB; ++nb)
 #pragma unroll
-    for (int mb = 0; mb < 2; ++mb)
+    for (int i = 0; i < 4; ++i) acc[nb][i] = 0.0f;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) acc[s][mb][r] = 0.0f;
+  for (int g = 0; g < C::NG; ++g)
 #pragma unroll
-  for (int mb = 0; mb < 2; ++mb)
-#pragma unroll
-    for (int kb = 0; kb < D / 16; ++kb) {
+    for (int mb = 0; mb < 2; ++mb) {
+      const float4 sz = *reinterpret_cast<const float4*>(ks + gid * C::KSTR + (g * 4 + 2 * mb) * 2);
       uint32_t a[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int idx = k_pair_index(D, mb, kb, r);
-        a[r] = extract_pair<KB>(kw, slot_word(KB, W, idx), slot_pos(KB, W, idx));
+      for (int r = 0; r < 4; ++r) a[r] = code_reg<KB, W>(kw, (2 * mb + (r & 1)) * C::NG + g, r >> 1);
+#pragma unroll
+      for (int nb = 0; nb < C::NB; ++nb) {
+        uint32_t c[4];
+        imma_u8s8(c, a, st.qb[nb][g][0], st.qb[nb][g][1], 0u);
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+          // |256 hi + lo| < 2^31: exact in int32, one rounding to fp32
+          const float v = (float)((int)c[2 * rh] * 256 + (int)c[2 * rh + 1]);
+          const float s = rh ? sz.z : sz.x, z = rh ? sz.w : sz.y;
+          acc[nb][2 * mb + rh] = fmaf(s, v, fmaf(z, st.qz[nb][g], acc[nb][2 * mb + rh]));
+        }
       }
-      mma_f16(acc[(kb / 2) / C::GPS][mb], a, st.qb[kb][0], st.qb[kb][1]);
-    }
-  const uint32_t* kmeta = reinterpret_cast<const uint32_t*>(rec + blob_bytes(KB, D));
-  float sc[2][2][2];
-#pragma unroll
-  for (int mb = 0; mb < 2; ++mb)
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) sc[mb][rr][0] = sc[mb][rr][1] = 0.0f;
-#pragma unroll
-  for (int s = 0; s < C::NSET; ++s)
-#pragma unroll
-    for (int e = 0; e < WarpState<D, G>::KE; ++e) {
-      // for G >= 2 both column parities of a thread share one K group
-      const int grp = s * C::GPS + (2 * tig + e) / G;
-      if (grp < C::NG) {
-        const uint4 mv = *reinterpret_cast<const uint4*>(kmeta + grp * 32 + gid * 4);
-        const uint32_t mw[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-        for (int mb = 0; mb < 2; ++mb)
-#pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const uint32_t m = mw[mb * 2 + rr];
-            const float sk = half_lo_to_float(m) * st.ksf[mb][rr][s][e];
-            const float z = __uint_as_float(m & 0xFFFF0000u);
-            if (G == 1) {
-              sc[mb][rr][e] = fmaf(sk, acc[s][mb][rr * 2 + e], fmaf(z, st.qsum[s][e], sc[mb][rr][e]));
-            } else {
-              sc[mb][rr][0] = fmaf(sk, acc[s][mb][rr * 2], fmaf(z, st.qsum[s][0], sc[mb][rr][0]));
-              sc[mb][rr][1] = fmaf(sk, acc[s][mb][rr * 2 + 1], fmaf(z, st.qsum[s][1], sc[mb][rr][1]));
-            }
-          }
-      }
-    }
-  // sum the group columns of each head across the quad of lanes sharing a row
-#pragma unroll
-  for (int mb = 0; mb < 2; ++mb)
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      float v0 = sc[mb][rr][0], v1 = sc[mb][rr][1];
-      if (G == 1) {
-        v0 += v1;
-        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
-        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
-        v1 = v0;
-      } else if (G == 2) {
-        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
-        v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
-        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
-        v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
-      } else if (G == 4) {
-        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
-        v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
-      }
-      x[mb][rr][0] = v0;
-      x[mb][rr][1] = v1;
     }
 }
 
-// Online softmax update; returns P as PV B-fragments pb[kb][rr].
+// Online softmax of one tile.  The probabilities are taken relative to the
+// running maximum m (p <= 1, 16-bit fixed point p_int = rint(65535 p)); m
+// moves -- and the state is rescaled -- only when a score of the tile exceeds
+// it, which after the first tiles is rare.  Returns the P B-fragments pb
+// (column n = 2 * head + term, term 0 = high byte).
 template <int D, int G>
-__device__ __forceinline__ void softmax_tile(WarpState<D, G>& st, const float (&x)[2][2][2], uint32_t (&pb)[2][2]) {
-  float tmax[2];
+__device__ __forceinline__ void softmax_tile(WarpState<D, G>& st, const float (&acc)[Cfg<D, G>::NB][4],
+                                             uint32_t (&pb)[Cfg<D, G>::NB][2], int lane) {
+  using C = Cfg<D, G>;
+  const int gid = lane >> 2, tig = lane & 3;
+  float x[C::NB][4];
+  bool grow = false;
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    float v = fmaxf(fmaxf(x[0][0][e], x[0][1][e]), fmaxf(x[1][0][e], x[1][1][e]));
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-    tmax[e] = v;
+  for (int nb = 0; nb < C::NB; ++nb) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[nb][i] = acc[nb][i] * st.xs[nb];
+    grow |= fmaxf(fmaxf(x[nb][0], x[nb][1]), fmaxf(x[nb][2], x[nb][3])) > st.m[nb];
   }
-  // Lazy rescale: the reference max only moves when a score exceeds it by
-  // more than kRescaleSlack (log2 units), so P <= 2^kRescaleSlack stays well
-  // inside fp16 and o is rescaled only a handful of times per work item.
-  const bool grow = tmax[0] > st.m[0] + kRescaleSlack || tmax[1] > st.m[1] + kRescaleSlack;
   if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float mn = fmaxf(st.m[e], tmax[e]);
-      const float alpha = ex2(st.m[e] - mn);
-      st.m[e] = mn;
-      st.l[e] *= alpha;
+    for (int nb = 0; nb < C::NB; ++nb) {
+      float v = fmaxf(fmaxf(x[nb][0], x[nb][1]), fmaxf(x[nb][2], x[nb][3]));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+      const float mn = fmaxf(st.m[nb], v);
+      const float alpha = ex2(st.m[nb] - mn);  // 0 while m = -inf
+      st.m[nb] = mn;
+      st.l[nb] *= alpha;
 #pragma unroll
       for (int mb = 0; mb < D / 16; ++mb) {
-        st.o[mb][e] *= alpha;
-        st.o[mb][2 + e] *= alpha;
+        st.o[nb][mb][0] *= alpha;
+        st.o[nb][mb][1] *= alpha;
       }
     }
   }
+  const int hl = gid >> 1;
+  const int src0 = 4 * tig + hl, src1 = 16 + 4 * tig + hl;
 #pragma unroll
-  for (int mb = 0; mb < 2; ++mb)
+  for (int nb = 0; nb < C::NB; ++nb) {
+    uint32_t y[4];
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr)
-      pb[mb][rr] = movmatrix_trans(pack_half2(ex2(x[mb][rr][0] - st.m[0]), ex2(x[mb][rr][1] - st.m[1])));
+    for (int i = 0; i < 4; ++i) y[i] = __float_as_uint(fmaf(ex2(x[nb][i] - st.m[nb]), kPScale, kBias));
+    // low 16 bits of y = p_int; byte e of hi/lo = token gid + 8e
+    const uint32_t u0 = __byte_perm(y[0], y[1], 0x5410), u1 = __byte_perm(y[2], y[3], 0x5410);
+    const uint32_t hi = __byte_perm(u0, u1, 0x7531), lo = __byte_perm(u0, u1, 0x6420);
+    // B element (k, n = gid): token 4 (k >> 4) + ((k >> 2) & 3) + 8 (k & 3),
+    // held by lane 4 * gid_src + head with gid_src = tig (k < 16) or tig + 4
+    const uint32_t h0 = __shfl_sync(0xffffffffu, hi, src0), l0 = __shfl_sync(0xffffffffu, lo, src0);
+    const uint32_t h1 = __shfl_sync(0xffffffffu, hi, src1), l1 = __shfl_sync(0xffffffffu, lo, src1);
+    const bool hv = hl < C::HB;
+    pb[nb][0] = hv ? ((gid & 1) ? l0 : h0) : 0u;
+    pb[nb][1] = hv ? ((gid & 1) ? l1 : h1) : 0u;
+  }
 }
 
+// P.V of one tile into the running state.  One k32 MMA per 16 channels; the
+// channel's scale/zero apply to the exact integer sum, and the zero term
+// needs sum_t p_t, which one more MMA with A = 1 delivers in the same layout.
 template <int D, int G, int VB>
-__device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st, const uint32_t (&pb)[2][2], int lane) {
+__device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st, const float* vs,
+                                        const uint32_t (&pb)[Cfg<D, G>::NB][2], int lane) {
+  using C = Cfg<D, G>;
   constexpr int W = words_per_lane(VB, D);
   const int gid = lane >> 2;
-  // sum_t p_t * 2^-24 per column: A = the fp16 subnormal 2^-24, so every
-  // accumulator below carries the same 2^-24 as the unpacked codes
-  float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  const uint32_t tiny[4] = {0x00010001u, 0x00010001u, 0x00010001u, 0x00010001u};
-  mma_f16(ps, tiny, pb[0][0], pb[0][1]);
-  mma_f16(ps, tiny, pb[1][0], pb[1][1]);
+  float ps[C::NB];
+  const uint32_t ones[4] = {0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u};
+#pragma unroll
+  for (int nb = 0; nb < C::NB; ++nb) {
+    uint32_t c[4];
+    imma_u8u8(c, ones, pb[nb][0], pb[nb][1], kBiasBits);
+    ps[nb] = fmaf(256.0f, __uint_as_float(c[0]) - kBias, __uint_as_float(c[1]) - kBias);
+    st.l[nb] += ps[nb];
+  }
   uint32_t vw[W];
   load_words<W>(vw, vrec, lane);
-  const uint32_t* vmeta = reinterpret_cast<const uint32_t*>(vrec + blob_bytes(VB, D)) + gid * (D / 8);
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
-    const uint4 mv = *reinterpret_cast<const uint4*>(vmeta + 4 * c);
-    const uint32_t mw[4] = {mv.x, mv.y, mv.z, mv.w};
+  for (int mb = 0; mb < D / 16; ++mb) {
+    const float4 sz = *reinterpret_cast<const float4*>(vs + gid * C::VSTR + 4 * mb);
+    uint32_t a[4];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int mb = 2 * c + half;
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int r = 0; r < 4; ++r) a[r] = code_reg<VB, W>(vw, 2 * mb + (r & 1), r >> 1);
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
-        uint32_t a[4];
+    for (int nb = 0; nb < C::NB; ++nb) {
+      uint32_t c[4];
+      imma_u8u8(c, a, pb[nb][0], pb[nb][1], 0u);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int idx = v_pair_index(mb, kb, r);
-          a[r] = extract_pair<VB>(vw, slot_word(VB, W, idx), slot_pos(VB, W, idx));
-        }
-        mma_f16(acc, a, pb[kb][0], pb[kb][1]);
-      }
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const uint32_t m = mw[half * 2 + rr];
-        const int cls = quad_class(VB, W, mb * 2 + rr);
-        float sv = half_lo_to_float(m);
-        if (cls) sv *= 1.0f / (float)(1 << (VB * cls));
-        const float z = __uint_as_float(m & 0xFFFF0000u);
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-          st.o[mb][rr * 2 + e] = fmaf(sv, acc[rr * 2 + e], fmaf(z, ps[e], st.o[mb][rr * 2 + e]));
+      for (int rh = 0; rh < 2; ++rh) {
+        const float v = (float)((int)c[2 * rh] * 256 + (int)c[2 * rh + 1]);
+        const float s = rh ? sz.z : sz.x, z = rh ? sz.w : sz.y;
+        st.o[nb][mb][rh] = fmaf(s, v, fmaf(z, ps[nb], st.o[nb][mb][rh]));
       }
     }
   }
-  st.l[0] += ps[0];
-  st.l[1] += ps[1];
-}
-
-template <int D, int G, int KB>
-__device__ __forceinline__ void score_tile(const uint8_t* rec, WarpState<D, G>& st, uint32_t (&pb)[2][2], int lane) {
-  float x[2][2][2];
-  qk_tile<D, G, KB>(rec, st, x, lane);
-  softmax_tile<D, G>(st, x, pb);
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
@@ -344,8 +380,9 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
 // warp and every warp keeps `stages` records in flight.
 template <int D, int G, int KB, int VB>
 __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log2, uint8_t* ring, int stages,
-                        int stage_bytes, uint64_t* bars, const uint8_t* src, int rec, int n_my, int warp, int lane,
-                        volatile int* abort_flag, int* status) {
+                        int stage_bytes, uint64_t* bars, float* scratch, const uint8_t* src, int rec, int n_my,
+                        int warp, int lane, volatile int* abort_flag, int* status) {
+  using C = Cfg<D, G>;
   const int n_w = n_my > warp ? (n_my - warp + NW - 1) / NW : 0;
   if (lane == 0) {
     for (int j = 0; j < stages && j < n_w; ++j) {
@@ -353,60 +390,37 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
       bulk_g2s(ring + (size_t)j * stage_bytes, src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec, &bars[j]);
     }
   }
-  setup_query<D, G, KB>(st, qh, scale_log2, lane);
-  // ring position of a tile: slot = j mod stages, parity = (j / stages) & 1,
-  // advanced incrementally (no integer division in the loop)
-  auto wait_slot = [&](int slot, int parity) -> bool {
-    return __all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], (uint32_t)parity));
-  };
-  auto refill = [&](int j, int slot) {  // the warp has finished reading tile j's slot
+  setup_query<D, G, KB, VB>(st, qh, scale_log2, lane);
+  float* ks = scratch;
+  float* vs = scratch + 8 * C::KSTR;
+  const int VOFF = blob_bytes(KB, D) + 4 * D;
+  int j = 0, slot = 0, parity = 0;  // ring position of tile j, advanced without division
+  bool ok = true;
+  for (; j < n_w; ++j) {
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], (uint32_t)parity));
+    if (!ok) break;
+    const uint8_t* cur = ring + (size_t)slot * stage_bytes;
+    convert_meta<D, G, KB, VB>(cur, st, ks, vs, lane);
+    __syncwarp();
+    float acc[C::NB][4];
+    qk_tile<D, G, KB>(cur, st, ks, acc, lane);
+    uint32_t pb[C::NB][2];
+    softmax_tile<D, G>(st, acc, pb, lane);
+    pv_tile<D, G, VB>(cur + VOFF, st, vs, pb, lane);
+    __syncwarp();  // every lane has finished reading the slot and the scratch
     if (lane == 0 && j + stages < n_w) {
       fence_proxy_async_smem();  // generic-proxy reads of the slot precede the async refill
       mbar_arrive_expect_tx(&bars[slot], (uint32_t)rec);
       bulk_g2s(ring + (size_t)slot * stage_bytes, src + (int64_t)(warp + (j + stages) * NW) * rec, (uint32_t)rec,
                &bars[slot]);
     }
-  };
-  const int VOFF = blob_bytes(KB, D) + 4 * D;
-  int j = 0;
-  bool ok = true;
-  if (n_w > 0) {
-    // software pipeline: the scores of tile j + 1 are computed in the same
-    // block as the P.V of tile j, so their MMA chains interleave
-    uint32_t pb[2][2];
-    int cs = 0;             // slot of tile j
-    int ns = 1, nph = 0;    // slot and parity of tile j + 1
-    if (ns == stages) {
-      ns = 0;
-      nph = 1;
+    if (++slot == stages) {
+      slot = 0;
+      parity ^= 1;
     }
-    ok = wait_slot(0, 0);
-    if (ok) score_tile<D, G, KB>(ring, st, pb, lane);
-    for (; ok && j + 1 < n_w; ++j) {
-      ok = wait_slot(ns, nph);
-      if (!ok) break;
-      const uint8_t* cur = ring + (size_t)cs * stage_bytes;
-      const uint8_t* nxt = ring + (size_t)ns * stage_bytes;
-      float x[2][2][2];
-      qk_tile<D, G, KB>(nxt, st, x, lane);
-      pv_tile<D, G, VB>(cur + VOFF, st, pb, lane);
-      softmax_tile<D, G>(st, x, pb);
-      __syncwarp();
-      refill(j, cs);
-      cs = ns;
-      if (++ns == stages) {
-        ns = 0;
-        nph ^= 1;
-      }
-      if (*abort_flag) {
-        ok = false;
-        break;
-      }
-    }
-    if (ok) {
-      pv_tile<D, G, VB>(ring + (size_t)cs * stage_bytes + VOFF, st, pb, lane);
-      __syncwarp();
-      ++j;
+    if (*abort_flag) {
+      ok = false;
+      break;
     }
   }
   if (!ok) {
@@ -421,11 +435,12 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
 template <int D, int G>
 __device__ __forceinline__ void consume_dispatch(int kb, int vb, WarpState<D, G>& st, const uint16_t* qh,
                                                  float scale_log2, uint8_t* ring, int stages, int stage_bytes,
-                                                 uint64_t* bars, const uint8_t* src, int rec, int n_my, int warp,
-                                                 int lane, volatile int* abort_flag, int* status) {
-#define RQ_C(KBV, VBV)                                                                                           \
-  consume<D, G, KBV, VBV>(st, qh, scale_log2, ring, stages, stage_bytes, bars, src, rec, n_my, warp, lane, abort_flag, \
-                          status)
+                                                 uint64_t* bars, float* scratch, const uint8_t* src, int rec,
+                                                 int n_my, int warp, int lane, volatile int* abort_flag,
+                                                 int* status) {
+#define RQ_C(KBV, VBV)                                                                                       \
+  consume<D, G, KBV, VBV>(st, qh, scale_log2, ring, stages, stage_bytes, bars, scratch, src, rec, n_my, warp, \
+                          lane, abort_flag, status)
 #define RQ_V(KBV)                  \
   switch (vb) {                    \
     case 2: RQ_C(KBV, 2); break;   \
@@ -443,21 +458,24 @@ __device__ __forceinline__ void consume_dispatch(int kb, int vb, WarpState<D, G>
 #undef RQ_C
 }
 
-// Canonical partial of one warp in shared memory: o[G][D], m[G], l[G].
+// Canonical partial of one warp in shared memory: o[G][D], m[G], l[G], with
+// o and l back in units of p (the tile path keeps them x 65535).
 template <int D, int G>
 __device__ void dump_tile_state(const WarpState<D, G>& st, float* slot, int lane) {
+  using C = Cfg<D, G>;
   const int gid = lane >> 2, tig = lane & 3;
+  constexpr float inv = 1.0f / kPScale;
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int n = 2 * tig + e;
-    if (n < G) {
+  for (int nb = 0; nb < C::NB; ++nb) {
+    const int h = 4 * nb + tig;
+    if (tig < C::HB) {
 #pragma unroll
       for (int mb = 0; mb < D / 16; ++mb)
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) slot[n * D + 16 * mb + 8 * rr + gid] = st.o[mb][rr * 2 + e] * 16777216.0f;
+        for (int rh = 0; rh < 2; ++rh) slot[h * D + 16 * mb + 8 * rh + gid] = st.o[nb][mb][rh] * inv;
       if (gid == 0) {
-        slot[G * D + n] = st.m[e];
-        slot[G * D + G + n] = st.l[e] * 16777216.0f;
+        slot[G * D + h] = st.m[nb];
+        slot[G * D + G + h] = st.l[nb] * inv;
       }
     }
   }
@@ -641,7 +659,7 @@ __device__ void combine_partials(const float* base, int n, float* dst, float* ou
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a) {
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[NW * kMaxStages];
@@ -651,12 +669,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int srel = blockIdx.y, item = blockIdx.x;
   const int NI = a.n_splits + a.n_win;  // work items of this stream
-  const int NG = (NI + kGroup - 1) / kGroup;
   const int h = srel % a.g.Hkv, b = (srel / a.g.Hkv) % a.g.B, lrel = srel / (a.g.Hkv * a.g.B);
   const int l = a.layer0 + lrel;
   const HeadDesc hd = a.desc[l * a.g.Hkv + h];
   const uint16_t* qh = a.q + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  float* merge = reinterpret_cast<float*>(smem);  // aliases the stages after the main loop
+  // dynamic shared memory: [per-warp scale scratch][stages | merge + window]
+  uint8_t* area = smem + (size_t)NW * C::SCRATCH * 4;
+  float* merge = reinterpret_cast<float*>(area);  // aliases the stages after the main loop
 
   if (tid == 0) {
     abort_flag = 0;
@@ -670,13 +689,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a)
   if (tiles_item) {
     const int t0 = (int)(((int64_t)item * a.n_tiles) / a.n_splits);
     const int t1 = (int)(((int64_t)(item + 1) * a.n_tiles) / a.n_splits);
-    const int n_my = t1 - t0;
     const int rec = hd.rec_bytes;
     const uint8_t* src = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)t0 * rec;
     if (warp < NW)
       consume_dispatch<D, G>(hd.k_bits, hd.v_bits, st, qh, a.scale_log2,
-                             smem + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
-                             bars + warp * kMaxStages, src, rec, n_my, warp, lane, &abort_flag, a.status);
+                             area + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
+                             bars + warp * kMaxStages, reinterpret_cast<float*>(smem) + warp * C::SCRATCH, src, rec,
+                             t1 - t0, warp, lane, &abort_flag, a.status);
   } else {
     // one 32-token chunk of the bf16 sink + recent window
     const uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
@@ -688,8 +707,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a)
   __syncthreads();
   if (abort_flag) return;
 
-  // merge the four warps' partial states into this item's partial
-  float* part = a.partials + ((size_t)srel * NI + item) * C::PART;
+  // merge the warps' partial states into this item's partial
+  float* ps = a.partials + (size_t)srel * NI * C::PART;
+  float* part = ps + (size_t)item * C::PART;
   for (int idx = tid; idx < G * D; idx += blockDim.x) {
     const int hh = idx / D;
     float M = -INFINITY;
@@ -713,28 +733,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(DecodeArgs a)
   // two-level log-sum-exp combine: the last item of each group of kGroup
   // merges the group; the last group merges the group results into out.
   uint32_t* cnt = a.counters + (size_t)srel * kCountersPerStream;
+  const int NGR = (NI + kGroup - 1) / kGroup;
   const int g = item / kGroup;
   const int gsize = min(kGroup, NI - g * kGroup);
   float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  float* gpart = a.partials + (size_t)a.n_streams * NI * C::PART + ((size_t)srel * NG + g) * C::PART;
+  float* gpart = a.partials + (size_t)a.n_streams * NI * C::PART + ((size_t)srel * NGR + g) * C::PART;
   __threadfence();
   __syncthreads();
-  if (tid == 0) is_last = (atomicAdd(&cnt[1 + g], 1u) == (unsigned)(gsize - 1));
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  combine_partials<D, G>(a.partials + ((size_t)srel * NI + g * kGroup) * C::PART, gsize, gpart,
-                         NG == 1 ? outp : nullptr, tid);
-  if (tid == 0) cnt[1 + g] = 0u;
-  if (NG == 1) return;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) is_last = (atomicAdd(&cnt[0], 1u) == (unsigned)(NG - 1));
+  if (tid == 0) is_last = (atomicAdd(&cnt[2 + g], 1u) == (unsigned)(gsize - 1));
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  combine_partials<D, G>(a.partials + (size_t)a.n_streams * NI * C::PART + (size_t)srel * NG * C::PART, NG,
-                         nullptr, outp, tid);
+  combine_partials<D, G>(ps + (size_t)g * kGroup * C::PART, gsize, gpart, NGR == 1 ? outp : nullptr, tid);
+  if (tid == 0) cnt[2 + g] = 0u;
+  if (NGR > 1) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = (atomicAdd(&cnt[0], 1u) == (unsigned)(NGR - 1));
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    combine_partials<D, G>(a.partials + (size_t)a.n_streams * NI * C::PART + (size_t)srel * NGR * C::PART, NGR,
+                           nullptr, outp, tid);
+  }
   if (tid == 0) cnt[0] = 0u;
 }
 
@@ -756,7 +777,9 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   int merge = (NW * part + G * D) * 4 + 2 * kWinChunk * D * 2;
   const int ring = NW * stages * stage_bytes;
   int need = ring > merge ? ring : merge;
-  return (need + 127) / 128 * 128;
+  // per-warp scale scratch of the tile path (Cfg<D, G>::SCRATCH floats)
+  const int scratch = NW * 8 * ((D / 32) * 8 + 4 + (D / 8) * 2 + 4) * 4;
+  return (need + 127) / 128 * 128 + scratch;
 }
 
 template <int D, int G>

@@ -11,26 +11,18 @@
 namespace rq {
 
 // ----------------------------------------------------------- format tables
-// Slot list of one lane ordered by (class, word, slot); entry i -> (word, slot).
-// b = 2: slot classes 0,1,2,3,4,0,1,2 (slots 0-4 of a 16-bit half lie inside
-//        an fp16 mantissa in place, 5-7 after a 10-bit shift);
-// b = 4: classes 0,1,0,1; b = 3, 8: all class 0 (natural order).
-__host__ __device__ constexpr int slot_word(int b, int W, int i) {
-  return b == 2 ? (i < 6 * W ? (i % (2 * W)) / 2 : (i - 6 * W) % W)
-       : b == 4 ? (i % (2 * W)) / 2
-                : i / (codes_per_word(b) / 2);
-}
-__host__ __device__ constexpr int slot_pos(int b, int W, int i) {
-  return b == 2 ? (i < 6 * W ? i / (2 * W) + 5 * ((i % (2 * W)) % 2) : 3 + (i - 6 * W) / W)
-       : b == 4 ? i / (2 * W) + 2 * ((i % (2 * W)) % 2)
-                : i % (codes_per_word(b) / 2);
-}
-// Slot-list index of the K pair (mb, kb, r) and of the V pair (mb, kb, r).
-__host__ __device__ constexpr int k_pair_index(int D, int mb, int kb, int r) {
-  return 4 * ((mb * 2 + (r & 1)) * (D / 32) + kb / 2) + (kb & 1) * 2 + (r >> 1);
-}
-__host__ __device__ constexpr int v_pair_index(int mb, int kb, int r) {
-  return 4 * (mb * 2 + (r & 1)) + kb * 2 + (r >> 1);
+// A lane of a code blob owns D/4 registers (rho, kh) of four bytes: the 8-bit
+// A-operand fragments of the m16n8k32 integer MMA.  Row group rho has class
+// j = rho mod C and both its registers come from source sigma = 2*(rho/C)+kh;
+// the code of byte e sits at bits 8e + b*j .. 8e + b*j + b - 1 of the source,
+// so masking the source word to those bits of every byte yields four codes
+// scaled by 2^(b*j).  3-bit sources past the W words are assembled from the
+// top bit pairs (bits 6, 7 of each byte) of three consecutive words.
+__host__ __device__ constexpr int n_classes(int b) { return b == 2 ? 4 : b == 8 ? 1 : 2; }
+__host__ __device__ constexpr int reg_class(int b, int rho) { return rho % n_classes(b); }
+__host__ __device__ constexpr int reg_source(int b, int rho, int kh) { return 2 * (rho / n_classes(b)) + kh; }
+__host__ __device__ constexpr uint32_t class_mask(int b, int j) {
+  return (((1u << b) - 1u) * 0x01010101u) << (b * j);
 }
 // Byte offset of word w of a lane inside a code blob of W words per lane.
 __host__ __device__ constexpr int word_offset(int W, int lane, int w) {
@@ -38,29 +30,34 @@ __host__ __device__ constexpr int word_offset(int W, int lane, int w) {
                          : (W / 4) * 512 + ((w - 4 * (W / 4)) * 32 + lane) * 4;
 }
 
-// Class of a slot: how many b-bit steps its codes sit above the lowest
-// position from which they are read in place (fp16 mantissa = bits 0..9 of a
-// 16-bit half).  b=2: slots 0..4 in place, 5..7 after a 10-bit shift;
-// b=4: slots 0,1 in place, 2,3 after an 8-bit shift; b=3, 8: every slot is
-// shifted down to bit 0 (class 0).
-__host__ __device__ constexpr int slot_class(int b, int p) {
-  return b == 2 ? (p < 5 ? p : p - 5) : b == 4 ? (p & 1) : 0;
+// Register (rho, kh) of a lane from its W code words (rho, kh compile-time
+// after unrolling): four codes * 2^(b*j) as u8 bytes.
+template <int B, int W>
+__device__ __forceinline__ uint32_t code_reg(const uint32_t* words, int rho, int kh) {
+  const int j = reg_class(B, rho), s = reg_source(B, rho, kh);
+  if (B == 3 && s >= W) {
+    const int q = s - W;
+    const uint32_t f = ((words[3 * q] >> 6) & 0x03030303u) | ((words[3 * q + 1] >> 4) & 0x0C0C0C0Cu) |
+                       ((words[3 * q + 2] >> 2) & 0x30303030u);
+    return f & class_mask(3, j);
+  }
+  return words[s] & class_mask(B, j);
 }
-// Class shared by the four pairs of quad q of a blob with W words per lane.
-__host__ __device__ constexpr int quad_class(int b, int W, int q) { return slot_class(b, slot_pos(b, W, 4 * q)); }
 
-// Pair of b-bit codes of slot p of word w as an fp16x2 of subnormals
-// c * 2^(b*class - 24): the code bits become the fp16 mantissa with a zero
-// exponent field, so the values are exact and need no offset removal.  The
-// 2^(b*class) factor is undone by the per-quad scale.
-template <int B>
-__device__ __forceinline__ uint32_t extract_pair(const uint32_t* words, int w, int p) {
-  constexpr uint32_t m = (1u << B) - 1u;
-  constexpr uint32_t mm = m | (m << 16);
-  if (B == 2) return p < 5 ? (words[w] & (mm << (2 * p))) : ((words[w] >> 10) & (mm << (2 * (p - 5))));
-  if (B == 4) return p < 2 ? (words[w] & (mm << (4 * p))) : ((words[w] >> 8) & (mm << (4 * (p - 2))));
-  if (B == 8) return p == 0 ? (words[w] & mm) : ((words[w] >> 8) & mm);
-  return (words[w] >> (B * p)) & mm;
+// Places code c (B bits) of byte e of register (rho, kh) into the lane's words.
+template <int B, int W>
+__device__ __forceinline__ void put_code(uint32_t* words, int rho, int kh, int e, uint32_t c) {
+  const int j = reg_class(B, rho), s = reg_source(B, rho, kh);
+  if (B == 3 && s >= W) {
+    const int q = s - W;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const int f = 3 * j + k;
+      words[3 * q + f / 2] |= ((c >> k) & 1u) << (8 * e + 6 + (f & 1));
+    }
+  } else {
+    words[s] |= c << (8 * e + B * j);
+  }
 }
 
 // ------------------------------------------------------------ tensor cores
@@ -71,6 +68,25 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D = A(16x32 u8, row) * B(32x8 s8 / u8, col) + C, s32 accumulate; every C
+// element is the same value c.  Results are returned as raw 32-bit words.
+__device__ __forceinline__ void imma_u8s8(uint32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                          uint32_t c) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c), "r"(c), "r"(c), "r"(c));
+}
+__device__ __forceinline__ void imma_u8u8(uint32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                          uint32_t c) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c), "r"(c), "r"(c), "r"(c));
 }
 
 // Transpose an 8x8 b16 matrix held one row-pair per thread (m8n8 fragment).

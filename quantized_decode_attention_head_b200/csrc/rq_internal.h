@@ -90,16 +90,19 @@ struct DecodeArgs {
   int* status;            // workspace status word
 };
 
-// Split-K combine: work items are merged in groups of kGroup, then groups.
+// Split-K combine: work items are merged in groups of kGroup, then the
+// groups.  Per stream: counter [0] finished groups, [2 + g] finished items
+// of group g ([1] unused).
 constexpr int kGroup = 8;
-constexpr int kCountersPerStream = 64;  // [0] group counter, [1 + g] item counters of group g
-constexpr int kMaxItems = kGroup * (kCountersPerStream - 1);
+constexpr int kCountersPerStream = 64;
+constexpr int kMaxItems = kGroup * (kCountersPerStream - 2);
 inline int group_count(int items) { return (items + kGroup - 1) / kGroup; }
 
 // Workspace layout (bytes): [status int32, pad to 256][kCountersPerStream u32
 // counters per stream of the whole cache (L*B*Hkv)][item partials of one
-// call][group partials of one call].  The counter region is sized for every
-// stream so calls with different layer arguments never overlap.
+// call: [stream][item][G*D + 2G] floats = o, m, l][group partials of one
+// call].  The counter region is sized for every stream so calls with
+// different layer arguments never overlap.
 inline size_t ws_counter_offset() { return 256; }
 inline size_t ws_partial_offset(int64_t all_streams) {
   return ws_counter_offset() + (size_t)all_streams * kCountersPerStream * 4;
@@ -131,9 +134,9 @@ cudaError_t noalloc_scratch(void** ptr);
 
 constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeThreads = kDecodeConsumerWarps * 32;
-// per-warp ring depth: about 64 KB of records in flight per CTA
+// per-warp ring depth: about 9 KB of records in flight per warp
 inline int decode_stages(int stage_bytes) {
-  int p = 65536 / (kDecodeConsumerWarps * stage_bytes);
+  int p = 9216 / stage_bytes;
   return p < 2 ? 2 : (p > 8 ? 8 : p);
 }
 constexpr int kDeviceTimeout = 7;  // == RQ_ERR_DEVICE_TIMEOUT

@@ -96,19 +96,19 @@ __device__ void pack_k(TileSmem<D>& sm, uint8_t* rec, int lane) {
   uint32_t words[W];
 #pragma unroll
   for (int w = 0; w < W; ++w) words[w] = 0;
+  // register (rho, kh), byte e: token gid + 8i, channel 32g + 16kh + 4tig + e
 #pragma unroll
-  for (int mb = 0; mb < 2; ++mb)
+  for (int rho = 0; rho < D / 8; ++rho)
 #pragma unroll
-    for (int kb = 0; kb < D / 16; ++kb)
+    for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int idx = k_pair_index(D, mb, kb, r);
-        const int w = slot_word(KB, W, idx), p = slot_pos(KB, W, idx);
-        const int t = 16 * mb + 8 * (r & 1) + gid;
-        const int d0 = 16 * kb + 8 * (r >> 1) + 2 * tig;
+      for (int e = 0; e < 4; e += 2) {
+        const int i = rho / NG, g = rho % NG;
+        const int t = gid + 8 * i, d0 = 32 * g + 16 * kh + 4 * tig + e;
         const uint32_t x = sm.k[t][d0 / 2];
-        const float rr = sm.kr[t][d0 / 32], z = sm.kz[t][d0 / 32];
-        words[w] |= (code_of<KB>(lo_bf16(x), z, rr) << (KB * p)) | (code_of<KB>(hi_bf16(x), z, rr) << (16 + KB * p));
+        const float rr = sm.kr[t][g], z = sm.kz[t][g];
+        put_code<KB, W>(words, rho, kh, e, code_of<KB>(lo_bf16(x), z, rr));
+        put_code<KB, W>(words, rho, kh, e + 1, code_of<KB>(hi_bf16(x), z, rr));
       }
 #pragma unroll
   for (int c = 0; c < W / 4; ++c)
@@ -149,22 +149,20 @@ __device__ void pack_v(TileSmem<D>& sm, uint8_t* vrec, int lane) {
   uint32_t words[W];
 #pragma unroll
   for (int w = 0; w < W; ++w) words[w] = 0;
+  // register (rho, kh), byte e: channel 16mb + 8rh + gid (rho = 2mb + rh),
+  // token 4kh + tig + 8e
 #pragma unroll
-  for (int mb = 0; mb < D / 16; ++mb)
+  for (int rho = 0; rho < D / 8; ++rho) {
+    const int d = 16 * (rho / 2) + 8 * (rho % 2) + gid;
+    const float rr = sm.vr[d], z = sm.vz[d];
 #pragma unroll
-    for (int kb = 0; kb < 2; ++kb)
+    for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int idx = v_pair_index(mb, kb, r);
-        const int w = slot_word(VB, W, idx), p = slot_pos(VB, W, idx);
-        const int d = 16 * mb + 8 * (r & 1) + gid;
-        const int t0 = 16 * kb + 8 * (r >> 1) + 2 * tig;
-        const uint32_t x0 = sm.v[t0][d >> 1], x1 = sm.v[t0 + 1][d >> 1];
-        const float v0 = (d & 1) ? hi_bf16(x0) : lo_bf16(x0);
-        const float v1 = (d & 1) ? hi_bf16(x1) : lo_bf16(x1);
-        const float rr = sm.vr[d], z = sm.vz[d];
-        words[w] |= (code_of<VB>(v0, z, rr) << (VB * p)) | (code_of<VB>(v1, z, rr) << (16 + VB * p));
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t x = sm.v[4 * kh + tig + 8 * e][d >> 1];
+        put_code<VB, W>(words, rho, kh, e, code_of<VB>((d & 1) ? hi_bf16(x) : lo_bf16(x), z, rr));
       }
+  }
 #pragma unroll
   for (int c = 0; c < W / 4; ++c)
     *reinterpret_cast<uint4*>(vrec + word_offset(W, lane, 4 * c)) =
