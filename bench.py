@@ -1,11 +1,12 @@
 """Benchmark: quantized-KV decode attention on the long-context workload.
 
 One *step* = one serving decode step of the hot path on one request's cache:
-rq_append_token (bf16 ring write; every 32nd step also quantizes and packs
-a tile) followed by rq_decode_attention (split-K over the packed tiles plus
-the bf16 window, fused combine).  The per-head bit allocation (host) and the
-bulk prefill quantize run before the timed loop and are reported separately
-(alloc_ms, quantize_gbs).
+rq_decode_step = rq_append_token (the new token enters the bf16 window; every
+32nd step a tile is quantized and packed) + rq_decode_attention (split-K over
+the packed tiles plus the bf16 window, fused combine), one kernel launch on
+the 31 steps in 32 that complete no tile.  The per-head bit allocation (host)
+and the bulk prefill quantize run before the timed loop and are reported
+separately (alloc_ms, quantize_gbs).
 
 Workload: long_128k -- batch 1, 32 query / 8 kv heads, head_dim 128, 131072
 tokens, K outlier channels lognormal(1.5), 2-bit average over {2,3,4}.  Four
@@ -295,10 +296,10 @@ def run_gpu(args):
         c = i % NC
         j = i // NC
         cache, (q, kn, vn) = caches[c], step_in[c]
-        cache.rq_append_token(0, kn[j, 0], vn[j, 0])
         if timed_events is not None:
             timed_events[0].record(stream)
-        cache.rq_decode_attention(0, q[j, 0], out=outs[c], n_splits=args.splits, workspace=ws)
+        # append + decode: one fused launch, two when the append completes a tile
+        cache.rq_decode_step(0, q[j, 0], kn[j, 0], vn[j, 0], out=outs[c], n_splits=args.splits, workspace=ws)
         if timed_events is not None:
             timed_events[1].record(stream)
 
@@ -307,14 +308,17 @@ def run_gpu(args):
         do_step(i)
     torch.cuda.synchronize()
     step_bytes = 0
-    dec_bytes_steps = []
+    fused_bytes = []  # per step: bytes of the single fused launch, or None on a tile-flush step
+    n_flush = 0
     for i in range(args.warmup, total_steps):
         c = i % NC
         T_old = caches[c].length(0) + (i - args.warmup) // NC  # length before this step's append
         ab = append_bytes(wl, rec, T_old)
         db = decode_bytes(wl, rec, T_old + 1)
         step_bytes += ab + db
-        dec_bytes_steps.append(db)
+        flush = split_lengths(T_old + 1, wl.n_sink, wl.n_recent)[1] != split_lengths(T_old, wl.n_sink, wl.n_recent)[1]
+        n_flush += flush
+        fused_bytes.append(None if flush else ab + db)
     if world > 1:
         dist.barrier()
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -330,9 +334,10 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     elapsed = start.elapsed_time(end) / 1e3
-    dec_times = [a.elapsed_time(b) / 1e3 for a, b in dec_events]
+    # roofline of the fused decode kernel: steps with one launch only
+    dec_times = [a.elapsed_time(b) / 1e3 for (a, b), fb in zip(dec_events, fused_bytes) if fb is not None]
     dec_avg = sum(dec_times) / len(dec_times)
-    dec_bytes_avg = sum(dec_bytes_steps) / len(dec_bytes_steps)
+    dec_bytes_avg = sum(fb for fb in fused_bytes if fb is not None) / len(dec_times)
     status = QuantizedKVCache.rq_decode_read_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status}")
@@ -361,8 +366,7 @@ def run_gpu(args):
         dq[c].copy_(pin_q[c][j, 0], non_blocking=True)
         dk[c].copy_(pin_k[c][j, 0], non_blocking=True)
         dv[c].copy_(pin_v[c][j, 0], non_blocking=True)
-        caches[c].rq_append_token(0, dk[c], dv[c])
-        caches[c].rq_decode_attention(0, dq[c], out=outs[c], n_splits=args.splits, workspace=ws)
+        caches[c].rq_decode_step(0, dq[c], dk[c], dv[c], out=outs[c], n_splits=args.splits, workspace=ws)
         host_out.copy_(outs[c], non_blocking=True)
     e2.record(stream)
     torch.cuda.synchronize()
@@ -391,7 +395,7 @@ def run_gpu(args):
     tr = traffic_record()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": (tr["bytes_per_launch_scaled"] if tr else None),
-                "kernel": "decode_kernel<128,4> (split-K + fused combine)",
+                "kernel": "decode_kernel<128,4> (fused append + split-K decode + combine; steps without a tile flush)",
                 "peak_source": f"{peak_kind} hbm_gbs (burst)", "algorithmic_bytes_per_launch": dec_bytes_avg,
                 "avg_launch_us": dec_avg * 1e6}
     cpu = None
@@ -425,7 +429,7 @@ def run_gpu(args):
         "alloc_ms": alloc_ms,
         "e2e": {"value": e2e_b_all / e2e_el_all / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": args.steps + n_flush,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "clocks": clk,

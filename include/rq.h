@@ -198,6 +198,22 @@ rq_status rq_decode_attention(rq_cache* cache, int layer, const void* q, float* 
                               float softmax_scale, int n_splits, void* workspace,
                               size_t ws_bytes, cudaStream_t stream);
 
+/* rq_decode_step -- one serving step: rq_append_token(layer, k_new, v_new)
+ *   followed by rq_decode_attention(layer, q, ...) over the cache that now
+ *   includes the new token, with the same arguments, layouts, results and
+ *   errors as those two calls (InnerQ Algorithm 1, decode phase: the current
+ *   token's key and value join the high-precision recent window).  When the
+ *   append does not complete a tile -- 31 steps in 32 -- both happen in one
+ *   kernel launch: the window work item that owns the newest position reads
+ *   the token from k_new / v_new and writes it into the cache.  When it does,
+ *   the tile is quantized first and the decode follows (two launches).  On an
+ *   error nothing is launched and the length is unchanged; otherwise the
+ *   length grows by one.  The pages have no separate counterpart: it is the
+ *   two operations above, fused. */
+rq_status rq_decode_step(rq_cache* cache, int layer, const void* q, const void* k_new, const void* v_new,
+                         float* out, float softmax_scale, int n_splits, void* workspace, size_t ws_bytes,
+                         cudaStream_t stream);
+
 /* Blocking read of the workspace status word: 0 when every kernel that used
  * this workspace completed normally, otherwise RQ_ERR_DEVICE_TIMEOUT in the
  * low byte (a pipeline wait gave up after ~1 s and the kernel returned

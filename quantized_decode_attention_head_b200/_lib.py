@@ -68,6 +68,7 @@ SIGNATURES = {
     "rq_decode_workspace_bytes": (_I, [_P, _I, ctypes.POINTER(_SZ)]),
     "rq_decode_workspace_init": (_I, [_P, _SZ, _P]),
     "rq_decode_attention": (_I, [_P, _I, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
+    "rq_decode_step": (_I, [_P, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "rq_decode_read_status": (_I, [_P, _IP]),
     "rq_decode_attention_noalloc": (_I, [_P, _I, _P, _P, ctypes.c_float, _I, _P]),
 }

@@ -181,6 +181,30 @@ class QuantizedKVCache:
             workspace.numel(), _stream_ptr(stream)))
         return out
 
+    def rq_decode_step(self, layer, q, k_new, v_new, out=None, softmax_scale=0.0, n_splits=0, workspace=None,
+                       stream=None):
+        """rq_append_token(layer, k_new, v_new) then rq_decode_attention(layer, q),
+        in one launch when the append completes no tile."""
+        import torch
+
+        nl = self.n_layers if layer == -1 else 1
+        qshape = (nl, self.batch, self.n_q_heads, self.head_dim) if layer == -1 else (
+            self.batch, self.n_q_heads, self.head_dim)
+        kshape = (nl, self.batch, self.n_kv_heads, self.head_dim) if layer == -1 else (
+            self.batch, self.n_kv_heads, self.head_dim)
+        _check_tensor("q", q, torch.bfloat16, qshape)
+        _check_tensor("k_new", k_new, torch.bfloat16, kshape)
+        _check_tensor("v_new", v_new, torch.bfloat16, kshape)
+        if out is None:
+            out = torch.empty(qshape, dtype=torch.float32, device=q.device)
+        _check_tensor("out", out, torch.float32, qshape)
+        if workspace is None:
+            workspace = self.make_workspace(n_splits, stream)
+        check("rq_decode_step", lib().rq_decode_step(
+            self.handle, layer, _dptr(q), _dptr(k_new), _dptr(v_new), _dptr(out), float(softmax_scale),
+            int(n_splits), _dptr(workspace), workspace.numel(), _stream_ptr(stream)))
+        return out
+
     @staticmethod
     def rq_decode_read_status(workspace) -> int:
         st = ctypes.c_int(0)

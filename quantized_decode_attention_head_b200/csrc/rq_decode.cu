@@ -493,24 +493,31 @@ __host__ __device__ inline int window_tokens(int T, int S, int Tq) { return (T <
 
 template <int D>
 __device__ __forceinline__ void window_issue_chunk(const DecodeArgs& a, const uint8_t* win, uint32_t* kbuf,
-                                                   uint32_t* vbuf, uint64_t* bar, int j0, int cnt) {
+                                                   uint32_t* vbuf, uint64_t* bar, int j0, int cnt,
+                                                   const uint16_t* knew, const uint16_t* vnew) {
   const int S = a.g.S, ring = a.g.R + kTile;
   const int n_sink = a.T < S ? a.T : S;
   mbar_arrive_expect_tx(bar, (uint32_t)(cnt * D * 2 * 2));
+  // appended in the same call: the newest token comes from the caller's rows
+  const int n_cache = knew ? cnt - 1 : cnt;
+  if (knew) {
+    bulk_g2s(kbuf + (size_t)n_cache * (D / 2), knew, (uint32_t)(D * 2), bar);
+    bulk_g2s(vbuf + (size_t)n_cache * (D / 2), vnew, (uint32_t)(D * 2), bar);
+  }
   int t = 0;
-  while (t < cnt) {
+  while (t < n_cache) {
     const int j = j0 + t;
     size_t row;  // K row inside the window block; its V row follows its block's K rows
     int run;
     size_t v_off;
     if (j < n_sink) {
       row = j;
-      run = min(cnt - t, n_sink - j);
+      run = min(n_cache - t, n_sink - j);
       v_off = S;
     } else {
       const int slot = (a.Tq + (j - n_sink)) % ring;
       row = (size_t)2 * S + slot;
-      run = min(cnt - t, ring - slot);
+      run = min(n_cache - t, ring - slot);
       v_off = ring;
     }
     bulk_g2s(kbuf + (size_t)t * (D / 2), win + row * D * 2, (uint32_t)(run * D * 2), bar);
@@ -520,8 +527,9 @@ __device__ __forceinline__ void window_issue_chunk(const DecodeArgs& a, const ui
 }
 
 template <int D, int G>
-__device__ void window_item(const DecodeArgs& a, const uint8_t* win, const uint16_t* qh, int chunk, float* scratch,
-                            uint64_t* bar, float* slot, int warp, int lane, volatile int* abort_flag) {
+__device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* qh, size_t knew_off, int chunk,
+                            float* scratch, uint64_t* bar, float* slot, int warp, int lane,
+                            volatile int* abort_flag) {
   constexpr int RW = D / 2;  // words per bf16 row
   constexpr int HW = (G + NW - 1) / NW;
   const int tid = warp * 32 + lane;
@@ -531,7 +539,11 @@ __device__ void window_item(const DecodeArgs& a, const uint8_t* win, const uint1
   float* qs = scratch;                                              // [G][D]
   uint32_t* kbuf = reinterpret_cast<uint32_t*>(qs + G * D);         // [32][RW]
   uint32_t* vbuf = kbuf + kWinChunk * RW;                           // [32][RW]
-  if (tid == 0 && cnt > 0) window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt);
+  // a fused append delivers the newest token (window index n_tok - 1) itself
+  const bool newest = a.k_new != nullptr && cnt > 0 && j0 + cnt == n_tok;
+  if (tid == 0 && cnt > 0)
+    window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt, newest ? a.k_new + knew_off : nullptr,
+                          newest ? a.v_new + knew_off : nullptr);
   for (int i = tid; i < G * D; i += NW * 32) qs[i] = bf16_bits_to_float(qh[i]);
   const bool ok = cnt == 0 || __all_sync(0xffffffffu, mbar_wait_bounded(bar, 0));
   if (!__syncthreads_and(ok)) {
@@ -540,6 +552,26 @@ __device__ void window_item(const DecodeArgs& a, const uint8_t* win, const uint1
       (void)mbar_wait_bounded(bar, 0);  // let the copies land before the CTA exits
     }
     return;
+  }
+  if (newest && tid < 2 * (D / 8)) {
+    // the appended token enters the cache (sink row, or its ring slot) for
+    // later calls; no other work item of this call reads that row
+    const int S = a.g.S, ring = a.g.R + kTile;
+    const int n_sink = a.T < S ? a.T : S;
+    const int j = n_tok - 1;
+    size_t krow, vrow;
+    if (j < n_sink) {
+      krow = j;
+      vrow = (size_t)S + j;
+    } else {
+      const int slot = (a.Tq + (j - n_sink)) % ring;
+      krow = (size_t)2 * S + slot;
+      vrow = (size_t)2 * S + ring + slot;
+    }
+    const int c = tid % (D / 8);
+    const bool isv = tid >= D / 8;
+    const uint4 x = reinterpret_cast<const uint4*>((isv ? vbuf : kbuf) + (size_t)(cnt - 1) * RW)[c];
+    reinterpret_cast<uint4*>(win + (isv ? vrow : krow) * D * 2)[c] = x;
   }
 #pragma unroll
   for (int j = 0; j < HW; ++j) {
@@ -698,9 +730,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
                              t1 - t0, warp, lane, &abort_flag, a.status);
   } else {
     // one 32-token chunk of the bf16 sink + recent window
-    const uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
-    window_item<D, G>(a, win, qh, item - a.n_splits, merge + NW * C::PART, &bars[0], merge + warp * C::PART, warp,
-                      lane, &abort_flag);
+    uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
+    const size_t knew_off = ((size_t)(lrel * a.g.B + b) * a.g.Hkv + h) * D;
+    window_item<D, G>(a, win, qh, knew_off, item - a.n_splits, merge + NW * C::PART, &bars[0],
+                      merge + warp * C::PART, warp, lane, &abort_flag);
   }
   __syncthreads();  // every stage read has completed; merge may now alias the stages
   if (tiles_item && warp < NW && !abort_flag) dump_tile_state<D, G>(st, merge + warp * C::PART, lane);

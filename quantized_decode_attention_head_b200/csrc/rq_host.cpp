@@ -115,6 +115,50 @@ int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, in
 
 rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
 
+// Decode arguments for layers [l0, l0 + nl) of a cache holding T tokens, with
+// the workspace checked and partitioned; the fused-append pointers are null.
+rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, float* out, float softmax_scale,
+                      int n_splits, void* workspace, size_t ws_bytes, rq::DecodeArgs& a, int& smem) {
+  const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
+  const int n_tiles = Tq / rq::kTile;
+  const int streams = nl * c->g.B * c->g.Hkv;
+  if (streams > 65535) return RQ_ERR_UNSUPPORTED;
+  const int stage_bytes = max_record(c, l0, nl);
+  const int n_win = rq::window_items(T, c->g.S, c->g.R);
+  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win) : n_splits;
+  if (splits > n_tiles) splits = n_tiles;
+  if (n_tiles > 0 && splits < 1) splits = 1;
+  if (splits + n_win > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
+  const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
+  if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + n_win, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
+  a.g = c->g;
+  a.buf = c->buf;
+  a.desc = reinterpret_cast<const HeadDesc*>(c->buf);
+  a.q = static_cast<const uint16_t*>(q);
+  a.out = out;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)c->g.D);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.layer0 = l0;
+  a.n_layers = nl;
+  a.T = T;
+  a.Tq = Tq;
+  a.n_tiles = n_tiles;
+  a.n_splits = splits;
+  a.n_win = n_win;
+  a.n_streams = streams;
+  a.stages = rq::decode_stages(stage_bytes);
+  a.stage_bytes = stage_bytes;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.status = reinterpret_cast<int*>(ws);
+  a.counters = reinterpret_cast<uint32_t*>(ws + rq::ws_counter_offset());
+  a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
+  a.k_new = nullptr;
+  a.v_new = nullptr;
+  smem = rq::decode_smem_bytes(splits + n_win, a.stages, stage_bytes, c->g.G, c->g.D);
+  if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
+  return RQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -278,44 +322,37 @@ rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out,
   if (!c || !q || !out || !workspace || n_splits < 0) return RQ_ERR_INVALID_ARG;
   int l0, nl;
   if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
-  const int T = c->length[l0];
-  const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
-  const int n_tiles = Tq / rq::kTile;
-  const int streams = nl * c->g.B * c->g.Hkv;
-  const int stage_bytes = max_record(c, l0, nl);
-  const int n_win = rq::window_items(T, c->g.S, c->g.R);
-  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win) : n_splits;
-  if (splits > n_tiles) splits = n_tiles;
-  if (n_tiles > 0 && splits < 1) splits = 1;
-  if (splits + n_win > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
-  const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
-  if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + n_win, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
-  if (streams > 65535) return RQ_ERR_UNSUPPORTED;
   rq::DecodeArgs a;
-  a.g = c->g;
-  a.buf = c->buf;
-  a.desc = reinterpret_cast<const HeadDesc*>(c->buf);
-  a.q = static_cast<const uint16_t*>(q);
-  a.out = out;
-  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)c->g.D);
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.layer0 = l0;
-  a.n_layers = nl;
-  a.T = T;
-  a.Tq = Tq;
-  a.n_tiles = n_tiles;
-  a.n_splits = splits;
-  a.n_win = n_win;
-  a.n_streams = streams;
-  a.stages = rq::decode_stages(stage_bytes);
-  a.stage_bytes = stage_bytes;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  a.status = reinterpret_cast<int*>(ws);
-  a.counters = reinterpret_cast<uint32_t*>(ws + rq::ws_counter_offset());
-  a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
-  const int smem = rq::decode_smem_bytes(splits + n_win, a.stages, stage_bytes, c->g.G, c->g.D);
-  if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
+  int smem = 0;
+  rq_status st = fill_decode(c, l0, nl, c->length[l0], q, out, softmax_scale, n_splits, workspace, ws_bytes, a, smem);
+  if (st != RQ_OK) return st;
   return cuda_status(rq::launch_decode(a, smem, stream));
+}
+
+rq_status rq_decode_step(rq_cache* c, int layer, const void* q, const void* k_new, const void* v_new, float* out,
+                         float softmax_scale, int n_splits, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!c || !q || !k_new || !v_new || !out || !workspace || n_splits < 0) return RQ_ERR_INVALID_ARG;
+  int l0, nl;
+  if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
+  const int T_old = c->length[l0];
+  if (T_old + 1 > c->max_tokens) return RQ_ERR_CAPACITY;
+  const int S = c->g.S, R = c->g.R;
+  if (rq::quantized_tokens(T_old + 1, S, R) != rq::quantized_tokens(T_old, S, R)) {
+    // the append completes a tile: quantize it first, then decode (two launches)
+    rq_status st = rq_append_token(c, layer, k_new, v_new, stream);
+    if (st != RQ_OK) return st;
+    return rq_decode_attention(c, layer, q, out, softmax_scale, n_splits, workspace, ws_bytes, stream);
+  }
+  rq::DecodeArgs a;
+  int smem = 0;
+  rq_status st = fill_decode(c, l0, nl, T_old + 1, q, out, softmax_scale, n_splits, workspace, ws_bytes, a, smem);
+  if (st != RQ_OK) return st;
+  a.k_new = static_cast<const uint16_t*>(k_new);
+  a.v_new = static_cast<const uint16_t*>(v_new);
+  st = cuda_status(rq::launch_decode(a, smem, stream));
+  if (st != RQ_OK) return st;
+  for (int l = l0; l < l0 + nl; ++l) c->length[l] = T_old + 1;
+  return RQ_OK;
 }
 
 }  // extern "C"
@@ -327,48 +364,17 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
   if (!c || !q || !out || n_splits < 0) return RQ_ERR_INVALID_ARG;
   int l0, nl;
   if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
-  const int T = c->length[l0];
-  const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
-  const int n_tiles = Tq / rq::kTile;
-  const int streams = nl * c->g.B * c->g.Hkv;
-  if (streams > 65535) return RQ_ERR_UNSUPPORTED;
-  const int stage_bytes = max_record(c, l0, nl);
-  const int n_win = rq::window_items(T, c->g.S, c->g.R);
-  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win) : n_splits;
-  if (splits > n_tiles) splits = n_tiles;
-  if (n_tiles > 0 && splits < 1) splits = 1;
-  if (splits + n_win > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
-  const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
-  if (rq::ws_total_bytes(all_streams, streams, splits + n_win, c->g.G, c->g.D) > rq::kNoAllocScratchBytes)
-    return RQ_ERR_WORKSPACE;  // more split partials than the fixed scratch array holds
   void* scratch = nullptr;
   if (rq::noalloc_scratch(&scratch) != cudaSuccess) return RQ_ERR_CUDA;
-  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  rq::DecodeArgs a;
+  int smem = 0;
+  rq_status st = fill_decode(c, l0, nl, c->length[l0], q, out, softmax_scale, n_splits, scratch,
+                             rq::kNoAllocScratchBytes, a, smem);
+  if (st == RQ_ERR_WORKSPACE) return RQ_ERR_WORKSPACE;  // more split partials than the fixed array holds
+  if (st != RQ_OK) return st;
   // status word and completion counters must start at zero; the array keeps
   // whatever the previous call (on any stream) left in it
-  if (cudaMemsetAsync(ws, 0, rq::ws_partial_offset(all_streams), stream) != cudaSuccess) return RQ_ERR_CUDA;
-  rq::DecodeArgs a;
-  a.g = c->g;
-  a.buf = c->buf;
-  a.desc = reinterpret_cast<const HeadDesc*>(c->buf);
-  a.q = static_cast<const uint16_t*>(q);
-  a.out = out;
-  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)c->g.D);
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.layer0 = l0;
-  a.n_layers = nl;
-  a.T = T;
-  a.Tq = Tq;
-  a.n_tiles = n_tiles;
-  a.n_splits = splits;
-  a.n_win = n_win;
-  a.n_streams = streams;
-  a.stages = rq::decode_stages(stage_bytes);
-  a.stage_bytes = stage_bytes;
-  a.status = reinterpret_cast<int*>(ws);
-  a.counters = reinterpret_cast<uint32_t*>(ws + rq::ws_counter_offset());
-  a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
-  const int smem = rq::decode_smem_bytes(splits + n_win, a.stages, stage_bytes, c->g.G, c->g.D);
-  if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
+  const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
+  if (cudaMemsetAsync(scratch, 0, rq::ws_partial_offset(all_streams), stream) != cudaSuccess) return RQ_ERR_CUDA;
   return cuda_status(rq::launch_decode(a, smem, stream));
 }

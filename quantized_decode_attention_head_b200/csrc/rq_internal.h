@@ -73,7 +73,7 @@ struct AppendArgs {
 
 struct DecodeArgs {
   Geom g;
-  const uint8_t* buf;
+  uint8_t* buf;
   const HeadDesc* desc;
   const uint16_t* q;      // [nL][B][Hq][D]
   float* out;             // [nL][B][Hq][D]
@@ -88,6 +88,8 @@ struct DecodeArgs {
   float* partials;        // [streams][n_splits+1][G*D + 2G]
   uint32_t* counters;     // [streams]
   int* status;            // workspace status word
+  const uint16_t* k_new;  // fused append: the token added in this call, [nL][B][Hkv][D] (else null)
+  const uint16_t* v_new;
 };
 
 // Split-K combine: work items are merged in groups of kGroup, then the

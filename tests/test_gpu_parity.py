@@ -131,6 +131,39 @@ def test_append_across_flushes(S, R):
     assert QuantizedKVCache.rq_decode_read_status(ws) == 0
 
 
+@pytest.mark.parametrize("S,R,context", [(4, 32, 4 + 32 + 32 * 2 + 5), (0, 16, 16 + 31), (2, 0, 0), (6, 40, 3)])
+def test_decode_step_equals_append_then_decode(S, R, context):
+    """rq_decode_step (fused append + decode) gives the oracle's append-then-
+    decode output at every step, across tile flushes and from a short or empty
+    cache, and leaves the cache bytes (tiles, sink, ring) bit-exact."""
+    wl = _small(n_layers=2, batch=2, n_sink=S, n_recent=R, context=context)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    steps = 80  # every case reaches S + R + 32 tokens: at least one tile flush
+    cache, st, (k, v, f) = _build(wl, kb, vb, extra=steps)
+    q, kn, vn = workloads.step_inputs(wl, steps, f, "cuda")
+    knp, vnp, qnp = to_f32(kn), to_f32(vn), to_f32(q).astype(np.float64)
+    ws = cache.make_workspace()
+    flushes = 0
+    for t in range(steps):
+        for (l, b, h), s in st.items():
+            flushes += s.append(knp[t, l, b, h], vnp[t, l, b, h])
+        if t % 2 == 0:  # all layers in one call
+            out = cache.rq_decode_step(-1, q[t].contiguous(), kn[t].contiguous(), vn[t].contiguous(),
+                                       workspace=ws).cpu().numpy()
+        else:
+            out = np.stack([cache.rq_decode_step(l, q[t, l].contiguous(), kn[t, l].contiguous(),
+                                                 vn[t, l].contiguous(), workspace=ws).cpu().numpy()
+                            for l in range(wl.n_layers)])
+        exp = oracle_decode(wl, st, qnp[t], [(l, b) for l in range(wl.n_layers) for b in range(wl.batch)])
+        for (l, b), e in exp.items():
+            assert_close(out[l, b], e, f"step {t} layer {l} b {b}")
+    assert flushes > 0
+    assert cache.length(0) == wl.context + steps
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+
+
 def test_append_from_empty_fills_sink_then_ring():
     wl = _small(n_layers=1, batch=1, context=0)
     kb, vb = _bits_grid(1, wl.n_kv_heads)
