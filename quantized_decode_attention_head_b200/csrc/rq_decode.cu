@@ -24,6 +24,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <cooperative_groups.h>
+
 #include <cfloat>
 #include <mutex>
 
@@ -690,8 +692,50 @@ __device__ void combine_partials(const float* base, int n, float* dst, float* ou
   }
 }
 
+// Final log-sum-exp merge of n partial states (o[G][D], m[G], l[G] each,
+// stride PART floats) into the normalised output, for the slice of outputs
+// owned by cluster rank `part`: one output per thread, all of its loads for
+// up to 16 partials in flight at once.
 template <int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a) {
+__device__ void merge_outputs(const float* base, int n, float* outp, int part, int tid) {
+  using C = Cfg<D, G>;
+  constexpr int PER = (G * D + kDecodeCluster - 1) / kDecodeCluster;  // outputs of one CTA
+  constexpr int U = 16;
+  for (int idx = part * PER + tid; idx < (part + 1) * PER && idx < G * D; idx += kDecodeThreads) {
+    const int hh = idx / D;
+    float M = -INFINITY, O = 0.0f, L = 0.0f;
+    for (int i0 = 0; i0 < n; i0 += U) {
+      float ov[U], mv[U], lv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const bool ok = i0 + u < n;
+        const float* pp = base + (size_t)(i0 + u) * C::PART;
+        ov[u] = ok ? __ldcg(pp + idx) : 0.0f;
+        mv[u] = ok ? __ldcg(pp + G * D + hh) : -INFINITY;
+        lv[u] = ok ? __ldcg(pp + G * D + G + hh) : 0.0f;
+      }
+      float nm = M;
+#pragma unroll
+      for (int u = 0; u < U; ++u) nm = fmaxf(nm, mv[u]);
+      if (nm == -INFINITY) continue;
+      const float sc = ex2(M - nm);  // 0 while M = -inf
+      O *= sc;
+      L *= sc;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float f = ex2(mv[u] - nm);
+        O = fmaf(ov[u], f, O);
+        L = fmaf(lv[u], f, L);
+      }
+      M = nm;
+    }
+    outp[idx] = L > 0.0f ? O / L : 0.0f;
+  }
+}
+
+template <int D, int G>
+__global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecodeThreads, 4)
+    decode_kernel(DecodeArgs a) {
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[NW * kMaxStages];
@@ -738,16 +782,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
   __syncthreads();  // every stage read has completed; merge may now alias the stages
   if (tiles_item && warp < NW && !abort_flag) dump_tile_state<D, G>(st, merge + warp * C::PART, lane);
   __syncthreads();
-  if (abort_flag) return;
+  const bool valid = !abort_flag;
 
-  // merge the warps' partial states into this item's partial
-  float* ps = a.partials + (size_t)srel * NI * C::PART;
-  float* part = ps + (size_t)item * C::PART;
+  // merge the warps' partial states into this item's partial (shared memory)
+  float* mypart = merge + NW * C::PART;
   for (int idx = tid; idx < G * D; idx += blockDim.x) {
     const int hh = idx / D;
     float M = -INFINITY;
+    if (valid) {
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, merge[w * C::PART + G * D + hh]);
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, merge[w * C::PART + G * D + hh]);
+    }
     float O = 0.0f, L = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll
@@ -757,39 +802,71 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
         L = fmaf(merge[w * C::PART + G * D + G + hh], f, L);
       }
     }
-    part[idx] = O;
+    mypart[idx] = O;
     if (idx % D == 0) {
-      part[G * D + hh] = M;
-      part[G * D + G + hh] = L;
+      mypart[G * D + hh] = M;
+      mypart[G * D + G + hh] = L;
     }
   }
-  // two-level log-sum-exp combine: the last item of each group of kGroup
-  // merges the group; the last group merges the group results into out.
-  uint32_t* cnt = a.counters + (size_t)srel * kCountersPerStream;
-  const int NGR = (NI + kGroup - 1) / kGroup;
-  const int g = item / kGroup;
-  const int gsize = min(kGroup, NI - g * kGroup);
-  float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  float* gpart = a.partials + (size_t)a.n_streams * NI * C::PART + ((size_t)srel * NGR + g) * C::PART;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) is_last = (atomicAdd(&cnt[2 + g], 1u) == (unsigned)(gsize - 1));
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  combine_partials<D, G>(ps + (size_t)g * kGroup * C::PART, gsize, gpart, NGR == 1 ? outp : nullptr, tid);
-  if (tid == 0) cnt[2 + g] = 0u;
-  if (NGR > 1) {
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) is_last = (atomicAdd(&cnt[0], 1u) == (unsigned)(NGR - 1));
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    combine_partials<D, G>(a.partials + (size_t)a.n_streams * NI * C::PART + (size_t)srel * NGR * C::PART, NGR,
-                           nullptr, outp, tid);
+  // Level 1: the kDecodeCluster items of a thread-block cluster (consecutive
+  // items of one stream) are merged by the cluster's first CTA straight from
+  // the others' shared memory.  Every CTA passes both cluster barriers on
+  // every path (no early exit before them).
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = (int)cluster.block_rank();
+  cluster.sync();  // all partials of the cluster are in shared memory
+  float* ps = a.partials + (size_t)srel * NI * C::PART;
+  const int ncl = (int)gridDim.x / kDecodeCluster;
+  if (crank == 0) {
+    const float* rp[kDecodeCluster];
+#pragma unroll
+    for (int r = 0; r < kDecodeCluster; ++r) rp[r] = cluster.map_shared_rank(mypart, r);
+    float* cp = ps + (size_t)(item / kDecodeCluster) * C::PART;
+    for (int idx = tid; idx < G * D; idx += blockDim.x) {
+      const int hh = idx / D;
+      float mv[kDecodeCluster];
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < kDecodeCluster; ++r) {
+        mv[r] = rp[r][G * D + hh];
+        M = fmaxf(M, mv[r]);
+      }
+      float O = 0.0f, L = 0.0f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int r = 0; r < kDecodeCluster; ++r) {
+          const float f = ex2(mv[r] - M);
+          O = fmaf(rp[r][idx], f, O);
+          L = fmaf(rp[r][G * D + G + hh], f, L);
+        }
+      }
+      cp[idx] = O;
+      if (idx % D == 0) {
+        cp[G * D + hh] = M;
+        cp[G * D + G + hh] = L;
+      }
+    }
   }
-  if (tid == 0) cnt[0] = 0u;
+  // the first CTA publishes the cluster partial and learns whether its
+  // cluster is the stream's last; it tells every CTA of the cluster
+  if (crank == 0) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const int last = atomicAdd(&a.counters[(size_t)srel * kCountersPerStream], 1u) == (unsigned)(ncl - 1);
+#pragma unroll
+      for (int r = 0; r < kDecodeCluster; ++r) *cluster.map_shared_rank(&is_last, r) = last;
+    }
+  }
+  cluster.sync();  // remote partial reads and the is_last stores are complete
+  if (!is_last) return;
+  // Level 2: the CTAs of the last cluster merge the cluster partials, each a
+  // slice of the outputs
+  __threadfence();
+  float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
+  merge_outputs<D, G>(ps, ncl, outp, crank, tid);
+  if (crank == 0 && tid == 0) a.counters[(size_t)srel * kCountersPerStream] = 0u;
 }
 
 template <int D, int G>
@@ -797,7 +874,7 @@ cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int streams = a.n_layers * a.g.B * a.g.Hkv;
-  dim3 grid(a.n_splits + a.n_win, streams);
+  dim3 grid(cluster_items(a.n_splits + a.n_win), streams);
   decode_kernel<D, G><<<grid, kDecodeThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
@@ -808,6 +885,7 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   const int part = G * D + 2 * G;
   // merge slots + window scratch (q, one K and one V chunk)
   int merge = (NW * part + G * D) * 4 + 2 * kWinChunk * D * 2;
+  if (merge < (NW + 1) * part * 4) merge = (NW + 1) * part * 4;  // warp slots + the item partial
   const int ring = NW * stages * stage_bytes;
   int need = ring > merge ? ring : merge;
   // per-warp scale scratch of the tile path (Cfg<D, G>::SCRATCH floats)
@@ -815,19 +893,23 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   return (need + 127) / 128 * 128 + scratch;
 }
 
+// CTAs of the decode kernel that the device holds at once, in whole clusters.
 template <int D, int G>
-int occupancy_dg(int smem) {
+int resident_ctas_dg(int smem) {
   if (cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return 1;
+    return kDecodeCluster;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kDecodeCluster * 64, 1, 1);
+  cfg.blockDim = dim3(kDecodeThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<D, G>, kDecodeThreads, smem) != cudaSuccess)
-    return 1;
-  return n > 0 ? n : 1;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<D, G>, &cfg) != cudaSuccess || n < 1) return kDecodeCluster;
+  return n * kDecodeCluster;
 }
 
-int decode_occupancy(int D, int G, int smem) {
+int decode_resident_ctas(int D, int G, int smem) {
 #define RQ_DG(DD, GG) \
-  if (D == DD && G == GG) return occupancy_dg<DD, GG>(smem);
+  if (D == DD && G == GG) return resident_ctas_dg<DD, GG>(smem);
   RQ_DG(128, 1) RQ_DG(128, 2) RQ_DG(128, 4) RQ_DG(128, 8)
   RQ_DG(64, 1) RQ_DG(64, 2) RQ_DG(64, 4) RQ_DG(64, 8)
 #undef RQ_DG

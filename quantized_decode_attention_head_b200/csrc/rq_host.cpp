@@ -97,14 +97,14 @@ int max_record(const rq_cache* c, int l0, int nl) {
   return r;
 }
 
-// Tile splits per stream so that all work items of the call (splits + one
-// window item per stream) fill the resident CTA slots of the GPU once.
+// Tile splits per stream so that all work items of the call (splits plus the
+// window items, padded to whole clusters) fill the resident CTA slots once.
 int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win) {
   if (n_tiles <= 0) return 0;
-  const int occ = rq::decode_occupancy(
+  const long slots = rq::decode_resident_ctas(
       c->g.D, c->g.G, rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes), stage_bytes, c->g.G, c->g.D));
-  const long slots = (long)occ * c->sm_count;
-  long s = slots / streams - n_win;
+  long per = (slots / streams) / rq::kDecodeCluster * rq::kDecodeCluster;
+  long s = per - n_win;
   if (s < 1) s = 1;
   const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;  // keep a CTA's pipeline busy
   if (s > max_by_work) s = max_by_work;
@@ -128,7 +128,7 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win) : n_splits;
   if (splits > n_tiles) splits = n_tiles;
   if (n_tiles > 0 && splits < 1) splits = 1;
-  if (splits + n_win > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
+  if (rq::cluster_items(splits + n_win) > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
   const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
   if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + n_win, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
   a.g = c->g;

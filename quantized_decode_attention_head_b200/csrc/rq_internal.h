@@ -92,26 +92,30 @@ struct DecodeArgs {
   const uint16_t* v_new;
 };
 
-// Split-K combine: work items are merged in groups of kGroup, then the
-// groups.  Per stream: counter [0] finished groups, [2 + g] finished items
-// of group g ([1] unused).
-constexpr int kGroup = 8;
+// Split-K combine.  The work items of a stream (tile splits, then window
+// chunks) form thread-block clusters of kDecodeCluster consecutive items
+// (the grid is padded with empty items to whole clusters); a cluster merges
+// its items through distributed shared memory, and the CTAs of the last
+// cluster of the stream to finish merge the cluster partials, each a slice
+// of the outputs.  Per stream counter [0] counts finished clusters.
+constexpr int kDecodeCluster = 4;
 constexpr int kCountersPerStream = 64;
-constexpr int kMaxItems = kGroup * (kCountersPerStream - 2);
-inline int group_count(int items) { return (items + kGroup - 1) / kGroup; }
+constexpr int kMaxItems = 496;
+__host__ __device__ inline int cluster_items(int items) {
+  return (items + kDecodeCluster - 1) / kDecodeCluster * kDecodeCluster;
+}
 
 // Workspace layout (bytes): [status int32, pad to 256][kCountersPerStream u32
-// counters per stream of the whole cache (L*B*Hkv)][item partials of one
-// call: [stream][item][G*D + 2G] floats = o, m, l][group partials of one
-// call].  The counter region is sized for every stream so calls with
-// different layer arguments never overlap.
+// counters per stream of the whole cache (L*B*Hkv)][partials of one call:
+// [stream][item][G*D + 2G] floats = o, m, l (cluster partials use the first
+// items' slots)].  The counter region is sized for every stream so calls
+// with different layer arguments never overlap.
 inline size_t ws_counter_offset() { return 256; }
 inline size_t ws_partial_offset(int64_t all_streams) {
   return ws_counter_offset() + (size_t)all_streams * kCountersPerStream * 4;
 }
 inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int items, int G, int D) {
-  return ws_partial_offset(all_streams) +
-         (size_t)call_streams * (items + group_count(items)) * (size_t)(G * D + 2 * G) * 4;
+  return ws_partial_offset(all_streams) + (size_t)call_streams * items * (size_t)(G * D + 2 * G) * 4;
 }
 // bf16 window tokens of a T-token cache and the number of 32-token window items
 inline int window_items(int T, int S, int R) {
@@ -127,7 +131,7 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int smem_bytes, cudaStream_t s);
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D);
-int decode_occupancy(int D, int G, int smem_bytes);  // resident CTAs per SM
+int decode_resident_ctas(int D, int G, int smem_bytes);  // CTAs resident on the device, whole clusters
 
 // Size of the device array behind rq_decode_attention_noalloc (bytes).
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
