@@ -483,12 +483,14 @@ __device__ void dump_tile_state(const WarpState<D, G>& st, float* slot, int lane
   }
 }
 
-// bf16 sink + recent window on CUDA cores.  The window is split into work
-// items of 32 tokens.  Thread 0 stages the item's K and V rows in shared
-// memory with at most six 1-D bulk copies (the rows of a chunk form at most
-// three contiguous runs: sink, ring, ring after wrap); warp w then takes heads
-// w, w + 4, ...: lane = token for q.k (K row words read in a lane-rotated
-// order so the 32 rows hit 32 banks), lane = channel for p.v.
+// bf16 sink + recent window on CUDA cores.  The window is split into chunks
+// of 32 tokens, kWinChunksPerItem consecutive chunks per work item.  For each
+// chunk thread 0 stages its K and V rows in shared memory with at most six
+// 1-D bulk copies (the rows of a chunk form at most three contiguous runs:
+// sink, ring, ring after wrap); warp w then takes heads w, w + 4, ...:
+// lane = token for q.k (K row words read in a lane-rotated order so the 32
+// rows hit 32 banks), lane = channel for p.v, and merges the chunk into its
+// running (m, l, o).
 constexpr int kWinChunk = 32;
 
 __host__ __device__ inline int window_tokens(int T, int S, int Tq) { return (T < S ? T : S) + (T - (T < S ? T : S) - Tq); }
@@ -529,59 +531,74 @@ __device__ __forceinline__ void window_issue_chunk(const DecodeArgs& a, const ui
 }
 
 template <int D, int G>
-__device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* qh, size_t knew_off, int chunk,
+__device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* qh, size_t knew_off, int witem,
                             float* scratch, uint64_t* bar, float* slot, int warp, int lane,
                             volatile int* abort_flag) {
   constexpr int RW = D / 2;  // words per bf16 row
   constexpr int HW = (G + NW - 1) / NW;
   const int tid = warp * 32 + lane;
   const int n_tok = window_tokens(a.T, a.g.S, a.Tq);
-  const int j0 = chunk * kWinChunk;
-  const int cnt = max(0, min(kWinChunk, n_tok - j0));
+  const int n_chunks = (n_tok + kWinChunk - 1) / kWinChunk;
+  const int c0 = witem * kWinChunksPerItem;
+  const int c1 = min(c0 + kWinChunksPerItem, n_chunks);
   float* qs = scratch;                                              // [G][D]
   uint32_t* kbuf = reinterpret_cast<uint32_t*>(qs + G * D);         // [32][RW]
   uint32_t* vbuf = kbuf + kWinChunk * RW;                           // [32][RW]
-  // a fused append delivers the newest token (window index n_tok - 1) itself
-  const bool newest = a.k_new != nullptr && cnt > 0 && j0 + cnt == n_tok;
-  if (tid == 0 && cnt > 0)
-    window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt, newest ? a.k_new + knew_off : nullptr,
-                          newest ? a.v_new + knew_off : nullptr);
   for (int i = tid; i < G * D; i += NW * 32) qs[i] = bf16_bits_to_float(qh[i]);
-  const bool ok = cnt == 0 || __all_sync(0xffffffffu, mbar_wait_bounded(bar, 0));
-  if (!__syncthreads_and(ok)) {
-    if (tid == 0) {
-      raise_abort(abort_flag, a.status);
-      (void)mbar_wait_bounded(bar, 0);  // let the copies land before the CTA exits
-    }
-    return;
-  }
-  if (newest && tid < 2 * (D / 8)) {
-    // the appended token enters the cache (sink row, or its ring slot) for
-    // later calls; no other work item of this call reads that row
-    const int S = a.g.S, ring = a.g.R + kTile;
-    const int n_sink = a.T < S ? a.T : S;
-    const int j = n_tok - 1;
-    size_t krow, vrow;
-    if (j < n_sink) {
-      krow = j;
-      vrow = (size_t)S + j;
-    } else {
-      const int slot = (a.Tq + (j - n_sink)) % ring;
-      krow = (size_t)2 * S + slot;
-      vrow = (size_t)2 * S + ring + slot;
-    }
-    const int c = tid % (D / 8);
-    const bool isv = tid >= D / 8;
-    const uint4 x = reinterpret_cast<const uint4*>((isv ? vbuf : kbuf) + (size_t)(cnt - 1) * RW)[c];
-    reinterpret_cast<uint4*>(win + (isv ? vrow : krow) * D * 2)[c] = x;
-  }
+  // running state of this warp's heads over the item's chunks
+  float m[HW], l[HW], o[HW][D / 32];
 #pragma unroll
-  for (int j = 0; j < HW; ++j) {
-    const int h = warp + NW * j;
-    float m = -INFINITY, l = 0.0f, o[D / 32];
+  for (int jh = 0; jh < HW; ++jh) {
+    m[jh] = -INFINITY;
+    l[jh] = 0.0f;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) o[c] = 0.0f;
-    if (h < G && cnt > 0) {
+    for (int c = 0; c < D / 32; ++c) o[jh][c] = 0.0f;
+  }
+  int parity = 0;
+  for (int ch = c0; ch < c1; ++ch, parity ^= 1) {
+    const int j0 = ch * kWinChunk;
+    const int cnt = min(kWinChunk, n_tok - j0);
+    // a fused append delivers the newest token (window index n_tok - 1) itself
+    const bool newest = a.k_new != nullptr && j0 + cnt == n_tok;
+    if (ch > c0) {
+      __syncthreads();  // every thread has finished reading the previous chunk
+      if (tid == 0) fence_proxy_async_smem();
+    }
+    if (tid == 0)
+      window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt, newest ? a.k_new + knew_off : nullptr,
+                            newest ? a.v_new + knew_off : nullptr);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, (uint32_t)parity));
+    if (!__syncthreads_and(ok)) {
+      if (tid == 0) {
+        raise_abort(abort_flag, a.status);
+        (void)mbar_wait_bounded(bar, (uint32_t)parity);  // let the copies land before the CTA exits
+      }
+      return;
+    }
+    if (newest && tid < 2 * (D / 8)) {
+      // the appended token enters the cache (sink row, or its ring slot) for
+      // later calls; no other work item of this call reads that row
+      const int S = a.g.S, ring = a.g.R + kTile;
+      const int n_sink = a.T < S ? a.T : S;
+      const int j = n_tok - 1;
+      size_t krow, vrow;
+      if (j < n_sink) {
+        krow = j;
+        vrow = (size_t)S + j;
+      } else {
+        const int rs = (a.Tq + (j - n_sink)) % ring;
+        krow = (size_t)2 * S + rs;
+        vrow = (size_t)2 * S + ring + rs;
+      }
+      const int c = tid % (D / 8);
+      const bool isv = tid >= D / 8;
+      const uint4 x = reinterpret_cast<const uint4*>((isv ? vbuf : kbuf) + (size_t)(cnt - 1) * RW)[c];
+      reinterpret_cast<uint4*>(win + (isv ? vrow : krow) * D * 2)[c] = x;
+    }
+#pragma unroll
+    for (int jh = 0; jh < HW; ++jh) {
+      const int h = warp + NW * jh;
+      if (h >= G) continue;
       float acc = 0.0f;
       if (lane < cnt) {
 #pragma unroll 8
@@ -593,25 +610,34 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
         }
       }
       const float x = lane < cnt ? acc * a.scale_log2 : -INFINITY;
-      m = warp_max(x);
-      const float p = ex2(x - m);
-      l = warp_sum(p);
+      const float mc = warp_max(x);
+      const float mn = fmaxf(m[jh], mc);
+      const float a_old = ex2(m[jh] - mn);  // 0 while m = -inf
+      const float p = ex2(x - mn);
+      l[jh] = l[jh] * a_old + warp_sum(p);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) o[jh][c] *= a_old;
       for (int t = 0; t < cnt; ++t) {
         const float pt = __shfl_sync(0xffffffffu, p, t);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           const int d = lane + 32 * c;
           const uint32_t vv = vbuf[t * RW + d / 2];
-          o[c] = fmaf(pt, (d & 1) ? bf16_bits_to_float(vv >> 16) : bf16_bits_to_float(vv & 0xFFFFu), o[c]);
+          o[jh][c] = fmaf(pt, (d & 1) ? bf16_bits_to_float(vv >> 16) : bf16_bits_to_float(vv & 0xFFFFu), o[jh][c]);
         }
       }
+      m[jh] = mn;
     }
+  }
+#pragma unroll
+  for (int jh = 0; jh < HW; ++jh) {
+    const int h = warp + NW * jh;
     if (h < G) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) slot[h * D + lane + 32 * c] = o[c];
+      for (int c = 0; c < D / 32; ++c) slot[h * D + lane + 32 * c] = o[jh][c];
       if (lane == 0) {
-        slot[G * D + h] = m;
-        slot[G * D + G + h] = l;
+        slot[G * D + h] = m[jh];
+        slot[G * D + G + h] = l[jh];
       }
     }
   }
@@ -623,71 +649,6 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
     if (lane == 0) {
       slot[G * D + h] = -INFINITY;
       slot[G * D + G + h] = 0.0f;
-    }
-  }
-}
-
-// Log-sum-exp merge of n partial states (stride PART floats from `base`)
-// into one: written to `dst` as a partial, or normalised into `outp`.  Each
-// thread owns OPT outputs and loads the o, m and l of up to U partials for
-// all of them at once (one round of independent loads per U partials).
-template <int D, int G>
-__device__ void combine_partials(const float* base, int n, float* dst, float* outp, int tid) {
-  using C = Cfg<D, G>;
-  constexpr int OPT = (G * D + kDecodeThreads - 1) / kDecodeThreads;
-  constexpr int U = OPT >= 32 ? 1 : 32 / OPT;  // at most 96 values in flight per thread
-  float M[OPT], L[OPT], O[OPT];
-#pragma unroll
-  for (int k = 0; k < OPT; ++k) {
-    M[k] = -INFINITY;
-    L[k] = 0.0f;
-    O[k] = 0.0f;
-  }
-  for (int i0 = 0; i0 < n; i0 += U) {
-    float ov[OPT][U], mv[OPT][U], lv[OPT][U];
-#pragma unroll
-    for (int k = 0; k < OPT; ++k) {
-      const int idx = tid + k * kDecodeThreads;
-      const int hh = idx < G * D ? idx / D : 0;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const bool ok = idx < G * D && i0 + u < n;
-        const float* pp = base + (size_t)(i0 + u) * C::PART;
-        ov[k][u] = ok ? __ldcg(pp + idx) : 0.0f;
-        mv[k][u] = ok ? __ldcg(pp + G * D + hh) : -INFINITY;
-        lv[k][u] = ok ? __ldcg(pp + G * D + G + hh) : 0.0f;
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < OPT; ++k) {
-      float nm = M[k];
-#pragma unroll
-      for (int u = 0; u < U; ++u) nm = fmaxf(nm, mv[k][u]);
-      if (nm == -INFINITY) continue;
-      const float a = ex2(M[k] - nm);  // 0 when M was -inf
-      O[k] *= a;
-      L[k] *= a;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const float f = ex2(mv[k][u] - nm);
-        O[k] = fmaf(ov[k][u], f, O[k]);
-        L[k] = fmaf(lv[k][u], f, L[k]);
-      }
-      M[k] = nm;
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < OPT; ++k) {
-    const int idx = tid + k * kDecodeThreads;
-    if (idx >= G * D) continue;
-    if (outp) {
-      outp[idx] = L[k] > 0.0f ? O[k] / L[k] : 0.0f;
-    } else {
-      dst[idx] = O[k];
-      if (idx % D == 0) {
-        dst[G * D + idx / D] = M[k];
-        dst[G * D + G + idx / D] = L[k];
-      }
     }
   }
 }

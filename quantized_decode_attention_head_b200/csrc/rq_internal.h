@@ -117,12 +117,13 @@ inline size_t ws_partial_offset(int64_t all_streams) {
 inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int items, int G, int D) {
   return ws_partial_offset(all_streams) + (size_t)call_streams * items * (size_t)(G * D + 2 * G) * 4;
 }
-// bf16 window tokens of a T-token cache and the number of 32-token window items
+// bf16 window tokens of a T-token cache and the number of window work items
+// (kWinChunksPerItem chunks of 32 tokens each; at least one item)
+constexpr int kWinChunksPerItem = 3;
 inline int window_items(int T, int S, int R) {
-  const int n_sink = T < S ? T : S;
   const int n_tok = T - quantized_tokens(T, S, R);
-  (void)n_sink;
-  const int n = (n_tok + kTile - 1) / kTile;
+  const int chunks = (n_tok + kTile - 1) / kTile;
+  const int n = (chunks + kWinChunksPerItem - 1) / kWinChunksPerItem;
   return n > 0 ? n : 1;
 }
 
