@@ -397,11 +397,12 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
   float* vs = scratch + 8 * C::KSTR;
   const int VOFF = blob_bytes(KB, D) + 4 * D;
   int j = 0, slot = 0, parity = 0;  // ring position of tile j, advanced without division
+  uint8_t* cur = ring;               // slot address of tile j
+  const uint8_t* nsrc = src + (int64_t)(warp + stages * NW) * rec;  // record of tile j + stages
   bool ok = true;
   for (; j < n_w; ++j) {
     ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], (uint32_t)parity));
     if (!ok) break;
-    const uint8_t* cur = ring + (size_t)slot * stage_bytes;
     convert_meta<D, G, KB, VB>(cur, st, ks, vs, lane);
     __syncwarp();
     float acc[C::NB][4];
@@ -413,14 +414,16 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
     if (lane == 0 && j + stages < n_w) {
       fence_proxy_async_smem();  // generic-proxy reads of the slot precede the async refill
       mbar_arrive_expect_tx(&bars[slot], (uint32_t)rec);
-      bulk_g2s(ring + (size_t)slot * stage_bytes, src + (int64_t)(warp + (j + stages) * NW) * rec, (uint32_t)rec,
-               &bars[slot]);
+      bulk_g2s(cur, nsrc, (uint32_t)rec, &bars[slot]);
     }
+    nsrc += (int64_t)NW * rec;
+    cur += stage_bytes;
     if (++slot == stages) {
       slot = 0;
       parity ^= 1;
+      cur = ring;
     }
-    if (*abort_flag) {
+    if ((j & 3) == 3 && *abort_flag) {  // another warp gave up: stop within four tiles
       ok = false;
       break;
     }

@@ -98,7 +98,10 @@ struct DecodeArgs {
 // its items through distributed shared memory, and the CTAs of the last
 // cluster of the stream to finish merge the cluster partials, each a slice
 // of the outputs.  Per stream counter [0] counts finished clusters.
-constexpr int kDecodeCluster = 4;
+#ifndef RQ_DECODE_CLUSTER
+#define RQ_DECODE_CLUSTER 4
+#endif
+constexpr int kDecodeCluster = RQ_DECODE_CLUSTER;
 constexpr int kCountersPerStream = 64;
 constexpr int kMaxItems = 496;
 __host__ __device__ inline int cluster_items(int items) {
