@@ -27,7 +27,9 @@
 #include <cooperative_groups.h>
 
 #include <cfloat>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "rq_device.cuh"
 #include "rq_internal.h"
@@ -833,9 +835,30 @@ __global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecode
   if (crank == 0 && tid == 0) a.counters[(size_t)srel * kCountersPerStream] = 0u;
 }
 
+// Host-side caches (per device) of the decode kernel's shared-memory
+// attribute and of its resident-cluster capacity: both are fixed for a given
+// (device, D, G, size), and querying them on every call costs more host time
+// than a decode step.
+std::mutex g_attr_mu;
+std::map<std::tuple<int, int, int>, int> g_smem_set;             // (dev, D, G) -> largest size set
+std::map<std::tuple<int, int, int, int>, int> g_resident;        // (dev, D, G, smem) -> CTAs
+
+template <int D, int G>
+cudaError_t ensure_smem(int smem) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  int& cur = g_smem_set[std::make_tuple(dev, D, G)];
+  if (cur >= smem) return cudaSuccess;
+  e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) cur = smem;
+  return e;
+}
+
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_smem<D, G>(smem);
   if (e != cudaSuccess) return e;
   const int streams = a.n_layers * a.g.B * a.g.Hkv;
   dim3 grid(cluster_items(a.n_splits + a.n_win), streams);
@@ -860,14 +883,22 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
 // CTAs of the decode kernel that the device holds at once, in whole clusters.
 template <int D, int G>
 int resident_ctas_dg(int smem) {
-  if (cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return kDecodeCluster;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return kDecodeCluster;
+  {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    auto it = g_resident.find(std::make_tuple(dev, D, G, smem));
+    if (it != g_resident.end()) return it->second;
+  }
+  if (ensure_smem<D, G>(smem) != cudaSuccess) return kDecodeCluster;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kDecodeCluster * 64, 1, 1);
   cfg.blockDim = dim3(kDecodeThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)smem;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<D, G>, &cfg) != cudaSuccess || n < 1) return kDecodeCluster;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  g_resident[std::make_tuple(dev, D, G, smem)] = n * kDecodeCluster;
   return n * kDecodeCluster;
 }
 

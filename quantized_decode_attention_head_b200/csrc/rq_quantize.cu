@@ -245,11 +245,12 @@ __global__ void copy_window_kernel(QuantizeArgs a) {
   }
 }
 
-// grid (n_layers*B*Hkv); one warp per stream.
+// grid (n_layers*B*Hkv); two warps per stream: warp 0 writes the token, and
+// on a flush warp 0 quantizes and packs K while warp 1 does V.
 template <int D>
-__global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(64) append_kernel(AppendArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  const int lane = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int srel = blockIdx.x;
   const int h = srel % a.g.Hkv, b = (srel / a.g.Hkv) % a.g.B, l = a.layer0 + srel / (a.g.Hkv * a.g.B);
   const HeadDesc hd = a.desc[l * a.g.Hkv + h];
@@ -266,14 +267,14 @@ __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
     vdst = win + ((size_t)2 * S + ring + slot) * D * 2;
   }
   constexpr int kChunks = D / 8;
-  if (lane < kChunks) {
-    reinterpret_cast<uint4*>(kdst)[lane] = __ldg(reinterpret_cast<const uint4*>(a.k_new + (size_t)srel * D) + lane);
-  } else if (lane < 2 * kChunks) {
-    reinterpret_cast<uint4*>(vdst)[lane - kChunks] =
-        __ldg(reinterpret_cast<const uint4*>(a.v_new + (size_t)srel * D) + lane - kChunks);
+  if (tid < kChunks) {
+    reinterpret_cast<uint4*>(kdst)[tid] = __ldg(reinterpret_cast<const uint4*>(a.k_new + (size_t)srel * D) + tid);
+  } else if (tid < 2 * kChunks) {
+    reinterpret_cast<uint4*>(vdst)[tid - kChunks] =
+        __ldg(reinterpret_cast<const uint4*>(a.v_new + (size_t)srel * D) + tid - kChunks);
   }
   if (!a.flush) return;
-  __syncwarp();
+  __syncthreads();
   TileSmem<D>& sm = *reinterpret_cast<TileSmem<D>*>(smem_raw);
   const uint16_t* krows[kTile];
   const uint16_t* vrows[kTile];
@@ -283,16 +284,31 @@ __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
     krows[t] = reinterpret_cast<const uint16_t*>(win + ((size_t)2 * S + slot) * D * 2);
     vrows[t] = reinterpret_cast<const uint16_t*>(win + ((size_t)2 * S + ring + slot) * D * 2);
   }
-  // rows were just written through global memory by this warp: plain loads
+  // rows were just written through global memory by this block: plain loads
 #pragma unroll 4
-  for (int j = lane; j < kTile * kChunks; j += 32) {
+  for (int j = tid; j < kTile * kChunks; j += 64) {
     const int t = j / kChunks, c = j % kChunks;
     *reinterpret_cast<uint4*>(&sm.k[t][c * 4]) = reinterpret_cast<const uint4*>(krows[t])[c];
     *reinterpret_cast<uint4*>(&sm.v[t][c * 4]) = reinterpret_cast<const uint4*>(vrows[t])[c];
   }
-  __syncwarp();
+  __syncthreads();
   uint8_t* rec = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)a.flush_tile * hd.rec_bytes;
-  quantize_staged_tile<D>(sm, hd.k_bits, hd.v_bits, rec, lane);
+  if (warp == 0) {
+    switch (hd.k_bits) {
+      case 2: pack_k<D, 2>(sm, rec, lane); break;
+      case 3: pack_k<D, 3>(sm, rec, lane); break;
+      case 4: pack_k<D, 4>(sm, rec, lane); break;
+      default: pack_k<D, 8>(sm, rec, lane); break;
+    }
+  } else {
+    uint8_t* vrec = rec + blob_bytes(hd.k_bits, D) + 4 * D;
+    switch (hd.v_bits) {
+      case 2: pack_v<D, 2>(sm, vrec, lane); break;
+      case 3: pack_v<D, 3>(sm, vrec, lane); break;
+      case 4: pack_v<D, 4>(sm, vrec, lane); break;
+      default: pack_v<D, 8>(sm, vrec, lane); break;
+    }
+  }
 }
 
 }  // namespace
@@ -322,10 +338,10 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
   const int streams = a.n_layers * a.g.B * a.g.Hkv;
   if (a.g.D == 128) {
     const int smem = a.flush ? (int)sizeof(TileSmem<128>) : 0;
-    append_kernel<128><<<streams, 32, smem, st>>>(a);
+    append_kernel<128><<<streams, 64, smem, st>>>(a);
   } else {
     const int smem = a.flush ? (int)sizeof(TileSmem<64>) : 0;
-    append_kernel<64><<<streams, 32, smem, st>>>(a);
+    append_kernel<64><<<streams, 64, smem, st>>>(a);
   }
   return cudaGetLastError();
 }
