@@ -321,23 +321,28 @@ def run_gpu(args):
         fused_bytes.append(None if flush else ab + db)
     if world > 1:
         dist.barrier()
-    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
+    # Events sit only around the tile-flush steps (two launches each): an
+    # event between two decode launches would stop the next launch from
+    # overlapping the previous one's tail (programmatic dependent launch).
+    flush_events = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for n, fb in enumerate(fused_bytes) if fb is None}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         torch.cuda.synchronize()
         start.record(stream)
         for n, i in enumerate(range(args.warmup, total_steps)):
-            do_step(i, dec_events[n])
+            do_step(i, flush_events.get(n))
         end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     elapsed = start.elapsed_time(end) / 1e3
-    # roofline of the fused decode kernel: steps with one launch only
-    dec_times = [a.elapsed_time(b) / 1e3 for (a, b), fb in zip(dec_events, fused_bytes) if fb is not None]
-    dec_avg = sum(dec_times) / len(dec_times)
-    dec_bytes_avg = sum(fb for fb in fused_bytes if fb is not None) / len(dec_times)
+    # roofline of the fused decode kernel: the timed region minus the flush
+    # steps, per single-launch step
+    flush_time = sum(a.elapsed_time(b) / 1e3 for a, b in flush_events.values())
+    n_fused = sum(fb is not None for fb in fused_bytes)
+    dec_avg = (elapsed - flush_time) / n_fused
+    dec_bytes_avg = sum(fb for fb in fused_bytes if fb is not None) / n_fused
     status = QuantizedKVCache.rq_decode_read_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status}")

@@ -719,12 +719,17 @@ __global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecode
   uint8_t* area = smem + (size_t)NW * C::SCRATCH * 4;
   float* merge = reinterpret_cast<float*>(area);  // aliases the stages after the main loop
 
+  // programmatic dependent launch: the next kernel of the stream may be
+  // scheduled now; it waits below for this grid's memory before reading any
+  // input, so only its launch and prologue overlap our tail
+  griddep_launch_dependents();
   if (tid == 0) {
     abort_flag = 0;
     for (int s = 0; s < NW * kMaxStages; ++s) mbar_init(&bars[s], 1);
     mbar_fence_init();
   }
   __syncthreads();
+  griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
 
   WarpState<D, G> st;
   const bool tiles_item = item < a.n_splits;
@@ -861,8 +866,18 @@ cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
   cudaError_t e = ensure_smem<D, G>(smem);
   if (e != cudaSuccess) return e;
   const int streams = a.n_layers * a.g.B * a.g.Hkv;
-  dim3 grid(cluster_items(a.n_splits + a.n_win), streams);
-  decode_kernel<D, G><<<grid, kDecodeThreads, smem, st>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cluster_items(a.n_splits + a.n_win), streams, 1);
+  cfg.blockDim = dim3(kDecodeThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = RQ_DECODE_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G>, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

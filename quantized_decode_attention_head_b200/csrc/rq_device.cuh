@@ -109,6 +109,15 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
+// ------------------------------------------- programmatic dependent launch
+// Lets the next kernel of the stream be scheduled before this one ends.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+// Waits until every prerequisite grid has completed and its memory is visible
+// (returns at once when the kernel was launched without the dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 // ------------------------------------------------------ mbarrier / bulk copy
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

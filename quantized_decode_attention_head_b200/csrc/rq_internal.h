@@ -102,6 +102,10 @@ struct DecodeArgs {
 #define RQ_DECODE_CLUSTER 4
 #endif
 constexpr int kDecodeCluster = RQ_DECODE_CLUSTER;
+// decode launches allow programmatic dependent launch (1) or not (0)
+#ifndef RQ_DECODE_PDL
+#define RQ_DECODE_PDL 1
+#endif
 constexpr int kCountersPerStream = 64;
 constexpr int kMaxItems = 496;
 __host__ __device__ inline int cluster_items(int items) {
