@@ -388,12 +388,17 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
                         int warp, int lane, volatile int* abort_flag, int* status) {
   using C = Cfg<D, G>;
   const int n_w = n_my > warp ? (n_my - warp + NW - 1) / NW : 0;
+  // Packed tiles are written only by kernels that complete before a decode
+  // launch may start (prefill, tile flush), never by the decode launch this
+  // one may overlap, so the first records can be fetched before waiting on
+  // it; the query, the window and the workspace are read after the wait.
   if (lane == 0) {
     for (int j = 0; j < stages && j < n_w; ++j) {
       mbar_arrive_expect_tx(&bars[j], (uint32_t)rec);
       bulk_g2s(ring + (size_t)j * stage_bytes, src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec, &bars[j]);
     }
   }
+  griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
   setup_query<D, G, KB, VB>(st, qh, scale_log2, lane);
   float* ks = scratch;
   float* vs = scratch + 8 * C::KSTR;
@@ -700,7 +705,7 @@ __device__ void merge_outputs(const float* base, int n, float* outp, int part, i
 }
 
 template <int D, int G>
-__global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecodeThreads, 4)
+__global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS)
     decode_kernel(DecodeArgs a) {
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -729,7 +734,6 @@ __global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecode
     mbar_fence_init();
   }
   __syncthreads();
-  griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
 
   WarpState<D, G> st;
   const bool tiles_item = item < a.n_splits;
@@ -744,7 +748,8 @@ __global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecode
                              bars + warp * kMaxStages, reinterpret_cast<float*>(smem) + warp * C::SCRATCH, src, rec,
                              t1 - t0, warp, lane, &abort_flag, a.status);
   } else {
-    // one 32-token chunk of the bf16 sink + recent window
+    griddep_wait();  // the window rows and the query may come from the previous kernel
+    // 32-token chunks of the bf16 sink + recent window
     uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
     const size_t knew_off = ((size_t)(lrel * a.g.B + b) * a.g.Hkv + h) * D;
     window_item<D, G>(a, win, qh, knew_off, item - a.n_splits, merge + NW * C::PART, &bars[0],

@@ -147,10 +147,18 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 cudaError_t noalloc_scratch(void** ptr);
 
 constexpr int kDecodeConsumerWarps = 4;
+// CTAs per SM the decode kernel's registers are sized for, and the bytes of
+// tile records in flight per warp
+#ifndef RQ_DECODE_MIN_BLOCKS
+#define RQ_DECODE_MIN_BLOCKS 4
+#endif
+#ifndef RQ_STAGE_BUDGET
+#define RQ_STAGE_BUDGET 6144
+#endif
 constexpr int kDecodeThreads = kDecodeConsumerWarps * 32;
-// per-warp ring depth: about 9 KB of records in flight per warp
+// per-warp ring depth: about 6 KB of records in flight per warp (at least two)
 inline int decode_stages(int stage_bytes) {
-  int p = 9216 / stage_bytes;
+  int p = RQ_STAGE_BUDGET / stage_bytes;
   return p < 2 ? 2 : (p > 8 ? 8 : p);
 }
 constexpr int kDeviceTimeout = 7;  // == RQ_ERR_DEVICE_TIMEOUT
