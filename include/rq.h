@@ -113,6 +113,39 @@ rq_status rq_allocate_bits(int n, const double* w, const double* alpha, const do
                            double avg_bits, const int* allowed, int n_allowed,
                            double* b_cont, int* b_int, double* log_lambda);
 
+/* ------------------------------------------------------ distortion calibration
+ * RateQuant fits its distortion model D(b) = alpha * beta^-b per quantizer
+ * from a small calibration set (§1 "Method"; §3.4, quantizer-agnostic
+ * extensions, K and V on separate curves) and gives a head whose fit is poor
+ * (R^2 < 0.96) the decay rate min(beta_fitted, beta_bar) (W.10); it caps
+ * sensitivities at 5 times their mean before allocating (W.14).  A joint K/V
+ * budget is one rq_allocate_bits call over the 2N (head, K|V) units with their
+ * own (w, alpha, beta).
+ *
+ * rq_measure_distortion -- mean squared error, per head and bit width, of
+ *   quantizing and dequantizing calibration samples with this library's rule
+ *   (the same groups and rounding as rq_quantize_kv; x_hat = c * s + z in
+ *   fp64).  x: device bf16 [n_heads][n_tokens][head_dim]; role 0 = K groups
+ *   (32 channels of a token), 1 = V groups (one channel over 32 tokens;
+ *   n_tokens a multiple of 32).  bits: host [n_bits] in {2,3,4,8}.  mse:
+ *   device double [n_heads][n_bits], overwritten.
+ * Errors: RQ_ERR_INVALID_ARG, RQ_ERR_UNSUPPORTED (head_dim, bits), RQ_ERR_CUDA. */
+rq_status rq_measure_distortion(const void* x, int n_heads, int n_tokens, int head_dim, int role,
+                                const int* bits, int n_bits, double* mse, cudaStream_t stream);
+
+/* rq_fit_distortion -- host, pure.  Per head, the least-squares line through
+ *   (b, ln mse) gives ln alpha - b ln beta and its R^2 (points with mse <= 0
+ *   are left out); heads with R^2 < r2_min get beta = min(beta, beta_bar),
+ *   beta_bar = mean fitted beta of the heads at or above r2_min (of all heads
+ *   when none is).  mse: host [n_heads][n_bits]; outputs host [n_heads].
+ * Errors: RQ_ERR_INVALID_ARG (fewer than two usable points for a head). */
+rq_status rq_fit_distortion(int n_heads, const int* bits, int n_bits, const double* mse, double r2_min,
+                            double* alpha, double* beta, double* r2);
+
+/* rq_cap_weights -- host, pure: w_out[i] = min(w[i], factor * mean(w))
+ *   (factor 5 in W.14).  w_out may alias w.  Errors: RQ_ERR_INVALID_ARG. */
+rq_status rq_cap_weights(int n, const double* w, double factor, double* w_out);
+
 /* --------------------------------------------------------------------- cache */
 typedef struct {
   int n_layers;      /* L >= 1 */

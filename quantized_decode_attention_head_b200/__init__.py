@@ -6,6 +6,8 @@ definitions.  Importing the package does not load the library; the first
 call does, and fails loudly if it has not been built.
 """
 
-from .api import QuantizedKVCache, rq_allocate_bits, rq_cache_bytes  # noqa: F401
+from .api import (QuantizedKVCache, rq_allocate_bits, rq_cache_bytes, rq_cap_weights,  # noqa: F401
+                  rq_fit_distortion, rq_measure_distortion)
 
-__all__ = ["QuantizedKVCache", "rq_allocate_bits", "rq_cache_bytes"]
+__all__ = ["QuantizedKVCache", "rq_allocate_bits", "rq_cache_bytes", "rq_cap_weights", "rq_fit_distortion",
+           "rq_measure_distortion"]

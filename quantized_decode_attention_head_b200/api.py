@@ -67,6 +67,47 @@ def rq_allocate_bits(w, alpha, beta, avg_bits, allowed):
     return {"b_cont": b_cont, "b_int": b_int.astype(np.int64), "log_lambda": nu.value}
 
 
+def rq_measure_distortion(x, role, bits, stream=None):
+    """Mean squared error of this library's quantizer per (head, bit width).
+    x: bf16 CUDA tensor [n_heads, n_tokens, head_dim]; role "K" or "V".
+    Returns a float64 numpy array [n_heads, len(bits)]."""
+    import torch
+
+    if x.dim() != 3:
+        raise ValueError("x must be [n_heads, n_tokens, head_dim]")
+    _check_tensor("x", x, torch.bfloat16)
+    h, t, d = x.shape
+    bits = np.ascontiguousarray(bits, dtype=np.int32)
+    mse = torch.empty((h, bits.size), dtype=torch.float64, device=x.device)
+    check("rq_measure_distortion", lib().rq_measure_distortion(
+        _dptr(x), h, t, d, 0 if role == "K" else 1, bits.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), bits.size,
+        _dptr(mse), _stream_ptr(stream)))
+    return mse.cpu().numpy()
+
+
+def rq_fit_distortion(bits, mse, r2_min=0.96):
+    """Per-head (alpha, beta, r2) of D(b) = alpha * beta^-b from an
+    [n_heads, n_bits] table, with the poor-fit fallback (host)."""
+    bits = np.ascontiguousarray(bits, dtype=np.int32)
+    mse = np.ascontiguousarray(mse, dtype=np.float64)
+    n = mse.shape[0]
+    alpha, beta, r2 = np.zeros(n), np.zeros(n), np.zeros(n)
+    dp = ctypes.POINTER(ctypes.c_double)
+    check("rq_fit_distortion", lib().rq_fit_distortion(
+        n, bits.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), bits.size, mse.ctypes.data_as(dp), float(r2_min),
+        alpha.ctypes.data_as(dp), beta.ctypes.data_as(dp), r2.ctypes.data_as(dp)))
+    return alpha, beta, r2
+
+
+def rq_cap_weights(w, factor=5.0):
+    """w_i <- min(w_i, factor * mean(w)) (host)."""
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    out = np.zeros_like(w)
+    dp = ctypes.POINTER(ctypes.c_double)
+    check("rq_cap_weights", lib().rq_cap_weights(w.size, w.ctypes.data_as(dp), float(factor), out.ctypes.data_as(dp)))
+    return out
+
+
 def _config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, n_sink, n_recent, max_tokens, k_bits, v_bits, group=32):
     kb = np.ascontiguousarray(np.asarray(k_bits, dtype=np.int32).reshape(-1))
     vb = np.ascontiguousarray(np.asarray(v_bits, dtype=np.int32).reshape(-1))

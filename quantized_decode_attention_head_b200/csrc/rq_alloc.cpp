@@ -170,3 +170,82 @@ extern "C" rq_status rq_allocate_bits(int n, const double* w, const double* alph
   if (log_lambda) *log_lambda = nu;
   return RQ_OK;
 }
+
+// ------------------------------------------------------ distortion calibration
+// RateQuant §1 / §3.4 (per-quantizer fit of D(b) = alpha * beta^-b), W.10
+// (fallback beta = min(beta_fitted, beta_bar) for fits with R^2 < r2_min),
+// W.14 (sensitivity cap).  The fit is the least-squares line through
+// (b, ln D); points with D <= 0 are left out.
+
+namespace {
+
+// Fit of one head; returns false when fewer than two points are usable.
+bool fit_one(const int* bits, const double* d, int n_bits, double& alpha, double& beta, double& r2) {
+  double sb = 0.0, sy = 0.0;
+  int m = 0;
+  for (int i = 0; i < n_bits; ++i)
+    if (d[i] > 0.0) {
+      sb += bits[i];
+      sy += std::log(d[i]);
+      ++m;
+    }
+  if (m < 2) return false;
+  const double bm = sb / m, ym = sy / m;
+  double sxx = 0.0, sxy = 0.0, syy = 0.0;
+  for (int i = 0; i < n_bits; ++i)
+    if (d[i] > 0.0) {
+      const double db = bits[i] - bm, dy = std::log(d[i]) - ym;
+      sxx += db * db;
+      sxy += db * dy;
+      syy += dy * dy;
+    }
+  if (!(sxx > 0.0)) return false;
+  const double slope = sxy / sxx;
+  const double icpt = ym - slope * bm;
+  double res = 0.0;
+  for (int i = 0; i < n_bits; ++i)
+    if (d[i] > 0.0) {
+      const double e = std::log(d[i]) - (icpt + slope * bits[i]);
+      res += e * e;
+    }
+  alpha = std::exp(icpt);
+  beta = std::exp(-slope);
+  r2 = syy > 0.0 ? 1.0 - res / syy : 1.0;
+  return true;
+}
+
+}  // namespace
+
+extern "C" rq_status rq_fit_distortion(int n_heads, const int* bits, int n_bits, const double* mse, double r2_min,
+                                       double* alpha, double* beta, double* r2) {
+  if (n_heads < 1 || n_bits < 2 || !bits || !mse || !alpha || !beta || !r2) return RQ_ERR_INVALID_ARG;
+  std::vector<double> a(n_heads), b(n_heads), q(n_heads);
+  for (int h = 0; h < n_heads; ++h)
+    if (!fit_one(bits, mse + (size_t)h * n_bits, n_bits, a[h], b[h], q[h])) return RQ_ERR_INVALID_ARG;
+  double sum_good = 0.0, sum_all = 0.0;
+  int n_good = 0;
+  for (int h = 0; h < n_heads; ++h) {
+    sum_all += b[h];
+    if (q[h] >= r2_min) {
+      sum_good += b[h];
+      ++n_good;
+    }
+  }
+  const double beta_bar = n_good > 0 ? sum_good / n_good : sum_all / n_heads;
+  for (int h = 0; h < n_heads; ++h) {
+    alpha[h] = a[h];
+    beta[h] = q[h] >= r2_min ? b[h] : std::min(b[h], beta_bar);
+    r2[h] = q[h];
+  }
+  return RQ_OK;
+}
+
+extern "C" rq_status rq_cap_weights(int n, const double* w, double factor, double* w_out) {
+  if (n < 1 || !w || !w_out || !(factor > 0.0)) return RQ_ERR_INVALID_ARG;
+  double mean = 0.0;
+  for (int i = 0; i < n; ++i) mean += w[i];
+  mean /= n;
+  const double cap = factor * mean;
+  for (int i = 0; i < n; ++i) w_out[i] = std::min(w[i], cap);
+  return RQ_OK;
+}

@@ -357,6 +357,20 @@ rq_status rq_decode_step(rq_cache* c, int layer, const void* q, const void* k_ne
 
 }  // extern "C"
 
+// Distortion of the library's quantizer on calibration samples (see include/rq.h).
+extern "C" rq_status rq_measure_distortion(const void* x, int n_heads, int n_tokens, int head_dim, int role,
+                                           const int* bits, int n_bits, double* mse, cudaStream_t stream) {
+  if (!x || !bits || !mse || n_heads < 1 || n_tokens < 1 || n_bits < 1 || (role != 0 && role != 1))
+    return RQ_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return RQ_ERR_UNSUPPORTED;
+  if (role == 1 && n_tokens % rq::kTile != 0) return RQ_ERR_INVALID_ARG;
+  if (n_heads > 65535) return RQ_ERR_UNSUPPORTED;
+  for (int i = 0; i < n_bits; ++i)
+    if (!valid_bits(bits[i])) return RQ_ERR_UNSUPPORTED;
+  return cuda_status(rq::launch_measure_distortion(static_cast<const uint16_t*>(x), n_heads, n_tokens, head_dim,
+                                                   role, bits, n_bits, mse, stream));
+}
+
 // Decode without a caller-supplied workspace (see include/rq.h).  Uses the
 // library's own device scratch array; allocates nothing.
 extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const void* q, float* out,

@@ -137,6 +137,10 @@ inline int window_items(int T, int S, int R) {
 // Kernel launchers (rq_kernels.cu).  Return cudaGetLastError() after launch.
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+// Mean squared quantization error per (head, bit width) of bf16 samples
+// x [n_heads][n_tokens][head_dim]; role 0 = K groups, 1 = V groups.
+cudaError_t launch_measure_distortion(const uint16_t* x, int n_heads, int n_tokens, int head_dim, int role,
+                                      const int* bits, int n_bits, double* mse, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int smem_bytes, cudaStream_t s);
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D);
 int decode_resident_ctas(int D, int G, int smem_bytes);  // CTAs resident on the device, whole clusters

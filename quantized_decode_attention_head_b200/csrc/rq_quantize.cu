@@ -311,6 +311,65 @@ __global__ void __launch_bounds__(64) append_kernel(AppendArgs a) {
   }
 }
 
+// Distortion measurement for calibration: for every (head, bit width), the
+// sum of squared errors of quantizing and dequantizing the head's samples
+// with the rule above (x_hat = c * s + z in fp64).  One warp per group at a
+// time (lane = element); K groups are 32 channels of a token, V groups one
+// channel over 32 tokens.  Accumulated in fp64 with one atomic per warp.
+template <int B>
+__device__ double group_sse(float x) {
+  float mn = x, mx = x;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  float r;
+  const uint32_t meta = group_params<B>(mn, mx, r);
+  const double s = (double)__half2float(__ushort_as_half((unsigned short)(meta & 0xFFFFu)));
+  const double z = (double)__uint_as_float(meta & 0xFFFF0000u);
+  const double xh = __dadd_rn(__dmul_rn((double)code_of<B>(x, mn, r), s), z);
+  const double e = (double)x - xh;
+  return e * e;
+}
+
+__global__ void measure_sse_kernel(const uint16_t* x, int n_tokens, int head_dim, int role, int b, int bi,
+                                   int n_bits, double* sse) {
+  const int head = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int n_warps = (gridDim.x * blockDim.x) >> 5;
+  const int per_row = head_dim / 32;
+  const long n_groups = role == 0 ? (long)n_tokens * per_row : (long)(n_tokens / kTile) * head_dim;
+  const uint16_t* xh = x + (size_t)head * n_tokens * head_dim;
+  double acc = 0.0;
+  for (long gi = warp; gi < n_groups; gi += n_warps) {
+    size_t idx;
+    if (role == 0) {
+      idx = (size_t)(gi / per_row) * head_dim + 32 * (gi % per_row) + lane;
+    } else {
+      idx = (size_t)(kTile * (gi / head_dim) + lane) * head_dim + gi % head_dim;
+    }
+    const float v = __uint_as_float((uint32_t)xh[idx] << 16);
+    double e2;
+    switch (b) {
+      case 2: e2 = group_sse<2>(v); break;
+      case 3: e2 = group_sse<3>(v); break;
+      case 4: e2 = group_sse<4>(v); break;
+      default: e2 = group_sse<8>(v); break;
+    }
+    acc += e2;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) atomicAdd(&sse[(size_t)head * n_bits + bi], acc);
+}
+
+__global__ void scale_kernel(double* v, int n, double f) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) v[i] *= f;
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t st) {
@@ -343,6 +402,20 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
     const int smem = a.flush ? (int)sizeof(TileSmem<64>) : 0;
     append_kernel<64><<<streams, 64, smem, st>>>(a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_measure_distortion(const uint16_t* x, int n_heads, int n_tokens, int head_dim, int role,
+                                      const int* bits, int n_bits, double* mse, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(mse, 0, sizeof(double) * (size_t)n_heads * n_bits, st);
+  if (e != cudaSuccess) return e;
+  for (int bi = 0; bi < n_bits; ++bi) {
+    measure_sse_kernel<<<dim3(64, n_heads), 256, 0, st>>>(x, n_tokens, head_dim, role, bits[bi], bi, n_bits, mse);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int n = n_heads * n_bits;
+  scale_kernel<<<(n + 255) / 256, 256, 0, st>>>(mse, n, 1.0 / ((double)n_tokens * head_dim));
   return cudaGetLastError();
 }
 

@@ -150,3 +150,31 @@ def test_cache_init_rejects_bad_arguments_before_cuda():
     assert lib.rq_decode_attention(None, 0, None, None, 0.0, 0, None, 0, None) == 1
     st = ctypes.c_int(0)
     assert lib.rq_decode_read_status(None, ctypes.byref(st)) == 1
+
+
+def test_fit_distortion_matches_the_oracle():
+    """Host calibration fit and fallback of the library against the oracle."""
+    from oracle import calibration as cal
+    from quantized_decode_attention_head_b200 import rq_fit_distortion
+
+    rng = np.random.default_rng(11)
+    bits = [2, 3, 4, 8]
+    alpha = rng.uniform(0.1, 1.0, 20)
+    beta = rng.uniform(3.0, 6.0, 20)
+    table = alpha[:, None] * beta[:, None] ** -np.array(bits, dtype=np.float64)[None]
+    table *= np.exp(rng.normal(0.0, 0.05, table.shape))  # small scatter
+    table[3] = [1.0, 0.02, 0.4, 0.3]  # a poor fit
+    a_l, b_l, r_l = rq_fit_distortion(bits, table)
+    a_o, b_o, r_o = cal.calibrate(bits, table)
+    assert np.allclose(a_l, a_o, rtol=1e-12) and np.allclose(b_l, b_o, rtol=1e-12)
+    assert np.allclose(r_l, r_o, rtol=1e-12, atol=1e-12)
+    assert r_l[3] < 0.96
+
+
+def test_cap_weights_matches_the_oracle():
+    from oracle import calibration as cal
+    from quantized_decode_attention_head_b200 import rq_cap_weights
+
+    w = np.array([0.5, 1.0, 2.0, 300.0, 1.5])
+    assert np.array_equal(rq_cap_weights(w), cal.cap_weights(w))
+    assert np.array_equal(rq_cap_weights(w, 2.0), cal.cap_weights(w, 2.0))
