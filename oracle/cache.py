@@ -20,6 +20,15 @@ Readings where the pages are silent (also listed in the design doc):
   32 recent tokens are quantized (same rule, same order) into the next tile.
   While T < S the token fills the sink.
 * The recent ring stores token position P at slot (P - S) mod (R + 32).
+* Per-channel K normalization (optional; InnerQ abstract: "per-channel
+  normalization of the key cache, computed once during prefill and folded
+  into the model parameters"): n_d = the smallest power of two >= the
+  absolute maximum of channel d of K over the prefill tokens (1 when that
+  maximum is 0 or nothing was prefilled).  Quantized tiles hold K / n (exact:
+  a power-of-two scaling) and dequantize to n * K_hat; the sink and recent
+  windows keep K as is; queries are multiplied by n (the folding) for the
+  quantized tokens only.  The statistic and the power-of-two rounding are this
+  library's reading; the page gives neither.
 """
 
 from __future__ import annotations
@@ -41,6 +50,15 @@ def split_lengths(n_tokens: int, n_sink: int, n_recent: int):
     return s, tq, n_tokens - s - tq
 
 
+def channel_norm(k: np.ndarray) -> np.ndarray:
+    """Smallest power of two >= max_t |k[t, d]| per channel (1 for a zero
+    channel), float32 [D]."""
+    m = np.max(np.abs(np.asarray(k, dtype=np.float32)), axis=0).astype(np.float64)
+    frac, e = np.frexp(m)  # m = frac * 2^e, frac in [0.5, 1)
+    e = np.where(frac == 0.5, e - 1, e)
+    return np.where(m > 0, np.ldexp(1.0, e), 1.0).astype(np.float32)
+
+
 def ring_slot(pos: int, n_sink: int, n_recent: int) -> int:
     return (pos - n_sink) % (n_recent + TILE)
 
@@ -48,8 +66,10 @@ def ring_slot(pos: int, n_sink: int, n_recent: int) -> int:
 class StreamCache:
     """Quantized cache of one stream, built token by token or by prefill."""
 
-    def __init__(self, head_dim, k_bits, v_bits, n_sink, n_recent):
+    def __init__(self, head_dim, k_bits, v_bits, n_sink, n_recent, k_norm=False):
         self.d = head_dim
+        self.k_norm = k_norm
+        self.nrm = np.ones(head_dim, dtype=np.float32)  # per-channel K normalization n_d
         self.kb = k_bits
         self.vb = v_bits
         self.S = n_sink
@@ -64,6 +84,8 @@ class StreamCache:
     def prefill(self, k: np.ndarray, v: np.ndarray):
         """k, v: float32 [T, D] holding bf16 values."""
         T = k.shape[0]
+        self.nrm = channel_norm(k) if (self.k_norm and T > 0) else np.ones(self.d, dtype=np.float32)
+        kn = (k / self.nrm).astype(np.float32)
         s, tq, r = split_lengths(T, self.S, self.R)
         self.sink_k = [k[i].copy() for i in range(s)]
         self.sink_v = [v[i].copy() for i in range(s)]
@@ -71,7 +93,7 @@ class StreamCache:
         n = tq // TILE
         if n:
             d = self.d
-            qb = qz.quantize_tiles(k[s : s + tq].reshape(n, TILE, d), v[s : s + tq].reshape(n, TILE, d), self.kb, self.vb)
+            qb = qz.quantize_tiles(kn[s : s + tq].reshape(n, TILE, d), v[s : s + tq].reshape(n, TILE, d), self.kb, self.vb)
             self.tiles = [{key: val[i] for key, val in qb.items()} for i in range(n)]
         self.recent = [(p, k[p].copy(), v[p].copy()) for p in range(s + tq, T)]
         self.T = T
@@ -88,7 +110,7 @@ class StreamCache:
         if len(self.recent) == self.R + TILE:
             old = self.recent[:TILE]
             self.recent = self.recent[TILE:]
-            kt = np.stack([o[1] for o in old])
+            kt = (np.stack([o[1] for o in old]) / self.nrm).astype(np.float32)
             vt = np.stack([o[2] for o in old])
             self.tiles.append(qz.quantize_tile(kt, vt, self.kb, self.vb))
             return True
@@ -107,7 +129,7 @@ class StreamCache:
             parts_v.append(np.stack(self.sink_v).astype(np.float64))
         if self.tiles:
             kh, vh = qz.dequantize_tile({key: np.stack([t[key] for t in self.tiles]) for key in self.tiles[0]})
-            parts_k.append(kh.reshape(-1, self.d))
+            parts_k.append(kh.reshape(-1, self.d) * self.nrm.astype(np.float64))
             parts_v.append(vh.reshape(-1, self.d))
         if self.recent:
             parts_k.append(np.stack([r[1] for r in self.recent]).astype(np.float64))

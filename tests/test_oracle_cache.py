@@ -99,3 +99,73 @@ def test_batched_records_equal_single_tile_records(kb, vb, d):
         ref = qz.quantize_tile(k[a : a + 32], v[a : a + 32], kb, vb)
         for key in ref:
             assert np.array_equal(back[key], ref[key]), key
+
+
+# ------------------------------------------------ per-channel K normalization
+def _bf16(x):
+    """Round float32 to the nearest bf16 value (ties to even)."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32).view(np.float32)
+
+
+def test_channel_norm_closed_forms():
+    k = np.zeros((3, 5), dtype=np.float32)
+    k[:, 0] = [0.5, -3.0, 1.0]   # max 3 -> 4
+    k[:, 1] = [4.0, -1.0, 0.0]   # max 4 -> 4 (already a power of two)
+    k[:, 2] = [0.3, 0.1, -0.2]   # max 0.3 -> 0.5
+    k[:, 3] = 0.0                # zero channel -> 1
+    k[:, 4] = [-1e-3, 0.0, 0.0]  # smallest power of two >= 1e-3 is 2^-9
+    n = ca.channel_norm(k)
+    assert n.tolist() == [4.0, 4.0, 0.5, 1.0, 2.0**-9]
+
+
+def test_k_norm_is_invariant_to_power_of_two_channel_scaling():
+    """With normalization, scaling a K channel by 2^j leaves every tile record
+    unchanged and scales the dequantized channel by exactly 2^j."""
+    rng = np.random.default_rng(9)
+    T, d = 4 + 32 * 3 + 40, 64
+    k = _bf16(rng.standard_normal((T, d), dtype=np.float32))
+    v = _bf16(rng.standard_normal((T, d), dtype=np.float32))
+    k2 = k.copy()
+    k2[:, 5] *= np.float32(8.0)
+    k2[:, 17] *= np.float32(0.25)
+    a = ca.StreamCache(d, 2, 3, 4, 32, k_norm=True)
+    b = ca.StreamCache(d, 2, 3, 4, 32, k_norm=True)
+    a.prefill(k, v)
+    b.prefill(k2, v)
+    assert np.array_equal(a.records(), b.records())
+    ka, _ = a.dequantized()
+    kb, _ = b.dequantized()
+    scale = np.ones(d)
+    scale[5], scale[17] = 8.0, 0.25
+    assert np.array_equal(ka * scale, kb)
+
+
+def test_k_norm_reduces_error_on_outlier_channels():
+    rng = np.random.default_rng(4)
+    T, d = 4 + 32 * 40 + 32, 128
+    f = np.exp(rng.standard_normal(d) * 1.5).astype(np.float32)
+    k = _bf16(rng.standard_normal((T, d), dtype=np.float32) * f)
+    v = _bf16(rng.standard_normal((T, d), dtype=np.float32))
+    err = {}
+    for norm in (False, True):
+        st = ca.StreamCache(d, 2, 2, 4, 32, k_norm=norm)
+        st.prefill(k, v)
+        kh, _ = st.dequantized()
+        # relative error per channel, averaged: outlier channels no longer
+        # coarsen the groups they share with small channels
+        err[norm] = np.mean(np.abs(kh - k) / (np.abs(k).max(axis=0) + 1e-30))
+    assert err[True] < 0.8 * err[False]
+
+
+def test_k_norm_without_prefill_is_the_identity():
+    rng = np.random.default_rng(5)
+    d = 64
+    a = ca.StreamCache(d, 2, 2, 2, 0, k_norm=True)
+    b = ca.StreamCache(d, 2, 2, 2, 0, k_norm=False)
+    for _ in range(40):
+        kk = _bf16(rng.standard_normal(d, dtype=np.float32) * 5)
+        vv = _bf16(rng.standard_normal(d, dtype=np.float32))
+        a.append(kk, vv)
+        b.append(kk, vv)
+    assert np.array_equal(a.records(), b.records())
