@@ -62,7 +62,8 @@
  *     s = fp16(min((max - min) / (2^b - 1), 65504)), z = min (bf16),
  *     c = clamp(rint((x - z) * (s > 0 ? 1/s : 0)), 0, 2^b - 1).
  *   Windows per stream: sink K [S][D], sink V [S][D], recent ring K [R+32][D],
- *   ring V [R+32][D] (bf16); token position P >= S sits in ring slot
+ *   ring V [R+32][D] (bf16), then the K normalization factors n [D] (fp32,
+ *   powers of two; all 1 unless k_norm); token position P >= S sits in ring slot
  *   (P - S) mod (R + 32).  With T tokens, Tq = 32*floor((T - S - R)/32) tokens
  *   (0 when T < S + R) are quantized; the rest stay bf16.
  */
@@ -159,6 +160,10 @@ typedef struct {
   int max_tokens;    /* capacity per sequence */
   const int* k_bits; /* host [L*Hkv] in {2,3,4,8}, index l*Hkv + h (copied) */
   const int* v_bits; /* host [L*Hkv] in {2,3,4,8} (copied) */
+  int k_norm;        /* 1: per-channel K normalization (InnerQ abstract): rq_quantize_kv sets
+                        n_d = smallest power of two >= max_t |K[t, d]| per stream and channel
+                        over the prefill tokens, tiles hold K / n, queries are multiplied by n
+                        for the quantized tokens; 0: n = 1.  Windows keep K as is. */
 } rq_cache_config;
 
 typedef struct rq_cache rq_cache; /* opaque host handle */
@@ -168,7 +173,8 @@ rq_status rq_cache_bytes(const rq_cache_config* cfg, size_t* bytes);
 
 /* Bind a caller-owned device buffer (>= rq_cache_bytes, 256-byte aligned) to
  * a new host handle with length 0.  Writes the buffer's descriptor header with
- * a synchronous cudaMemcpy on the current device (the only blocking call
+ * a synchronous cudaMemcpy on the current device and sets every stream's K
+ * normalization factors to 1, waiting for both (the only blocking call
  * besides rq_decode_read_status).  *out receives the handle. */
 rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes, rq_cache** out);
 

@@ -44,6 +44,7 @@ class CacheConfig(ctypes.Structure):
         ("max_tokens", ctypes.c_int),
         ("k_bits", ctypes.POINTER(ctypes.c_int)),
         ("v_bits", ctypes.POINTER(ctypes.c_int)),
+        ("k_norm", ctypes.c_int),
     ]
 
 

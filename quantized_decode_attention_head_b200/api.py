@@ -108,13 +108,14 @@ def rq_cap_weights(w, factor=5.0):
     return out
 
 
-def _config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, n_sink, n_recent, max_tokens, k_bits, v_bits, group=32):
+def _config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, n_sink, n_recent, max_tokens, k_bits, v_bits, group=32,
+            k_norm=False):
     kb = np.ascontiguousarray(np.asarray(k_bits, dtype=np.int32).reshape(-1))
     vb = np.ascontiguousarray(np.asarray(v_bits, dtype=np.int32).reshape(-1))
     ip = ctypes.POINTER(ctypes.c_int)
     cfg = CacheConfig(
         n_layers, batch, n_q_heads, n_kv_heads, head_dim, group, n_sink, n_recent, max_tokens,
-        kb.ctypes.data_as(ip), vb.ctypes.data_as(ip),
+        kb.ctypes.data_as(ip), vb.ctypes.data_as(ip), int(bool(k_norm)),
     )
     return cfg, (kb, vb)
 
@@ -130,7 +131,7 @@ class QuantizedKVCache:
     """Owns a device buffer (torch uint8 tensor) and the library's host handle."""
 
     def __init__(self, n_layers, batch, n_q_heads, n_kv_heads, head_dim, n_sink, n_recent, max_tokens,
-                 k_bits, v_bits, device="cuda", group=32):
+                 k_bits, v_bits, device="cuda", group=32, k_norm=False):
         import torch
 
         self.n_layers, self.batch = n_layers, batch
@@ -139,7 +140,8 @@ class QuantizedKVCache:
         self.k_bits = np.asarray(k_bits, dtype=np.int32).reshape(n_layers, n_kv_heads)
         self.v_bits = np.asarray(v_bits, dtype=np.int32).reshape(n_layers, n_kv_heads)
         cfg, keep = _config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, n_sink, n_recent, max_tokens,
-                            self.k_bits, self.v_bits, group)
+                            self.k_bits, self.v_bits, group, k_norm)
+        self.k_norm = bool(k_norm)
         nbytes = ctypes.c_size_t(0)
         check("rq_cache_bytes", lib().rq_cache_bytes(ctypes.byref(cfg), ctypes.byref(nbytes)))
         self.nbytes = nbytes.value
@@ -163,6 +165,16 @@ class QuantizedKVCache:
         t = ctypes.c_int(0)
         check("rq_cache_length", lib().rq_cache_length(self.handle, layer, ctypes.byref(t)))
         return t.value
+
+    def k_norm_factors(self, layer, b, kv_head):
+        """The stream's per-channel K normalization factors n[D] (a device view)."""
+        import torch
+
+        lay = self.stream_layout(layer, b, kv_head)
+        d = self.head_dim
+        rows = (2 * self.n_sink + 2 * (self.n_recent + 32)) * d * 2
+        off = lay["window_offset"] + rows
+        return self.buffer[off : off + 4 * d].view(torch.float32)
 
     def stream_layout(self, layer, b, kv_head):
         to, wo = ctypes.c_size_t(0), ctypes.c_size_t(0)

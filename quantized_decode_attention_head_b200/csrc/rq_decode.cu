@@ -87,7 +87,7 @@ __device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) 
 // split into two s8 terms q_int = 256 q1 + q2, laid out as the k32 x n8
 // B-fragments of the q.K^T MMA (column n = 2 * head + term).
 template <int D, int G, int KB, int VB>
-__device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, float scale_log2, int lane) {
+__device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, const float* nrm, float scale_log2, int lane) {
   using C = Cfg<D, G>;
   const int gid = lane >> 2, tig = lane & 3;
   const int hl = gid >> 1, tau = gid & 1;
@@ -105,9 +105,12 @@ __device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, float scale
         uint2 u = make_uint2(0u, 0u);
         if (hv) u = __ldg(reinterpret_cast<const uint2*>(qp + 32 * g + 16 * kh + 4 * tig));
         const uint32_t w[2] = {u.x, u.y};
+        // K normalization folded into q for the packed tiles: q_d * n_d (exact, powers of two)
+        const float4 nv = *reinterpret_cast<const float4*>(nrm + 32 * g + 16 * kh + 4 * tig);
+        const float nn[4] = {nv.x, nv.y, nv.z, nv.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float x = bf16_bits_to_float(e & 1 ? w[e >> 1] >> 16 : w[e >> 1] & 0xFFFFu);
+          const float x = bf16_bits_to_float(e & 1 ? w[e >> 1] >> 16 : w[e >> 1] & 0xFFFFu) * nn[e];
           qv[g][4 * kh + e] = x;
           mx = fmaxf(mx, fabsf(x));
         }
@@ -383,7 +386,8 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
 // slot as soon as the warp has read it, so the warp never waits on another
 // warp and every warp keeps `stages` records in flight.
 template <int D, int G, int KB, int VB>
-__device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log2, uint8_t* ring, int stages,
+__device__ void consume(WarpState<D, G>& st, const uint16_t* qh, const float* nrm, float scale_log2, uint8_t* ring,
+                        int stages,
                         int stage_bytes, uint64_t* bars, float* scratch, const uint8_t* src, int rec, int n_my,
                         int warp, int lane, volatile int* abort_flag, int* status) {
   using C = Cfg<D, G>;
@@ -399,7 +403,7 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
     }
   }
   griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
-  setup_query<D, G, KB, VB>(st, qh, scale_log2, lane);
+  setup_query<D, G, KB, VB>(st, qh, nrm, scale_log2, lane);
   float* ks = scratch;
   float* vs = scratch + 8 * C::KSTR;
   const int VOFF = blob_bytes(KB, D) + 4 * D;
@@ -446,12 +450,12 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, float scale_log
 
 template <int D, int G>
 __device__ __forceinline__ void consume_dispatch(int kb, int vb, WarpState<D, G>& st, const uint16_t* qh,
-                                                 float scale_log2, uint8_t* ring, int stages, int stage_bytes,
+                                                 const float* nrm, float scale_log2, uint8_t* ring, int stages, int stage_bytes,
                                                  uint64_t* bars, float* scratch, const uint8_t* src, int rec,
                                                  int n_my, int warp, int lane, volatile int* abort_flag,
                                                  int* status) {
 #define RQ_C(KBV, VBV)                                                                                       \
-  consume<D, G, KBV, VBV>(st, qh, scale_log2, ring, stages, stage_bytes, bars, scratch, src, rec, n_my, warp, \
+  consume<D, G, KBV, VBV>(st, qh, nrm, scale_log2, ring, stages, stage_bytes, bars, scratch, src, rec, n_my, warp, \
                           lane, abort_flag, status)
 #define RQ_V(KBV)                  \
   switch (vb) {                    \
@@ -743,7 +747,10 @@ __global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecode
     const int rec = hd.rec_bytes;
     const uint8_t* src = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)t0 * rec;
     if (warp < NW)
-      consume_dispatch<D, G>(hd.k_bits, hd.v_bits, st, qh, a.scale_log2,
+      consume_dispatch<D, G>(hd.k_bits, hd.v_bits, st, qh,
+                             reinterpret_cast<const float*>(a.buf + hd.win_base + (int64_t)b * a.g.win_bytes +
+                                                            window_rows_bytes(a.g.S, a.g.R, D)),
+                             a.scale_log2,
                              area + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
                              bars + warp * kMaxStages, reinterpret_cast<float*>(smem) + warp * C::SCRATCH, src, rec,
                              t1 - t0, warp, lane, &abort_flag, a.status);

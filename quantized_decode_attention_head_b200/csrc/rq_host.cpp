@@ -21,6 +21,7 @@ struct rq_cache {
   size_t bytes;
   std::vector<int> length;  // tokens per layer
   int sm_count;
+  int k_norm;               // per-channel K normalization set by the prefill
 };
 
 namespace {
@@ -215,8 +216,11 @@ rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes,
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) c->sm_count = n;
   }
-  const cudaError_t e =
-      cudaMemcpy(c->buf, c->desc.data(), c->desc.size() * sizeof(HeadDesc), cudaMemcpyHostToDevice);
+  c->k_norm = cfg->k_norm ? 1 : 0;
+  cudaError_t e = cudaMemcpy(c->buf, c->desc.data(), c->desc.size() * sizeof(HeadDesc), cudaMemcpyHostToDevice);
+  // normalization factors start at 1 (a cache built by appends only)
+  if (e == cudaSuccess) e = rq::launch_norm_reset(c->buf, reinterpret_cast<const HeadDesc*>(c->buf), c->g, 0);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(0);
   if (e != cudaSuccess) {
     delete c;
     return RQ_ERR_CUDA;
@@ -256,6 +260,7 @@ rq_status rq_quantize_kv(rq_cache* c, const void* k, const void* v, int n_tokens
   a.v = static_cast<const uint16_t*>(v);
   a.T = n_tokens;
   a.Tq = rq::quantized_tokens(n_tokens, c->g.S, c->g.R);
+  a.k_norm = c->k_norm;
   if (n_tokens > 0) {
     const rq_status st = cuda_status(rq::launch_quantize(a, stream));
     if (st != RQ_OK) return st;

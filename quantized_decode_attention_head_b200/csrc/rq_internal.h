@@ -38,10 +38,12 @@ __host__ __device__ constexpr int record_bytes(int kb, int vb, int d) {
   return blob_bytes(kb, d) + 4 * d + blob_bytes(vb, d) + 4 * d;
 }
 
-// Window block of one stream: [sink K][sink V][ring K][ring V], bf16 rows of D.
-__host__ __device__ inline int64_t window_bytes(int S, int R, int D) {
+// Window block of one stream: [sink K][sink V][ring K][ring V] bf16 rows of D,
+// then the per-channel K normalization factors n[D] (fp32).
+__host__ __device__ inline int64_t window_rows_bytes(int S, int R, int D) {
   return (int64_t)(2 * S + 2 * (R + kTile)) * D * 2;
 }
+__host__ __device__ inline int64_t window_bytes(int S, int R, int D) { return window_rows_bytes(S, R, D) + 4 * D; }
 
 // Quantized token count for T tokens (multiple of 32; recent window in [R, R+32)).
 __host__ __device__ inline int quantized_tokens(int T, int S, int R) {
@@ -56,6 +58,7 @@ struct QuantizeArgs {
   const uint16_t* v;
   int T;
   int Tq;
+  int k_norm;          // set n from the prefill (1) or to 1 (0)
 };
 
 struct AppendArgs {
@@ -136,6 +139,8 @@ inline int window_items(int T, int S, int R) {
 
 // Kernel launchers (rq_kernels.cu).  Return cudaGetLastError() after launch.
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
+// Sets every stream's K normalization factors to 1 (cache initialisation).
+cudaError_t launch_norm_reset(uint8_t* buf, const HeadDesc* desc, const Geom& g, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 // Mean squared quantization error per (head, bit width) of bf16 samples
 // x [n_heads][n_tokens][head_dim]; role 0 = K groups, 1 = V groups.

@@ -30,7 +30,19 @@ struct TileSmem {
   float kz[kTile][D / 32];  // zero per (token, group)
   float vr[D];
   float vz[D];
+  float kinv[D];  // 1 / n per channel (K normalization; powers of two)
 };
+
+// Stream's K normalization factors n[D] (fp32), stored after its window rows.
+__device__ __forceinline__ float* stream_norm(uint8_t* buf, const HeadDesc& hd, const Geom& g, int b) {
+  return reinterpret_cast<float*>(buf + hd.win_base + (int64_t)b * g.win_bytes + window_rows_bytes(g.S, g.R, g.D));
+}
+
+// 1 / n of the stream into shared memory (one warp).
+template <int D>
+__device__ __forceinline__ void stage_kinv(TileSmem<D>& sm, const float* nrm, int lane) {
+  for (int d = lane; d < D; d += 32) sm.kinv[d] = 1.0f / nrm[d];
+}
 
 __device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -79,9 +91,11 @@ __device__ void pack_k(TileSmem<D>& sm, uint8_t* rec, int lane) {
       float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const uint32_t w = sm.k[t][grp * 16 + ((c + (t >> 3)) & 15)];
-        mn = fminf(mn, fminf(lo_bf16(w), hi_bf16(w)));
-        mx = fmaxf(mx, fmaxf(lo_bf16(w), hi_bf16(w)));
+        const int cw = grp * 16 + ((c + (t >> 3)) & 15);
+        const uint32_t w = sm.k[t][cw];
+        const float x0 = lo_bf16(w) * sm.kinv[2 * cw], x1 = hi_bf16(w) * sm.kinv[2 * cw + 1];
+        mn = fminf(mn, fminf(x0, x1));
+        mx = fmaxf(mx, fmaxf(x0, x1));
       }
       float r;
       const uint32_t meta = group_params<KB>(mn, mx, r);
@@ -107,8 +121,8 @@ __device__ void pack_k(TileSmem<D>& sm, uint8_t* rec, int lane) {
         const int t = gid + 8 * i, d0 = 32 * g + 16 * kh + 4 * tig + e;
         const uint32_t x = sm.k[t][d0 / 2];
         const float rr = sm.kr[t][g], z = sm.kz[t][g];
-        put_code<KB, W>(words, rho, kh, e, code_of<KB>(lo_bf16(x), z, rr));
-        put_code<KB, W>(words, rho, kh, e + 1, code_of<KB>(hi_bf16(x), z, rr));
+        put_code<KB, W>(words, rho, kh, e, code_of<KB>(lo_bf16(x) * sm.kinv[d0], z, rr));
+        put_code<KB, W>(words, rho, kh, e + 1, code_of<KB>(hi_bf16(x) * sm.kinv[d0 + 1], z, rr));
       }
 #pragma unroll
   for (int c = 0; c < W / 4; ++c)
@@ -210,6 +224,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quantize_tiles_kernel(Quanti
   }
   stage_rows<D>(sm.k, krows, lane);
   stage_rows<D>(sm.v, vrows, lane);
+  stage_kinv<D>(sm, stream_norm(a.buf, hd, a.g, b), lane);
   __syncwarp();
   uint8_t* rec = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)tile * hd.rec_bytes;
   quantize_staged_tile<D>(sm, hd.k_bits, hd.v_bits, rec, lane);
@@ -284,6 +299,7 @@ __global__ void __launch_bounds__(64) append_kernel(AppendArgs a) {
     krows[t] = reinterpret_cast<const uint16_t*>(win + ((size_t)2 * S + slot) * D * 2);
     vrows[t] = reinterpret_cast<const uint16_t*>(win + ((size_t)2 * S + ring + slot) * D * 2);
   }
+  if (warp == 0) stage_kinv<D>(sm, stream_norm(a.buf, hd, a.g, b), lane);
   // rows were just written through global memory by this block: plain loads
 #pragma unroll 4
   for (int j = tid; j < kTile * kChunks; j += 64) {
@@ -370,10 +386,66 @@ __global__ void scale_kernel(double* v, int n, double f) {
   if (i < n) v[i] *= f;
 }
 
+// K normalization factors of every stream: set to a constant (1 at cache
+// initialisation and for prefills without normalization, 0 before a maximum).
+__global__ void norm_fill_kernel(uint8_t* buf, const HeadDesc* desc, Geom g, float value) {
+  const int s = blockIdx.x;
+  const int h = s % g.Hkv, b = (s / g.Hkv) % g.B, l = s / (g.Hkv * g.B);
+  const HeadDesc hd = desc[l * g.Hkv + h];
+  float* n = stream_norm(buf, hd, g, b);
+  for (int d = threadIdx.x; d < g.D; d += blockDim.x) n[d] = value;
+}
+
+// max over the prefill tokens of |K[t, d]| per stream and channel, as the
+// bits of a non-negative float (ordered like unsigned integers)
+__global__ void norm_max_kernel(QuantizeArgs a, int tokens_per_block) {
+  const int s = blockIdx.y;
+  const int h = s % a.g.Hkv, b = (s / a.g.Hkv) % a.g.B, l = s / (a.g.Hkv * a.g.B);
+  const HeadDesc hd = a.desc[l * a.g.Hkv + h];
+  const int D = a.g.D;
+  const int t0 = blockIdx.x * tokens_per_block, t1 = min(a.T, t0 + tokens_per_block);
+  const uint16_t* k = a.k + (size_t)s * a.T * D;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float m = 0.0f;
+    for (int t = t0; t < t1; ++t) m = fmaxf(m, fabsf(__uint_as_float((uint32_t)k[(size_t)t * D + d] << 16)));
+    atomicMax(reinterpret_cast<unsigned int*>(stream_norm(a.buf, hd, a.g, b)) + d, __float_as_uint(m));
+  }
+}
+
+// maximum -> smallest power of two >= it (1 for a zero channel)
+__global__ void norm_finalize_kernel(QuantizeArgs a) {
+  const int s = blockIdx.x;
+  const int h = s % a.g.Hkv, b = (s / a.g.Hkv) % a.g.B, l = s / (a.g.Hkv * a.g.B);
+  const HeadDesc hd = a.desc[l * a.g.Hkv + h];
+  float* n = stream_norm(a.buf, hd, a.g, b);
+  for (int d = threadIdx.x; d < a.g.D; d += blockDim.x) {
+    const float m = n[d];
+    int e = 0;
+    const float f = frexpf(m, &e);  // m = f * 2^e, f in [0.5, 1)
+    n[d] = m > 0.0f ? ldexpf(1.0f, f == 0.5f ? e - 1 : e) : 1.0f;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_norm_reset(uint8_t* buf, const HeadDesc* desc, const Geom& g, cudaStream_t st) {
+  norm_fill_kernel<<<g.L * g.B * g.Hkv, 128, 0, st>>>(buf, desc, g, 1.0f);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t st) {
   const int streams = a.g.L * a.g.B * a.g.Hkv;
+  // the prefill fixes the K normalization factors before any tile is packed
+  if (a.k_norm && a.T > 0) {
+    norm_fill_kernel<<<streams, 128, 0, st>>>(a.buf, a.desc, a.g, 0.0f);
+    const int tpb = 1024;
+    norm_max_kernel<<<dim3((a.T + tpb - 1) / tpb, streams), 128, 0, st>>>(a, tpb);
+    norm_finalize_kernel<<<streams, 128, 0, st>>>(a);
+  } else {
+    norm_fill_kernel<<<streams, 128, 0, st>>>(a.buf, a.desc, a.g, 1.0f);
+  }
+  cudaError_t e0 = cudaGetLastError();
+  if (e0 != cudaSuccess) return e0;
   const int n_tiles = a.Tq / kTile;
   if (n_tiles > 0) {
     dim3 grid((n_tiles + kQuantWarps - 1) / kQuantWarps, streams);

@@ -46,17 +46,17 @@ def workload_bits(wl):
     return (lk, lv), (ok, ov)
 
 
-def make_cache(wl, k_bits, v_bits, max_tokens):
+def make_cache(wl, k_bits, v_bits, max_tokens, k_norm=False):
     return QuantizedKVCache(wl.n_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n_sink,
-                            wl.n_recent, max_tokens, k_bits, v_bits)
+                            wl.n_recent, max_tokens, k_bits, v_bits, k_norm=k_norm)
 
 
-def oracle_streams(wl, k_bits, v_bits, k_np, v_np, which):
+def oracle_streams(wl, k_bits, v_bits, k_np, v_np, which, k_norm=False):
     """Oracle StreamCache for each (l, b, h) in ``which`` from float32 inputs
     [L, B, H, T, D]."""
     out = {}
     for (l, b, h) in which:
-        st = ca.StreamCache(wl.head_dim, int(k_bits[l, h]), int(v_bits[l, h]), wl.n_sink, wl.n_recent)
+        st = ca.StreamCache(wl.head_dim, int(k_bits[l, h]), int(v_bits[l, h]), wl.n_sink, wl.n_recent, k_norm=k_norm)
         st.prefill(k_np[l, b, h], v_np[l, b, h])
         out[(l, b, h)] = st
     return out
@@ -91,6 +91,7 @@ def check_stream_bytes(cache: QuantizedKVCache, st: ca.StreamCache, l, b, h, til
     for (kind, kv, slot), bits in st.window_rows().items():
         row = (slot + (S if kv == "v" else 0)) if kind == "sink" else (2 * S + slot + (ring if kv == "v" else 0))
         assert np.array_equal(win[row * d : (row + 1) * d], bits), (kind, kv, slot)
+    assert np.array_equal(cache.k_norm_factors(l, b, h).cpu().numpy(), st.nrm)
 
 
 def oracle_decode(wl, streams, q_np, which_lb):

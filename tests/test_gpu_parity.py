@@ -164,6 +164,37 @@ def test_decode_step_equals_append_then_decode(S, R, context):
     assert QuantizedKVCache.rq_decode_read_status(ws) == 0
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_k_norm_prefill_decode_and_steps(d):
+    """Per-channel K normalization: factors, tile records and window rows bit
+    for bit against the oracle after the prefill and after fused steps across
+    tile flushes; decoded outputs within the parity tolerance."""
+    wl = _small(head_dim=d, n_q_heads=16, n_kv_heads=4, k_sigma=1.0, context=4 + 32 * 5 + 32 + 7)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    steps = 40
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, wl.context + steps, k_norm=True)
+    cache.rq_quantize_kv(k, v)
+    st = oracle_streams(wl, kb, vb, to_f32(k), to_f32(v), all_streams(wl), k_norm=True)
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    q, kn, vn = workloads.step_inputs(wl, steps, f, "cuda")
+    knp, vnp, qnp = to_f32(kn), to_f32(vn), to_f32(q).astype(np.float64)
+    ws = cache.make_workspace()
+    for t in range(steps):
+        for (l, b, h), s in st.items():
+            s.append(knp[t, l, b, h], vnp[t, l, b, h])
+        out = cache.rq_decode_step(-1, q[t].contiguous(), kn[t].contiguous(), vn[t].contiguous(),
+                                   workspace=ws).cpu().numpy()
+        if t % 7 == 0 or t == steps - 1:
+            exp = oracle_decode(wl, st, qnp[t], [(l, b) for l in range(wl.n_layers) for b in range(wl.batch)])
+            for (l, b), e in exp.items():
+                assert_close(out[l, b], e, f"k_norm step {t} layer {l} b {b}")
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+
+
 def test_append_from_empty_fills_sink_then_ring():
     wl = _small(n_layers=1, batch=1, context=0)
     kb, vb = _bits_grid(1, wl.n_kv_heads)

@@ -106,13 +106,14 @@ def _cfg(**kw):
 def test_cache_bytes_accounting():
     c = _cfg()
     n = rq_cache_bytes(**c)
-    # header + per-head tile regions + windows, each region 256-aligned
+    # header + per-head tile regions + windows (bf16 rows, then D fp32 K
+    # normalization factors), each region 256-aligned
     tiles = (512 - 4 - 32) // 32
     rec = {2: 4 * 128 * 2 + 512, 3: 7 * 128 * 2 + 512, 4: 8 * 128 * 2 + 512, 8: 16 * 128 * 2 + 512}
     expect = 256
     for b in (2, 3, 4, 8):
         expect += -(-(tiles * rec[b]) // 256) * 256
-    expect += 4 * -(-((2 * 4 + 2 * 64) * 64 * 2) // 256) * 256
+    expect += 4 * -(-((2 * 4 + 2 * 64) * 64 * 2 + 4 * 64) // 256) * 256
     assert n == expect
 
 
