@@ -218,6 +218,22 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ GPU arm
+def aggregate_ranks(elapsed, step_bytes, e2e_elapsed, e2e_bytes, world, device):
+    """Whole-job figures of the replicas: bytes summed over ranks, time of the
+    slowest rank (both the device-timed loop and the end-to-end loop)."""
+    if world <= 1:
+        return elapsed, step_bytes, e2e_elapsed, e2e_bytes
+    import torch
+    import torch.distributed as dist
+
+    vals = torch.tensor([elapsed, step_bytes, e2e_elapsed, e2e_bytes], dtype=torch.float64, device=device)
+    mx = vals.clone()
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    sm = vals.clone()
+    dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+    return mx[0].item(), sm[1].item(), mx[2].item(), sm[3].item()
+
+
 def traffic_record():
     """ncu DRAM traffic of the decode kernel recorded for the current sources."""
     import hashlib
@@ -386,19 +402,11 @@ def run_gpu(args):
     h2d = dev_in[0].numel() * 2
     d2h = host_out.numel() * 4
 
-    # aggregate over ranks: bytes summed, time = slowest rank
-    vals = torch.tensor([elapsed, step_bytes, e2e_elapsed, e2e_bytes, dec_avg], dtype=torch.float64, device="cuda")
+    elapsed_all, bytes_all, e2e_el_all, e2e_b_all = aggregate_ranks(elapsed, step_bytes, e2e_elapsed, e2e_bytes,
+                                                                    world, "cuda")
     if world > 1:
-        mx = vals.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = vals.clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        elapsed_all, bytes_all = mx[0].item(), sm[1].item()
-        e2e_el_all, e2e_b_all = mx[2].item(), sm[3].item()
         dist.barrier()
         dist.destroy_process_group()
-    else:
-        elapsed_all, bytes_all, e2e_el_all, e2e_b_all = elapsed, step_bytes, e2e_elapsed, e2e_bytes
     if rank != 0:
         return 0
 
