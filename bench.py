@@ -41,6 +41,7 @@ if ROOT not in sys.path:
 
 METRIC = "quantized-KV decode attention: effective HBM GB/s & µs/step; quantize GB/s"
 WORKLOAD = "long_128k"
+L2_BYTES = 126_000_000
 
 
 def _peaks():
@@ -215,6 +216,168 @@ def run_reference(args):
     }
     print(json.dumps(line))
     return 0
+
+
+# ------------------------------------------------------ secondary measurements
+def workload_bits(wl):
+    """Per-(layer, kv-head) K and V bit widths of a workload from the host
+    allocation (one shared budget, or separate K and V budgets)."""
+    from quantized_decode_attention_head_b200 import rq_allocate_bits, workloads
+
+    inp = workloads.allocation_inputs(wl)
+    shape = (wl.n_layers, wl.n_kv_heads)
+    if "kv" in inp:
+        w, a, b, avg = inp["kv"]
+        kb = rq_allocate_bits(w, a, b, avg, wl.allowed)["b_int"].reshape(shape)
+        return kb, kb
+    return tuple(rq_allocate_bits(*inp[key], wl.allowed)["b_int"].reshape(shape) for key in ("k", "v"))
+
+
+def _bits_text(kb, vb):
+    cnt = lambda x: ",".join(f"{b}:{int((x == b).sum())}" for b in sorted(set(x.ravel().tolist())))
+    return f"K {{{cnt(kb)}}} V {{{cnt(vb)}}} heads per bit width"
+
+
+def sweep_workloads(names, peak, launches=20):
+    """Prefill quantize and one decode of every layer in one launch
+    (rq_decode_attention, layer -1) on other benchmark caches.  A cache
+    smaller than twice the 126 MB L2 is decoded round-robin over enough
+    copies to span twice the L2.  Device time by CUDA events around `launches`
+    back-to-back launches after 3 warm-up launches."""
+    import torch
+
+    from quantized_decode_attention_head_b200 import QuantizedKVCache, workloads
+
+    res = {}
+    stream = torch.cuda.current_stream()
+    for name in names:
+        try:
+            wl = workloads.CONFIGS[name]
+            kb, vb = workload_bits(wl)
+            caches, qs, qtime, qbytes = [], [], None, 0
+            ncopy = 1
+            c = 0
+            while c < ncopy:
+                k, v, f = workloads.kv_inputs(wl, "cuda", seed=wl.seed + 100 * c)
+                cache = QuantizedKVCache(wl.n_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                                         wl.n_sink, wl.n_recent, wl.context + 64, kb, vb)
+                cache.rq_quantize_kv(k, v)  # first call pays one-time set-up
+                torch.cuda.synchronize()
+                if c == 0:
+                    rec = [[cache.stream_layout(l, 0, h)["record_bytes"] for h in range(wl.n_kv_heads)]
+                           for l in range(wl.n_layers)]
+                    dbytes = decode_bytes(wl, rec, wl.context)
+                    ncopy = max(1, -(-2 * L2_BYTES // dbytes))  # the copies span twice the L2
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    cache.rq_quantize_kv(k, v)
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    qtime = e0.elapsed_time(e1) / 1e3
+                    qbytes = k.numel() * 2 * 2 + dbytes
+                del k, v
+                q = workloads.step_inputs(wl, 1, f, "cuda", seed=wl.seed + 100 * c)[0][0].contiguous()
+                caches.append(cache)
+                qs.append(q)
+                c += 1
+            ws = caches[0].make_workspace()
+            out = torch.empty(qs[0].shape, dtype=torch.float32, device="cuda")
+            for i in range(3):
+                caches[i % ncopy].rq_decode_attention(-1, qs[i % ncopy], out=out, workspace=ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(launches):
+                caches[i % ncopy].rq_decode_attention(-1, qs[i % ncopy], out=out, workspace=ws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if QuantizedKVCache.rq_decode_read_status(ws) != 0:
+                raise RuntimeError("device status")
+            t = e0.elapsed_time(e1) / 1e3 / launches
+            res[name] = {"decode_us": t * 1e6, "decode_gbs": dbytes / t / 1e9, "frac": dbytes / t / 1e9 / peak,
+                         "bytes_per_launch": dbytes, "streams": wl.n_layers * wl.batch * wl.n_kv_heads,
+                         "context": wl.context, "copies": ncopy, "bits": _bits_text(kb, vb),
+                         "quantize_gbs": qbytes / qtime / 1e9}
+            del caches, qs, ws, out
+            torch.cuda.empty_cache()
+        except Exception as exc:  # a secondary figure never hides the main line
+            res[name] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+    return res
+
+
+def step_loop_graph(steps=64, copies=4, replays=20):
+    """The Llama-3-8B-shaped workload's decode loop -- `steps` serving steps
+    (rq_decode_step: append + decode) over `copies` caches round-robin --
+    timed per step as eager launches and as one CUDA graph of the whole loop.
+    The graph is captured on a second, identical set of caches; its first
+    replay performs the same steps on the same data, so its outputs must equal
+    the eager loop's bit for bit.  Later replays repeat the captured steps
+    (same lengths, same slots) and time the loop."""
+    import torch
+
+    from quantized_decode_attention_head_b200 import QuantizedKVCache, workloads
+
+    wl = workloads.CONFIGS["llama3_8b"]
+    kb, vb = workload_bits(wl)
+    per = -(-steps // copies)
+    stream = torch.cuda.current_stream()
+
+    def make_set():
+        cs, ins = [], []
+        for c in range(copies):
+            k, v, f = workloads.kv_inputs(wl, "cuda", seed=wl.seed + 100 * c)
+            cache = QuantizedKVCache(wl.n_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n_sink,
+                                     wl.n_recent, wl.context + per + 32, kb, vb)
+            cache.rq_quantize_kv(k, v)
+            del k, v
+            cs.append(cache)
+            ins.append(workloads.step_inputs(wl, per, f, "cuda", seed=wl.seed + 100 * c))
+        return cs, ins
+
+    shape = (wl.batch, wl.n_q_heads, wl.head_dim)
+    eager_set, ins = make_set()
+    graph_set, _ = make_set()
+    ws_e, ws_g = eager_set[0].make_workspace(), graph_set[0].make_workspace()
+    out_e = torch.empty((steps,) + shape, dtype=torch.float32, device="cuda")
+    out_g = torch.empty_like(out_e)
+    # one decode without append on every cache: one-time host set-up outside the loops
+    for cs, ws in ((eager_set, ws_e), (graph_set, ws_g)):
+        for c in range(copies):
+            cs[c].rq_decode_attention(0, ins[c][0][0, 0], out=out_e[0], workspace=ws)
+    torch.cuda.synchronize()
+
+    def loop(cs, ws, out):
+        for i in range(steps):
+            c, j = i % copies, i // copies
+            q, kn, vn = ins[c]
+            cs[c].rq_decode_step(0, q[j, 0], kn[j, 0], vn[j, 0], out=out[i], workspace=ws)
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    loop(eager_set, ws_e, out_e)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    eager_us = e0.elapsed_time(e1) * 1e3 / steps
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        loop(graph_set, ws_g, out_g)
+    g.replay()
+    torch.cuda.synchronize()
+    same = bool(torch.equal(out_e, out_g))
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(replays):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    graph_us = e0.elapsed_time(e1) * 1e3 / (steps * replays)
+    st = (QuantizedKVCache.rq_decode_read_status(ws_e), QuantizedKVCache.rq_decode_read_status(ws_g))
+    del g
+    return {"steps": steps, "copies": copies, "eager_us_per_step": eager_us, "graph_us_per_step": graph_us,
+            "graph_equals_eager": same, "device_status": list(st), "bits": _bits_text(kb, vb),
+            "note": "eager: one timed pass of the loop (first use of each length); graph: mean of "
+                    f"{replays} replays"}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -424,6 +587,13 @@ def run_gpu(args):
         cpu = {"value": res["decode_gbs"], "unit": "GB/s", "cores": res["threads"], "kind": "oracle",
                "sample": res["sample"]}
     clk = clocks.summary()
+    extra = {}
+    if world == 1 and not args.no_sweep:
+        try:
+            extra["llama3_8b_step_loop"] = step_loop_graph()
+        except Exception as exc:  # a secondary figure never hides the main line
+            extra["llama3_8b_step_loop"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        extra["workloads"] = sweep_workloads(["llama3_8b", "mistral_7b_b64", "qwen3_8b"], peak)
     line = {
         "metric": METRIC,
         "value": bytes_all / elapsed_all / 1e9,
@@ -454,6 +624,7 @@ def run_gpu(args):
         "cpu_baseline": cpu,
         "clocks": clk,
     }
+    line.update(extra)
     print(json.dumps(line))
     return 0
 
@@ -468,6 +639,8 @@ def main():
     ap.add_argument("--copies", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the secondary figures (other workloads, CUDA-graph step loop)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -5,20 +5,25 @@
 // recent window (items n_splits..).  Four warps process tiles; lane 0 of each
 // streams the warp's own tile records into a private ring of shared-memory
 // stages with 1-D bulk copies (cp.async.bulk, TMA engine) completing on
-// mbarriers.  The last CTA
-// of a stream to finish merges all items' partial softmax states
-// (log-sum-exp) and writes the output -- no second launch.
+// mbarriers.  Consecutive items of a stream form thread-block clusters; the
+// first CTA of each cluster merges its cluster's partial softmax states
+// (log-sum-exp) from distributed shared memory, and the CTAs of the stream's
+// last cluster to finish merge the cluster partials and write the output --
+// no second launch.
 //
 // Per tile (32 tokens), with the G query heads that share the kv head:
-//   q.K^T  : tensor-core MMA (m16n8k16, f16 in, f32 accumulate).  A = the
-//            packed K codes unpacked in registers to fp16 subnormals c*2^-24
-//            (exact), B = q scaled by 2^kq into fp16 range.  Each 32-channel
-//            K group gets its own 8-column slot so its fp16 scale and bf16
-//            zero factor out of the inner sum (InnerQ grouping):
+//   q.K^T  : integer tensor-core MMA (mma.sync m16n8k32, u8 x s8 -> s32).
+//            A = the packed K codes, masked in registers to one code class
+//            per byte (a byte then reads code * 2^(b j), exact), B = q in
+//            16-bit fixed point per head split into two s8 terms
+//            (q_int = 256 q1 + q2, one column each).  One MMA per 32-channel
+//            K group, so the group's fp16 scale and bf16 zero factor out of
+//            the exact integer sum (InnerQ grouping):
 //              score = sum_grp s_grp * sum_d q_d c_d + z_grp * sum_d q_d.
-//   softmax: online, base 2, running max per head.
-//   P.V    : MMA with A = V codes (channel x token), B = P (fp16), fp32
-//            accumulate; the V scale/zero are per channel for the whole tile:
+//   softmax: online, base 2, running max per head; P in 16-bit fixed point
+//            relative to the running max, split into two u8 terms.
+//   P.V    : MMA (u8 x u8 -> s32) with A = V codes (channel x token), B = P;
+//            the V scale/zero are per channel for the whole tile:
 //              o_d += s_d * sum_t p_t c_td + z_d * sum_t p_t,
 //            where sum_t p_t comes from the same MMA with A = 1.
 #include <cuda_bf16.h>
@@ -670,12 +675,13 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
 // Final log-sum-exp merge of n partial states (o[G][D], m[G], l[G] each,
 // stride PART floats) into the normalised output, for the slice of outputs
 // owned by cluster rank `part`: one output per thread, all of its loads for
-// up to 16 partials in flight at once.
+// up to 24 partials in flight at once (a stream of the long-context cache has
+// 17 cluster partials, so one round trip to L2 covers them).
 template <int D, int G>
 __device__ void merge_outputs(const float* base, int n, float* outp, int part, int tid) {
   using C = Cfg<D, G>;
   constexpr int PER = (G * D + kDecodeCluster - 1) / kDecodeCluster;  // outputs of one CTA
-  constexpr int U = 16;
+  constexpr int U = 24;
   for (int idx = part * PER + tid; idx < (part + 1) * PER && idx < G * D; idx += kDecodeThreads) {
     const int hh = idx / D;
     float M = -INFINITY, O = 0.0f, L = 0.0f;
