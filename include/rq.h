@@ -278,8 +278,10 @@ rq_status rq_decode_read_status(const void* workspace, int* device_status);
  *   race and corrupt each other's results; serialise them.
  * Arguments as rq_decode_attention, minus the workspace.  The device status
  *   word is not readable through the C ABI for this variant.
+ * n_splits = 0 takes the automatic plan, reduced to the most splits whose
+ *   partials fit the array when the plan needs more.
  * Errors: RQ_ERR_INVALID_ARG; RQ_ERR_WORKSPACE when the split partials of the
- *   call (about (n_splits + 1) * streams * (G*D + 2G) * 4 bytes) exceed the
+ *   call (about (n_splits + 2) * streams * (G*D + 2G) * 4 bytes) exceed the
  *   array -- reduce n_splits or decode fewer layers per call; RQ_ERR_CUDA. */
 rq_status rq_decode_attention_noalloc(rq_cache* cache, int layer, const void* q, float* out,
                                       float softmax_scale, int n_splits, cudaStream_t stream);

@@ -674,13 +674,13 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
 
 // Final log-sum-exp merge of n partial states (o[G][D], m[G], l[G] each,
 // stride PART floats) into the normalised output, for the slice of outputs
-// owned by cluster rank `part`: one output per thread, all of its loads for
+// owned by cluster rank `part` (of CL): one output per thread, all of its loads for
 // up to 24 partials in flight at once (a stream of the long-context cache has
 // 17 cluster partials, so one round trip to L2 covers them).
-template <int D, int G>
+template <int D, int G, int CL>
 __device__ void merge_outputs(const float* base, int n, float* outp, int part, int tid) {
   using C = Cfg<D, G>;
-  constexpr int PER = (G * D + kDecodeCluster - 1) / kDecodeCluster;  // outputs of one CTA
+  constexpr int PER = (G * D + CL - 1) / CL;  // outputs of one CTA
   constexpr int U = 24;
   for (int idx = part * PER + tid; idx < (part + 1) * PER && idx < G * D; idx += kDecodeThreads) {
     const int hh = idx / D;
@@ -714,9 +714,10 @@ __device__ void merge_outputs(const float* base, int n, float* outp, int part, i
   }
 }
 
-template <int D, int G>
-__global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS)
-    decode_kernel(DecodeArgs a) {
+// CL = CTAs per thread-block cluster (kDecodeCluster, or 1: no cluster); the
+// cluster shape is given at launch.
+template <int D, int G, int CL>
+__global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_kernel(DecodeArgs a) {
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[NW * kMaxStages];
@@ -797,45 +798,52 @@ __global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecode
       mypart[G * D + G + hh] = L;
     }
   }
-  // Level 1: the kDecodeCluster items of a thread-block cluster (consecutive
-  // items of one stream) are merged by the cluster's first CTA straight from
-  // the others' shared memory.  Every CTA passes both cluster barriers on
-  // every path (no early exit before them).
+  // Level 1: the CL items of a thread-block cluster (consecutive items of one
+  // stream) are merged by the cluster's first CTA straight from the others'
+  // shared memory (CL = 1: the CTA stores its own partial).  Every CTA passes
+  // both cluster barriers on every path (no early exit before them).
   namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int crank = (int)cluster.block_rank();
-  cluster.sync();  // all partials of the cluster are in shared memory
   float* ps = a.partials + (size_t)srel * NI * C::PART;
-  const int ncl = (int)gridDim.x / kDecodeCluster;
-  if (crank == 0) {
-    const float* rp[kDecodeCluster];
+  const int ncl = (int)gridDim.x / CL;
+  int crank = 0;
+  if constexpr (CL > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    crank = (int)cluster.block_rank();
+    cluster.sync();  // all partials of the cluster are in shared memory
+    if (crank == 0) {
+      const float* rp[CL];
 #pragma unroll
-    for (int r = 0; r < kDecodeCluster; ++r) rp[r] = cluster.map_shared_rank(mypart, r);
-    float* cp = ps + (size_t)(item / kDecodeCluster) * C::PART;
-    for (int idx = tid; idx < G * D; idx += blockDim.x) {
-      const int hh = idx / D;
-      float mv[kDecodeCluster];
-      float M = -INFINITY;
+      for (int r = 0; r < CL; ++r) rp[r] = cluster.map_shared_rank(mypart, r);
+      float* cp = ps + (size_t)(item / CL) * C::PART;
+      for (int idx = tid; idx < G * D; idx += blockDim.x) {
+        const int hh = idx / D;
+        float mv[CL];
+        float M = -INFINITY;
 #pragma unroll
-      for (int r = 0; r < kDecodeCluster; ++r) {
-        mv[r] = rp[r][G * D + hh];
-        M = fmaxf(M, mv[r]);
-      }
-      float O = 0.0f, L = 0.0f;
-      if (M != -INFINITY) {
+        for (int r = 0; r < CL; ++r) {
+          mv[r] = rp[r][G * D + hh];
+          M = fmaxf(M, mv[r]);
+        }
+        float O = 0.0f, L = 0.0f;
+        if (M != -INFINITY) {
 #pragma unroll
-        for (int r = 0; r < kDecodeCluster; ++r) {
-          const float f = ex2(mv[r] - M);
-          O = fmaf(rp[r][idx], f, O);
-          L = fmaf(rp[r][G * D + G + hh], f, L);
+          for (int r = 0; r < CL; ++r) {
+            const float f = ex2(mv[r] - M);
+            O = fmaf(rp[r][idx], f, O);
+            L = fmaf(rp[r][G * D + G + hh], f, L);
+          }
+        }
+        cp[idx] = O;
+        if (idx % D == 0) {
+          cp[G * D + hh] = M;
+          cp[G * D + G + hh] = L;
         }
       }
-      cp[idx] = O;
-      if (idx % D == 0) {
-        cp[G * D + hh] = M;
-        cp[G * D + G + hh] = L;
-      }
     }
+  } else {
+    __syncthreads();  // the item partial is complete in shared memory
+    float* cp = ps + (size_t)item * C::PART;
+    for (int idx = tid; idx < C::PART; idx += blockDim.x) cp[idx] = mypart[idx];
   }
   // the first CTA publishes the cluster partial and learns whether its
   // cluster is the stream's last; it tells every CTA of the cluster
@@ -844,59 +852,126 @@ __global__ void __cluster_dims__(kDecodeCluster, 1, 1) __launch_bounds__(kDecode
     __syncthreads();
     if (tid == 0) {
       const int last = atomicAdd(&a.counters[(size_t)srel * kCountersPerStream], 1u) == (unsigned)(ncl - 1);
+      if constexpr (CL > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
 #pragma unroll
-      for (int r = 0; r < kDecodeCluster; ++r) *cluster.map_shared_rank(&is_last, r) = last;
+        for (int r = 0; r < CL; ++r) *cluster.map_shared_rank(&is_last, r) = last;
+      } else {
+        is_last = last;
+      }
     }
   }
-  cluster.sync();  // remote partial reads and the is_last stores are complete
+  if constexpr (CL > 1) {
+    cg::this_cluster().sync();  // remote partial reads and the is_last stores are complete
+  } else {
+    __syncthreads();
+  }
   if (!is_last) return;
   // Level 2: the CTAs of the last cluster merge the cluster partials, each a
   // slice of the outputs
   __threadfence();
   float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  merge_outputs<D, G>(ps, ncl, outp, crank, tid);
+  merge_outputs<D, G, CL>(ps, ncl, outp, crank, tid);
   if (crank == 0 && tid == 0) a.counters[(size_t)srel * kCountersPerStream] = 0u;
 }
 
 // Host-side caches (per device) of the decode kernel's shared-memory
-// attribute and of its resident-cluster capacity: both are fixed for a given
-// (device, D, G, size), and querying them on every call costs more host time
-// than a decode step.
+// attribute and of its resident capacity: both are fixed for a given
+// (device, D, G, cluster, size), and querying them on every call costs more
+// host time than a decode step.
 std::mutex g_attr_mu;
-std::map<std::tuple<int, int, int>, int> g_smem_set;             // (dev, D, G) -> largest size set
-std::map<std::tuple<int, int, int, int>, int> g_resident;        // (dev, D, G, smem) -> CTAs
+std::map<std::tuple<int, int, int, int>, int> g_smem_set;        // (dev, D, G, CL) -> largest size set
+std::map<std::tuple<int, int, int, int, int>, int> g_resident;   // (dev, D, G, CL, smem) -> CTAs
 
-template <int D, int G>
+template <int D, int G, int CL>
 cudaError_t ensure_smem(int smem) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_attr_mu);
-  int& cur = g_smem_set[std::make_tuple(dev, D, G)];
+  int& cur = g_smem_set[std::make_tuple(dev, D, G, CL)];
   if (cur >= smem) return cudaSuccess;
-  e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(decode_kernel<D, G, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) cur = smem;
   return e;
 }
 
-template <int D, int G>
-cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
-  cudaError_t e = ensure_smem<D, G>(smem);
+template <int D, int G, int CL>
+cudaError_t launch_dgc(const DecodeArgs& a, int smem, cudaStream_t st) {
+  cudaError_t e = ensure_smem<D, G, CL>(smem);
   if (e != cudaSuccess) return e;
   const int streams = a.n_layers * a.g.B * a.g.Hkv;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cluster_items(a.n_splits + a.n_win), streams, 1);
+  cfg.gridDim = dim3(cluster_items(a.n_splits + a.n_win, CL), streams, 1);
   cfg.blockDim = dim3(kDecodeThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = RQ_DECODE_PDL;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G>, a);
+  if (CL > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = CL;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G, CL>, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
+  if (a.cluster == 1) return launch_dgc<D, G, 1>(a, smem, st);
+  if (a.cluster == kDecodeCluster) return launch_dgc<D, G, kDecodeCluster>(a, smem, st);
+  return cudaErrorInvalidValue;
+}
+
+// CTAs of the decode kernel that the device holds at once, in whole clusters.
+template <int D, int G, int CL>
+int resident_ctas_dgc(int smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CL;
+  {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    auto it = g_resident.find(std::make_tuple(dev, D, G, CL, smem));
+    if (it != g_resident.end()) return it->second;
+  }
+  if (ensure_smem<D, G, CL>(smem) != cudaSuccess) return CL;
+  int n = 0;
+  if (CL > 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CL * 64, 1, 1);
+    cfg.blockDim = dim3(kDecodeThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<D, G, CL>, &cfg) != cudaSuccess || n < 1) return CL;
+    n *= CL;
+  } else {
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<D, G, CL>, kDecodeThreads, smem) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || per_sm < 1 || sms < 1)
+      return 1;
+    n = per_sm * sms;
+  }
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  g_resident[std::make_tuple(dev, D, G, CL, smem)] = n;
+  return n;
+}
+
+template <int D, int G>
+int resident_ctas_dg(int cluster, int smem) {
+  return cluster == 1 ? resident_ctas_dgc<D, G, 1>(smem) : resident_ctas_dgc<D, G, kDecodeCluster>(smem);
 }
 
 }  // namespace
@@ -913,31 +988,9 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   return (need + 127) / 128 * 128 + scratch;
 }
 
-// CTAs of the decode kernel that the device holds at once, in whole clusters.
-template <int D, int G>
-int resident_ctas_dg(int smem) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return kDecodeCluster;
-  {
-    std::lock_guard<std::mutex> lock(g_attr_mu);
-    auto it = g_resident.find(std::make_tuple(dev, D, G, smem));
-    if (it != g_resident.end()) return it->second;
-  }
-  if (ensure_smem<D, G>(smem) != cudaSuccess) return kDecodeCluster;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kDecodeCluster * 64, 1, 1);
-  cfg.blockDim = dim3(kDecodeThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)smem;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<D, G>, &cfg) != cudaSuccess || n < 1) return kDecodeCluster;
-  std::lock_guard<std::mutex> lock(g_attr_mu);
-  g_resident[std::make_tuple(dev, D, G, smem)] = n * kDecodeCluster;
-  return n * kDecodeCluster;
-}
-
-int decode_resident_ctas(int D, int G, int smem) {
+int decode_resident_ctas(int D, int G, int cluster, int smem) {
 #define RQ_DG(DD, GG) \
-  if (D == DD && G == GG) return resident_ctas_dg<DD, GG>(smem);
+  if (D == DD && G == GG) return resident_ctas_dg<DD, GG>(cluster, smem);
   RQ_DG(128, 1) RQ_DG(128, 2) RQ_DG(128, 4) RQ_DG(128, 8)
   RQ_DG(64, 1) RQ_DG(64, 2) RQ_DG(64, 4) RQ_DG(64, 8)
 #undef RQ_DG

@@ -98,16 +98,29 @@ int max_record(const rq_cache* c, int l0, int nl) {
   return r;
 }
 
-// Tile splits per stream so that all work items of the call (splits plus the
-// window items, padded to whole clusters) fill the resident CTA slots once.
-int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win) {
+// Tile splits per stream and cluster size of a decode call (auto mode).
+// One wave -- every stream's items fit the resident slots once in clusters
+// of kDecodeCluster: the splits fill the slots and the window items share the
+// stream's last cluster.  Several waves: single-CTA items of about
+// kWaveTilesPerItem tiles (more when the slots allow), so that no CTA holds
+// a slot at a cluster barrier while the others of its cluster still work.
+int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win, int* cluster) {
+  *cluster = rq::kDecodeCluster;
   if (n_tiles <= 0) return 0;
-  const long slots = rq::decode_resident_ctas(
-      c->g.D, c->g.G, rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes), stage_bytes, c->g.G, c->g.D));
-  long per = (slots / streams) / rq::kDecodeCluster * rq::kDecodeCluster;
-  long s = per - n_win;
-  if (s < 1) s = 1;
+  const int smem = rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes), stage_bytes, c->g.G, c->g.D);
+  const long slots = rq::decode_resident_ctas(c->g.D, c->g.G, rq::kDecodeCluster, smem);
+  const long per = (slots / streams) / rq::kDecodeCluster * rq::kDecodeCluster;
   const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;  // keep a CTA's pipeline busy
+  long s;
+  if (per >= 2 * rq::kDecodeCluster) {
+    s = per - n_win;
+  } else {
+    *cluster = 1;
+    const long slots1 = rq::decode_resident_ctas(c->g.D, c->g.G, 1, smem);
+    s = (n_tiles + rq::kWaveTilesPerItem - 1) / rq::kWaveTilesPerItem;
+    if (slots1 / streams - n_win > s) s = slots1 / streams - n_win;
+  }
+  if (s < 1) s = 1;
   if (s > max_by_work) s = max_by_work;
   if (s > n_tiles) s = n_tiles;
   if (s > rq::kMaxItems - n_win) s = rq::kMaxItems - n_win;
@@ -126,10 +139,11 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   if (streams > 65535) return RQ_ERR_UNSUPPORTED;
   const int stage_bytes = max_record(c, l0, nl);
   const int n_win = rq::window_items(T, c->g.S, c->g.R);
-  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win) : n_splits;
+  int cluster = rq::kDecodeCluster;  // explicit split counts run in clusters
+  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win, &cluster) : n_splits;
   if (splits > n_tiles) splits = n_tiles;
   if (n_tiles > 0 && splits < 1) splits = 1;
-  if (rq::cluster_items(splits + n_win) > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
+  if (rq::cluster_items(splits + n_win, cluster) > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
   const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
   if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + n_win, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
   a.g = c->g;
@@ -147,6 +161,7 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   a.n_splits = splits;
   a.n_win = n_win;
   a.n_streams = streams;
+  a.cluster = cluster;
   a.stages = rq::decode_stages(stage_bytes);
   a.stage_bytes = stage_bytes;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -302,8 +317,9 @@ rq_status rq_decode_workspace_bytes(const rq_cache* c, int n_splits, size_t* byt
   int s = n_splits;
   const int rec = max_record(c, 0, c->g.L);
   const int nw = (c->g.S + c->g.R + 2 * rq::kTile - 1) / rq::kTile;  // most window items any length can need
-  const int a1 = auto_splits(c, streams_layer, max_tiles, rec, 1);
-  const int a2 = auto_splits(c, streams_layer * c->g.L, max_tiles, rec, 1);
+  int cl = 0;
+  const int a1 = auto_splits(c, streams_layer, max_tiles, rec, 1, &cl);
+  const int a2 = auto_splits(c, streams_layer * c->g.L, max_tiles, rec, 1, &cl);
   if (s < a1) s = a1;
   if (s < a2) s = a2;
   if (s > rq::kMaxItems - nw) s = rq::kMaxItems - nw;
@@ -387,13 +403,24 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
   if (rq::noalloc_scratch(&scratch) != cudaSuccess) return RQ_ERR_CUDA;
   rq::DecodeArgs a;
   int smem = 0;
+  const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
   rq_status st = fill_decode(c, l0, nl, c->length[l0], q, out, softmax_scale, n_splits, scratch,
                              rq::kNoAllocScratchBytes, a, smem);
+  if (st == RQ_ERR_WORKSPACE && n_splits == 0) {
+    // the automatic plan needs more partials than the array holds: take the
+    // most splits whose partials fit
+    const int64_t streams = (int64_t)nl * c->g.B * c->g.Hkv;
+    const int64_t items = (int64_t)(rq::kNoAllocScratchBytes - rq::ws_partial_offset(all_streams)) /
+                          (streams * (int64_t)(c->g.G * c->g.D + 2 * c->g.G) * 4);
+    const int64_t s = items - rq::window_items(c->length[l0], c->g.S, c->g.R);
+    if (s >= 1)
+      st = fill_decode(c, l0, nl, c->length[l0], q, out, softmax_scale, (int)s, scratch, rq::kNoAllocScratchBytes,
+                       a, smem);
+  }
   if (st == RQ_ERR_WORKSPACE) return RQ_ERR_WORKSPACE;  // more split partials than the fixed array holds
   if (st != RQ_OK) return st;
   // status word and completion counters must start at zero; the array keeps
   // whatever the previous call (on any stream) left in it
-  const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
   if (cudaMemsetAsync(scratch, 0, rq::ws_partial_offset(all_streams), stream) != cudaSuccess) return RQ_ERR_CUDA;
   return cuda_status(rq::launch_decode(a, smem, stream));
 }

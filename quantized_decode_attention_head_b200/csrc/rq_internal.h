@@ -86,6 +86,7 @@ struct DecodeArgs {
   int n_splits;           // tile splits: items [0, n_splits)
   int n_win;              // bf16 window items (32 tokens each): items [n_splits, n_splits + n_win)
   int n_streams;          // streams of this call
+  int cluster;            // CTAs per thread-block cluster: kDecodeCluster or 1
   int stages;             // per-warp ring depth (2..8)
   int stage_bytes;        // bytes per stage (max record size in the call)
   float* partials;        // [streams][n_splits+1][G*D + 2G]
@@ -96,11 +97,14 @@ struct DecodeArgs {
 };
 
 // Split-K combine.  The work items of a stream (tile splits, then window
-// chunks) form thread-block clusters of kDecodeCluster consecutive items
-// (the grid is padded with empty items to whole clusters); a cluster merges
-// its items through distributed shared memory, and the CTAs of the last
-// cluster of the stream to finish merge the cluster partials, each a slice
-// of the outputs.  Per stream counter [0] counts finished clusters.
+// chunks) form thread-block clusters of `cluster` consecutive items (the grid
+// is padded with empty items to whole clusters); a cluster merges its items
+// through distributed shared memory, and the CTAs of the last cluster of the
+// stream to finish merge the cluster partials, each a slice of the outputs.
+// Per stream counter [0] counts finished clusters.  Calls whose items fill
+// the device once run in clusters of kDecodeCluster; calls that need several
+// waves of CTAs run single-CTA items (cluster 1), so that no CTA holds a slot
+// at a cluster barrier while the others of its cluster still work.
 #ifndef RQ_DECODE_CLUSTER
 #define RQ_DECODE_CLUSTER 4
 #endif
@@ -111,8 +115,10 @@ constexpr int kDecodeCluster = RQ_DECODE_CLUSTER;
 #endif
 constexpr int kCountersPerStream = 64;
 constexpr int kMaxItems = 496;
-__host__ __device__ inline int cluster_items(int items) {
-  return (items + kDecodeCluster - 1) / kDecodeCluster * kDecodeCluster;
+// tiles per work item aimed at when a call runs in several waves
+constexpr int kWaveTilesPerItem = 128;
+__host__ __device__ inline int cluster_items(int items, int cluster) {
+  return (items + cluster - 1) / cluster * cluster;
 }
 
 // Workspace layout (bytes): [status int32, pad to 256][kCountersPerStream u32
@@ -148,7 +154,9 @@ cudaError_t launch_measure_distortion(const uint16_t* x, int n_heads, int n_toke
                                       const int* bits, int n_bits, double* mse, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int smem_bytes, cudaStream_t s);
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D);
-int decode_resident_ctas(int D, int G, int smem_bytes);  // CTAs resident on the device, whole clusters
+// CTAs of the decode kernel resident on the device at once, in whole clusters
+// of `cluster` CTAs
+int decode_resident_ctas(int D, int G, int cluster, int smem_bytes);
 
 // Size of the device array behind rq_decode_attention_noalloc (bytes).
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;

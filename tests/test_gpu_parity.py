@@ -80,6 +80,37 @@ def test_decode_all_layers_call():
         assert_close(got[l, b], e, f"layer {l} b {b}")
 
 
+def test_many_streams_single_cta_items():
+    """A call with more streams than the device holds clusters for in one
+    wave: the automatic plan runs single-CTA work items (no clusters) in
+    several waves.  Every stream's output against the oracle, for the
+    all-layers decode, a fused decode step and an explicit split count (which
+    keeps clusters), before and after a step."""
+    # 80 streams of 40 tiles: more than the 68 that one wave of clusters holds
+    # on a 148-SM device, few enough that the plan takes several splits each
+    wl = _small(n_layers=2, batch=10, context=4 + 32 * 40 + 32 + 11)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    cache, st, (k, v, f) = _build(wl, kb, vb)
+    q, kn, vn = workloads.step_inputs(wl, 2, f, "cuda")
+    which = [(l, b) for l in range(wl.n_layers) for b in range(wl.batch)]
+    ws = cache.make_workspace()
+    exp = oracle_decode(wl, st, to_f32(q[0]).astype(np.float64), which)
+    for splits in [0, 3]:
+        got = cache.rq_decode_attention(-1, q[0].contiguous(), n_splits=splits, workspace=ws).cpu().numpy()
+        for (l, b), e in exp.items():
+            assert_close(got[l, b], e, f"layer {l} b {b} splits {splits}")
+    got = cache.rq_decode_step(-1, q[1].contiguous(), kn[1].contiguous(), vn[1].contiguous(),
+                               workspace=ws).cpu().numpy()
+    for (l, b, h), s in st.items():
+        s.append(to_f32(kn[1, l, b, h]), to_f32(vn[1, l, b, h]))
+    exp = oracle_decode(wl, st, to_f32(q[1]).astype(np.float64), which)
+    for (l, b), e in exp.items():
+        assert_close(got[l, b], e, f"step: layer {l} b {b}")
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+
+
 @pytest.mark.parametrize("T", [0, 1, 3, 4, 20, 36, 67, 68, 69, 100])
 def test_short_caches(T):
     # T < S, T < S + R (no tiles), exactly one tile, ragged windows
