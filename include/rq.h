@@ -241,14 +241,21 @@ rq_status rq_decode_attention(rq_cache* cache, int layer, const void* q, float* 
  *   followed by rq_decode_attention(layer, q, ...) over the cache that now
  *   includes the new token, with the same arguments, layouts, results and
  *   errors as those two calls (InnerQ Algorithm 1, decode phase: the current
- *   token's key and value join the high-precision recent window).  When the
- *   append does not complete a tile -- 31 steps in 32 -- both happen in one
- *   kernel launch: the window work item that owns the newest position reads
- *   the token from k_new / v_new and writes it into the cache.  When it does,
- *   the tile is quantized first and the decode follows (two launches).  On an
- *   error nothing is launched and the length is unchanged; otherwise the
- *   length grows by one.  The pages have no separate counterpart: it is the
- *   two operations above, fused. */
+ *   token's key and value join the high-precision recent window).  Both
+ *   happen in one kernel launch: the window work item that owns the newest
+ *   position reads the token from k_new / v_new and writes it into the
+ *   cache.  When the NEXT append will complete a tile (its 32 tokens are the
+ *   oldest of the recent window, all present already), one more work item of
+ *   this launch quantizes and packs that tile into its slot, which nothing
+ *   reads until then; the next rq_decode_step on the same layers then only
+ *   advances the length past it.  A step whose append completes a tile that
+ *   was not packed ahead -- the first step after rq_quantize_kv or
+ *   rq_append_token, or any step when n_recent < 2 -- quantizes the tile
+ *   first and decodes after (two launches).  Results are those of the two
+ *   calls in every case.  Workspace: rq_decode_workspace_bytes includes the
+ *   extra item.  On an error nothing is launched and the length is
+ *   unchanged; otherwise the length grows by one.  The pages have no
+ *   separate counterpart: it is the two operations above, fused. */
 rq_status rq_decode_step(rq_cache* cache, int layer, const void* q, const void* k_new, const void* v_new,
                          float* out, float softmax_scale, int n_splits, void* workspace, size_t ws_bytes,
                          cudaStream_t stream);

@@ -237,7 +237,9 @@ class QuantizedKVCache:
     def rq_decode_step(self, layer, q, k_new, v_new, out=None, softmax_scale=0.0, n_splits=0, workspace=None,
                        stream=None):
         """rq_append_token(layer, k_new, v_new) then rq_decode_attention(layer, q),
-        in one launch when the append completes no tile."""
+        in one launch (the step before a tile flush also packs that tile
+        ahead); two launches only when the completed tile was not packed
+        ahead by the previous step."""
         import torch
 
         nl = self.n_layers if layer == -1 else 1

@@ -38,6 +38,7 @@
 
 #include "rq_device.cuh"
 #include "rq_internal.h"
+#include "rq_pack.cuh"
 
 namespace rq {
 namespace {
@@ -401,10 +402,12 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, const float* nr
   // launch may start (prefill, tile flush), never by the decode launch this
   // one may overlap, so the first records can be fetched before waiting on
   // it; the query, the window and the workspace are read after the wait.
+  const uint64_t policy = l2_evict_first_policy();  // tile records are read once per launch
   if (lane == 0) {
     for (int j = 0; j < stages && j < n_w; ++j) {
       mbar_arrive_expect_tx(&bars[j], (uint32_t)rec);
-      bulk_g2s(ring + (size_t)j * stage_bytes, src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec, &bars[j]);
+      bulk_g2s_hint(ring + (size_t)j * stage_bytes, src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec, &bars[j],
+                    policy);
     }
   }
   griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
@@ -430,7 +433,7 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, const float* nr
     if (lane == 0 && j + stages < n_w) {
       fence_proxy_async_smem();  // generic-proxy reads of the slot precede the async refill
       mbar_arrive_expect_tx(&bars[slot], (uint32_t)rec);
-      bulk_g2s(cur, nsrc, (uint32_t)rec, &bars[slot]);
+      bulk_g2s_hint(cur, nsrc, (uint32_t)rec, &bars[slot], policy);
     }
     nsrc += (int64_t)NW * rec;
     cur += stage_bytes;
@@ -672,6 +675,46 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
   }
 }
 
+// Pack-ahead item (a fused step whose next append completes a tile): the 32
+// oldest ring tokens -- exactly the tile that append will flush -- are
+// quantized and packed into tile slot a.pack_tile, which no item of this
+// launch reads, so the next step needs no separate flush launch.  The rows
+// it reads are not the one this launch's window item writes (n_recent >= 2).
+// Warp 0 packs K, warp 1 V.  Leaves empty partial states in the warp slots.
+template <int D, int G>
+__device__ void pack_item(const DecodeArgs& a, const HeadDesc& hd, int b, uint8_t* area, float* merge, int tid) {
+  using C = Cfg<D, G>;
+  const int warp = tid >> 5, lane = tid & 31;
+  TileSmem<D>& sm = *reinterpret_cast<TileSmem<D>*>(area);
+  uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
+  const int S = a.g.S, ring = a.g.R + kTile;
+  griddep_wait();
+  if (warp == 0) stage_kinv<D>(sm.kinv, stream_norm(a.buf, hd, a.g, b), lane);
+  constexpr int kChunks = D / 8;
+  for (int j = tid; j < kTile * kChunks; j += blockDim.x) {
+    const int t = j / kChunks, c = j % kChunks;
+    const int slot = (a.pack_pos + t - S) % ring;
+    const uint4* krow = reinterpret_cast<const uint4*>(win + ((size_t)2 * S + slot) * D * 2);
+    const uint4* vrow = reinterpret_cast<const uint4*>(win + ((size_t)2 * S + ring + slot) * D * 2);
+    *reinterpret_cast<uint4*>(&sm.k.x[t][c * 4]) = __ldg(krow + c);
+    *reinterpret_cast<uint4*>(&sm.v.x[t][c * 4]) = __ldg(vrow + c);
+  }
+  __syncthreads();
+  uint8_t* rec = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)a.pack_tile * hd.rec_bytes;
+  if (warp == 0) {
+    pack_k_dispatch<D, true>(sm.k, sm.kinv, hd.k_bits, rec, lane);
+  } else if (warp == 1) {
+    pack_v_dispatch<D>(sm.v, hd.v_bits, rec + blob_bytes(hd.k_bits, D) + 4 * D, lane);
+  }
+  __syncthreads();  // the staged tile is dead; its memory becomes the warp slots
+  float* slot = merge + warp * C::PART;
+  for (int i = lane; i < G * D; i += 32) slot[i] = 0.0f;
+  if (lane < G) {
+    slot[G * D + lane] = -INFINITY;
+    slot[G * D + G + lane] = 0.0f;
+  }
+}
+
 // Final log-sum-exp merge of n partial states (o[G][D], m[G], l[G] each,
 // stride PART floats) into the normalised output, for the slice of outputs
 // owned by cluster rank `part` (of CL): one output per thread, all of its loads for
@@ -726,7 +769,7 @@ __global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_k
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int srel = blockIdx.y, item = blockIdx.x;
-  const int NI = a.n_splits + a.n_win;  // work items of this stream
+  const int NI = a.n_splits + a.n_win + a.n_pack;  // work items of this stream
   const int h = srel % a.g.Hkv, b = (srel / a.g.Hkv) % a.g.B, lrel = srel / (a.g.Hkv * a.g.B);
   const int l = a.layer0 + lrel;
   const HeadDesc hd = a.desc[l * a.g.Hkv + h];
@@ -761,6 +804,8 @@ __global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_k
                              area + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
                              bars + warp * kMaxStages, reinterpret_cast<float*>(smem) + warp * C::SCRATCH, src, rec,
                              t1 - t0, warp, lane, &abort_flag, a.status);
+  } else if (a.n_pack && item == a.n_splits + a.n_win) {
+    pack_item<D, G>(a, hd, b, area, merge, tid);
   } else {
     griddep_wait();  // the window rows and the query may come from the previous kernel
     // 32-token chunks of the bf16 sink + recent window
@@ -902,7 +947,7 @@ cudaError_t launch_dgc(const DecodeArgs& a, int smem, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int streams = a.n_layers * a.g.B * a.g.Hkv;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cluster_items(a.n_splits + a.n_win, CL), streams, 1);
+  cfg.gridDim = dim3(cluster_items(a.n_splits + a.n_win + a.n_pack, CL), streams, 1);
   cfg.blockDim = dim3(kDecodeThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = st;
@@ -983,6 +1028,9 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   if (merge < (NW + 1) * part * 4) merge = (NW + 1) * part * 4;  // warp slots + the item partial
   const int ring = NW * stages * stage_bytes;
   int need = ring > merge ? ring : merge;
+  // a pack-ahead item stages one K and one V tile
+  const int pack = D == 128 ? (int)sizeof(TileSmem<128>) : (int)sizeof(TileSmem<64>);
+  if (need < pack) need = pack;
   // per-warp scale scratch of the tile path (Cfg<D, G>::SCRATCH floats)
   const int scratch = NW * 8 * ((D / 32) * 8 + 4 + (D / 8) * 2 + 4) * 4;
   return (need + 127) / 128 * 128 + scratch;

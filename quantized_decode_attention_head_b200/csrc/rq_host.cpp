@@ -20,6 +20,9 @@ struct rq_cache {
   uint8_t* buf;
   size_t bytes;
   std::vector<int> length;  // tokens per layer
+  // per layer: the length at which a fused step packed the tile that the
+  // next append completes (-1: none), see rq_decode_step
+  std::vector<int> packed_ahead;
   int sm_count;
   int k_norm;               // per-channel K normalization set by the prefill
 };
@@ -132,7 +135,8 @@ rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_
 // Decode arguments for layers [l0, l0 + nl) of a cache holding T tokens, with
 // the workspace checked and partitioned; the fused-append pointers are null.
 rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, float* out, float softmax_scale,
-                      int n_splits, void* workspace, size_t ws_bytes, rq::DecodeArgs& a, int& smem) {
+                      int n_splits, void* workspace, size_t ws_bytes, rq::DecodeArgs& a, int& smem,
+                      int n_pack = 0) {
   const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
   const int n_tiles = Tq / rq::kTile;
   const int streams = nl * c->g.B * c->g.Hkv;
@@ -140,12 +144,14 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   const int stage_bytes = max_record(c, l0, nl);
   const int n_win = rq::window_items(T, c->g.S, c->g.R);
   int cluster = rq::kDecodeCluster;  // explicit split counts run in clusters
-  int splits = n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win, &cluster) : n_splits;
+  int splits =
+      n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win + n_pack, &cluster) : n_splits;
   if (splits > n_tiles) splits = n_tiles;
   if (n_tiles > 0 && splits < 1) splits = 1;
-  if (rq::cluster_items(splits + n_win, cluster) > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
+  const int items = splits + n_win + n_pack;
+  if (rq::cluster_items(items, cluster) > rq::kMaxItems) return RQ_ERR_UNSUPPORTED;
   const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
-  if (ws_bytes < rq::ws_total_bytes(all_streams, streams, splits + n_win, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
+  if (ws_bytes < rq::ws_total_bytes(all_streams, streams, items, c->g.G, c->g.D)) return RQ_ERR_WORKSPACE;
   a.g = c->g;
   a.buf = c->buf;
   a.desc = reinterpret_cast<const HeadDesc*>(c->buf);
@@ -160,6 +166,9 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   a.n_tiles = n_tiles;
   a.n_splits = splits;
   a.n_win = n_win;
+  a.n_pack = n_pack;
+  a.pack_pos = 0;
+  a.pack_tile = 0;
   a.n_streams = streams;
   a.cluster = cluster;
   a.stages = rq::decode_stages(stage_bytes);
@@ -170,7 +179,7 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   a.partials = reinterpret_cast<float*>(ws + rq::ws_partial_offset(all_streams));
   a.k_new = nullptr;
   a.v_new = nullptr;
-  smem = rq::decode_smem_bytes(splits + n_win, a.stages, stage_bytes, c->g.G, c->g.D);
+  smem = rq::decode_smem_bytes(items, a.stages, stage_bytes, c->g.G, c->g.D);
   if (smem > 227 * 1024) return RQ_ERR_UNSUPPORTED;
   return RQ_OK;
 }
@@ -225,6 +234,7 @@ rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes,
   c->buf = static_cast<uint8_t*>(dev_buf);
   c->bytes = bytes;
   c->length.assign(c->g.L, 0);
+  c->packed_ahead.assign(c->g.L, -1);
   int dev = 0;
   c->sm_count = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) {
@@ -280,7 +290,10 @@ rq_status rq_quantize_kv(rq_cache* c, const void* k, const void* v, int n_tokens
     const rq_status st = cuda_status(rq::launch_quantize(a, stream));
     if (st != RQ_OK) return st;
   }
-  for (int l = 0; l < c->g.L; ++l) c->length[l] = n_tokens;
+  for (int l = 0; l < c->g.L; ++l) {
+    c->length[l] = n_tokens;
+    c->packed_ahead[l] = -1;
+  }
   return RQ_OK;
 }
 
@@ -324,7 +337,7 @@ rq_status rq_decode_workspace_bytes(const rq_cache* c, int n_splits, size_t* byt
   if (s < a2) s = a2;
   if (s > rq::kMaxItems - nw) s = rq::kMaxItems - nw;
   const int64_t all = (int64_t)streams_layer * c->g.L;
-  *bytes = rq::ws_total_bytes(all, all, s + nw, c->g.G, c->g.D);
+  *bytes = rq::ws_total_bytes(all, all, s + nw + 1, c->g.G, c->g.D);  // + a pack-ahead item
   return RQ_OK;
 }
 
@@ -358,21 +371,37 @@ rq_status rq_decode_step(rq_cache* c, int layer, const void* q, const void* k_ne
   const int T_old = c->length[l0];
   if (T_old + 1 > c->max_tokens) return RQ_ERR_CAPACITY;
   const int S = c->g.S, R = c->g.R;
-  if (rq::quantized_tokens(T_old + 1, S, R) != rq::quantized_tokens(T_old, S, R)) {
-    // the append completes a tile: quantize it first, then decode (two launches)
+  bool packed = true;  // the previous fused step packed the tile this append completes
+  for (int l = l0; l < l0 + nl; ++l) packed = packed && c->packed_ahead[l] == T_old;
+  if (rq::quantized_tokens(T_old + 1, S, R) != rq::quantized_tokens(T_old, S, R) && !packed) {
+    // the append completes a tile that is not packed yet: quantize it first,
+    // then decode (two launches)
     rq_status st = rq_append_token(c, layer, k_new, v_new, stream);
     if (st != RQ_OK) return st;
     return rq_decode_attention(c, layer, q, out, softmax_scale, n_splits, workspace, ws_bytes, stream);
   }
+  // One launch: append (the window item writes the new token) + decode, and,
+  // when the next append will complete a tile, that tile is packed ahead by
+  // one more work item.  Its 32 tokens are the oldest of the ring, all
+  // present now; with n_recent >= 2 the token appended here is not among them.
+  const int T = T_old + 1;
+  const int Tq = rq::quantized_tokens(T, S, R);
+  const int n_pack =
+      (R >= 2 && T + 1 <= c->max_tokens && rq::quantized_tokens(T + 1, S, R) != Tq) ? 1 : 0;
   rq::DecodeArgs a;
   int smem = 0;
-  rq_status st = fill_decode(c, l0, nl, T_old + 1, q, out, softmax_scale, n_splits, workspace, ws_bytes, a, smem);
+  rq_status st = fill_decode(c, l0, nl, T, q, out, softmax_scale, n_splits, workspace, ws_bytes, a, smem, n_pack);
   if (st != RQ_OK) return st;
   a.k_new = static_cast<const uint16_t*>(k_new);
   a.v_new = static_cast<const uint16_t*>(v_new);
+  a.pack_pos = S + Tq;
+  a.pack_tile = Tq / rq::kTile;
   st = cuda_status(rq::launch_decode(a, smem, stream));
   if (st != RQ_OK) return st;
-  for (int l = l0; l < l0 + nl; ++l) c->length[l] = T_old + 1;
+  for (int l = l0; l < l0 + nl; ++l) {
+    c->length[l] = T;
+    c->packed_ahead[l] = n_pack ? T : -1;
+  }
   return RQ_OK;
 }
 

@@ -85,6 +85,9 @@ struct DecodeArgs {
   int T, Tq, n_tiles;
   int n_splits;           // tile splits: items [0, n_splits)
   int n_win;              // bf16 window items (32 tokens each): items [n_splits, n_splits + n_win)
+  int n_pack;             // 1: item n_splits + n_win packs the tile the next append completes
+  int pack_pos;           // its first token (absolute position) and its tile slot
+  int pack_tile;
   int n_streams;          // streams of this call
   int cluster;            // CTAs per thread-block cluster: kDecodeCluster or 1
   int stages;             // per-warp ring depth (2..8)

@@ -1,210 +1,45 @@
 // Quantize-and-pack kernels: prefill of whole tiles, window copy, and the
-// decode-time append with tile flush.
-//
-// InnerQ grouping (arXiv 2602.23200, abstract / "Core claim"): K groups run
-// along head_dim per token (32 channels), V groups along tokens per channel
-// (the 32 tokens of a tile).  Asymmetric min/max quantization with an fp16
-// scale and a bf16 zero; bit widths 2, 3, 4, 8 per (layer, kv-head).
-//
-// Every arithmetic step of the rounding rule is an IEEE fp32 operation with
-// round-to-nearest-even (__fsub_rn, __fdiv_rn, __frcp_rn, __fmul_rn,
-// __float2half_rn, __float2int_rn), so codes and scales are reproducible
-// bit for bit on any IEEE machine.
+// decode-time append with tile flush (the tile rule itself is in
+// rq_pack.cuh).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "rq_device.cuh"
 #include "rq_internal.h"
+#include "rq_pack.cuh"
 
 namespace rq {
 namespace {
 
 constexpr int kQuantWarps = 4;
 
+// Prefill: one warp stages and packs K, then V, through one half tile, so
+// that five 4-warp CTAs fit an SM.
 template <int D>
-struct TileSmem {
-  static constexpr int kStride = D / 2 + 4;  // words per staged row (16-byte aligned)
-  uint32_t k[kTile][kStride];                // bf16 pairs
-  uint32_t v[kTile][kStride];
-  float kr[kTile][D / 32];  // 1 / scale per (token, group)
-  float kz[kTile][D / 32];  // zero per (token, group)
-  float vr[D];
-  float vz[D];
-  float kinv[D];  // 1 / n per channel (K normalization; powers of two)
+struct PrefillSmem {
+  HalfTile<D> t;
+  float kinv[D];
 };
 
-// Stream's K normalization factors n[D] (fp32), stored after its window rows.
-__device__ __forceinline__ float* stream_norm(uint8_t* buf, const HeadDesc& hd, const Geom& g, int b) {
-  return reinterpret_cast<float*>(buf + hd.win_base + (int64_t)b * g.win_bytes + window_rows_bytes(g.S, g.R, g.D));
-}
-
-// 1 / n of the stream into shared memory (one warp).
+// Stage 32 consecutive rows of D bf16 (row t at base + t * D) into the smem
+// tile (whole warp).
 template <int D>
-__device__ __forceinline__ void stage_kinv(TileSmem<D>& sm, const float* nrm, int lane) {
-  for (int d = lane; d < D; d += 32) sm.kinv[d] = 1.0f / nrm[d];
-}
-
-__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// Scale/zero of one group from its min and max; returns the meta word.
-template <int B>
-__device__ __forceinline__ uint32_t group_params(float mn, float mx, float& r) {
-  float s32 = __fdiv_rn(__fsub_rn(mx, mn), (float)((1 << B) - 1));
-  s32 = fminf(s32, 65504.0f);
-  const __half h = __float2half_rn(s32);
-  const float s = __half2float(h);
-  r = s > 0.0f ? __frcp_rn(s) : 0.0f;
-  return (uint32_t)__half_as_ushort(h) | ((__float_as_uint(mn) >> 16) << 16);
-}
-
-template <int B>
-__device__ __forceinline__ uint32_t code_of(float x, float z, float r) {
-  int c = __float2int_rn(__fmul_rn(__fsub_rn(x, z), r));
-  c = c < 0 ? 0 : c;
-  c = c > (1 << B) - 1 ? (1 << B) - 1 : c;
-  return (uint32_t)c;
-}
-
-// Stage 32 rows of D bf16 (row t at rows[t]) into the smem tile (whole warp).
-template <int D>
-__device__ __forceinline__ void stage_rows(uint32_t (*dst)[TileSmem<D>::kStride], const uint16_t* const* rows,
-                                           int lane) {
+__device__ __forceinline__ void stage_rows_contig(uint32_t (*dst)[HalfTile<D>::kStride], const uint16_t* base,
+                                                  int lane) {
   constexpr int kChunks = D / 8;  // 16-byte chunks per row
-#pragma unroll 4
-  for (int j = lane; j < kTile * kChunks; j += 32) {
-    const int t = j / kChunks, c = j % kChunks;
-    const uint4 x = __ldg(reinterpret_cast<const uint4*>(rows[t]) + c);
-    *reinterpret_cast<uint4*>(&dst[t][c * 4]) = x;
-  }
-}
-
-template <int D, int KB>
-__device__ void pack_k(TileSmem<D>& sm, uint8_t* rec, int lane) {
-  constexpr int NG = D / 32;
-  constexpr int W = words_per_lane(KB, D);
-  // statistics: lane = token, rotated word order spreads smem banks
-  {
-    const int t = lane;
-#pragma unroll
-    for (int grp = 0; grp < NG; ++grp) {
-      float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int cw = grp * 16 + ((c + (t >> 3)) & 15);
-        const uint32_t w = sm.k[t][cw];
-        const float x0 = lo_bf16(w) * sm.kinv[2 * cw], x1 = hi_bf16(w) * sm.kinv[2 * cw + 1];
-        mn = fminf(mn, fminf(x0, x1));
-        mx = fmaxf(mx, fmaxf(x0, x1));
-      }
-      float r;
-      const uint32_t meta = group_params<KB>(mn, mx, r);
-      sm.kr[t][grp] = r;
-      sm.kz[t][grp] = mn;
-      const int i = (t & 7) * 4 + (t >> 4) * 2 + ((t >> 3) & 1);
-      reinterpret_cast<uint32_t*>(rec + blob_bytes(KB, D))[grp * 32 + i] = meta;
-    }
-  }
-  __syncwarp();
-  const int gid = lane >> 2, tig = lane & 3;
-  uint32_t words[W];
-#pragma unroll
-  for (int w = 0; w < W; ++w) words[w] = 0;
-  // register (rho, kh), byte e: token gid + 8i, channel 32g + 16kh + 4tig + e
-#pragma unroll
-  for (int rho = 0; rho < D / 8; ++rho)
-#pragma unroll
-    for (int kh = 0; kh < 2; ++kh)
-#pragma unroll
-      for (int e = 0; e < 4; e += 2) {
-        const int i = rho / NG, g = rho % NG;
-        const int t = gid + 8 * i, d0 = 32 * g + 16 * kh + 4 * tig + e;
-        const uint32_t x = sm.k[t][d0 / 2];
-        const float rr = sm.kr[t][g], z = sm.kz[t][g];
-        put_code<KB, W>(words, rho, kh, e, code_of<KB>(lo_bf16(x) * sm.kinv[d0], z, rr));
-        put_code<KB, W>(words, rho, kh, e + 1, code_of<KB>(hi_bf16(x) * sm.kinv[d0 + 1], z, rr));
-      }
-#pragma unroll
-  for (int c = 0; c < W / 4; ++c)
-    *reinterpret_cast<uint4*>(rec + word_offset(W, lane, 4 * c)) =
-        make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
-#pragma unroll
-  for (int w = 4 * (W / 4); w < W; ++w) *reinterpret_cast<uint32_t*>(rec + word_offset(W, lane, w)) = words[w];
-}
-
-template <int D, int VB>
-__device__ void pack_v(TileSmem<D>& sm, uint8_t* vrec, int lane) {
-  constexpr int W = words_per_lane(VB, D);
-  // statistics: each lane owns channel pairs (2w, 2w+1)
-#pragma unroll
-  for (int w = lane; w < D / 2; w += 32) {
-    float mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY;
+  const uint4* src = reinterpret_cast<const uint4*>(base);
 #pragma unroll 8
-    for (int t = 0; t < kTile; ++t) {
-      const uint32_t x = sm.v[t][w];
-      mn0 = fminf(mn0, lo_bf16(x));
-      mx0 = fmaxf(mx0, lo_bf16(x));
-      mn1 = fminf(mn1, hi_bf16(x));
-      mx1 = fmaxf(mx1, hi_bf16(x));
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int d = 2 * w + h;
-      float r;
-      const uint32_t meta = group_params<VB>(h ? mn1 : mn0, h ? mx1 : mx0, r);
-      sm.vr[d] = r;
-      sm.vz[d] = h ? mn1 : mn0;
-      const int i = (d & 7) * (D / 8) + (d >> 4) * 2 + ((d >> 3) & 1);
-      reinterpret_cast<uint32_t*>(vrec + blob_bytes(VB, D))[i] = meta;
-    }
-  }
-  __syncwarp();
-  const int gid = lane >> 2, tig = lane & 3;
-  uint32_t words[W];
-#pragma unroll
-  for (int w = 0; w < W; ++w) words[w] = 0;
-  // register (rho, kh), byte e: channel 16mb + 8rh + gid (rho = 2mb + rh),
-  // token 4kh + tig + 8e
-#pragma unroll
-  for (int rho = 0; rho < D / 8; ++rho) {
-    const int d = 16 * (rho / 2) + 8 * (rho % 2) + gid;
-    const float rr = sm.vr[d], z = sm.vz[d];
-#pragma unroll
-    for (int kh = 0; kh < 2; ++kh)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t x = sm.v[4 * kh + tig + 8 * e][d >> 1];
-        put_code<VB, W>(words, rho, kh, e, code_of<VB>((d & 1) ? hi_bf16(x) : lo_bf16(x), z, rr));
-      }
-  }
-#pragma unroll
-  for (int c = 0; c < W / 4; ++c)
-    *reinterpret_cast<uint4*>(vrec + word_offset(W, lane, 4 * c)) =
-        make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
-#pragma unroll
-  for (int w = 4 * (W / 4); w < W; ++w) *reinterpret_cast<uint32_t*>(vrec + word_offset(W, lane, w)) = words[w];
-}
-
-template <int D>
-__device__ void quantize_staged_tile(TileSmem<D>& sm, int kb, int vb, uint8_t* rec, int lane) {
-  switch (kb) {
-    case 2: pack_k<D, 2>(sm, rec, lane); break;
-    case 3: pack_k<D, 3>(sm, rec, lane); break;
-    case 4: pack_k<D, 4>(sm, rec, lane); break;
-    default: pack_k<D, 8>(sm, rec, lane); break;
-  }
-  uint8_t* vrec = rec + blob_bytes(kb, D) + 4 * D;
-  switch (vb) {
-    case 2: pack_v<D, 2>(sm, vrec, lane); break;
-    case 3: pack_v<D, 3>(sm, vrec, lane); break;
-    case 4: pack_v<D, 4>(sm, vrec, lane); break;
-    default: pack_v<D, 8>(sm, vrec, lane); break;
+  for (int j = lane; j < kTile * kChunks; j += 32) {
+    const uint4 x = __ldg(src + j);
+    *reinterpret_cast<uint4*>(&dst[j / kChunks][(j % kChunks) * 4]) = x;
   }
 }
 
-// grid (ceil(tiles / 4), L*B*Hkv); one warp per tile.
-template <int D>
-__global__ void __launch_bounds__(kQuantWarps * 32) quantize_tiles_kernel(QuantizeArgs a) {
+// grid (ceil(tiles / 4), L*B*Hkv); one warp per tile: K rows staged and
+// packed, then V rows through the same buffer.  KN: the cache normalizes K.
+constexpr int kQuantMinBlocks = 5;
+template <int D, bool KN>
+__global__ void __launch_bounds__(kQuantWarps * 32, kQuantMinBlocks) quantize_tiles_kernel(QuantizeArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = a.Tq / kTile;
@@ -213,24 +48,23 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quantize_tiles_kernel(Quanti
   const int s = blockIdx.y;
   const int h = s % a.g.Hkv, b = (s / a.g.Hkv) % a.g.B, l = s / (a.g.Hkv * a.g.B);
   const HeadDesc hd = a.desc[l * a.g.Hkv + h];
-  TileSmem<D>& sm = reinterpret_cast<TileSmem<D>*>(smem_raw)[warp];
+  PrefillSmem<D>& sm = reinterpret_cast<PrefillSmem<D>*>(smem_raw)[warp];
   const size_t row0 = ((size_t)s * a.T + a.g.S + (size_t)tile * kTile) * D;
-  const uint16_t* krows[kTile];
-  const uint16_t* vrows[kTile];
-#pragma unroll
-  for (int t = 0; t < kTile; ++t) {
-    krows[t] = a.k + row0 + (size_t)t * D;
-    vrows[t] = a.v + row0 + (size_t)t * D;
-  }
-  stage_rows<D>(sm.k, krows, lane);
-  stage_rows<D>(sm.v, vrows, lane);
-  stage_kinv<D>(sm, stream_norm(a.buf, hd, a.g, b), lane);
+  stage_rows_contig<D>(sm.t.x, a.k + row0, lane);
+  if (KN) stage_kinv<D>(sm.kinv, stream_norm(a.buf, hd, a.g, b), lane);
   __syncwarp();
   uint8_t* rec = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)tile * hd.rec_bytes;
-  quantize_staged_tile<D>(sm, hd.k_bits, hd.v_bits, rec, lane);
+  pack_k_dispatch<D, KN>(sm.t, sm.kinv, hd.k_bits, rec, lane);
+  __syncwarp();  // every lane has read the K rows and statistics
+  stage_rows_contig<D>(sm.t.x, a.v + row0, lane);
+  __syncwarp();
+  pack_v_dispatch<D>(sm.t, hd.v_bits, rec + blob_bytes(hd.k_bits, D) + 4 * D, lane);
 }
 
-// Copy sink tokens [0, min(S,T)) and recent tokens [S+Tq, T) into the window block.
+// Copy sink tokens [0, min(S,T)) and recent tokens [S+Tq, T) into the window
+// block.  grid (streams, Y): the stream's 16-byte chunks (K and V rows) are
+// spread over Y blocks, one or two chunks per thread, so that the copy is a
+// few load latencies long rather than a chain of them.
 __global__ void copy_window_kernel(QuantizeArgs a) {
   const int s = blockIdx.x;
   const int h = s % a.g.Hkv, b = (s / a.g.Hkv) % a.g.B, l = s / (a.g.Hkv * a.g.B);
@@ -241,7 +75,7 @@ __global__ void copy_window_kernel(QuantizeArgs a) {
   const int rows = n_sink + (a.T - n_sink - a.Tq);
   const int chunks = D / 8;
   const size_t src0 = (size_t)s * a.T * D;
-  for (int j = threadIdx.x; j < rows * chunks * 2; j += blockDim.x) {
+  for (int j = blockIdx.y * blockDim.x + threadIdx.x; j < rows * chunks * 2; j += gridDim.y * blockDim.x) {
     const int kv = j / (rows * chunks);
     const int rj = (j % (rows * chunks)) / chunks, c = j % chunks;
     int pos, dst_row;
@@ -299,31 +133,20 @@ __global__ void __launch_bounds__(64) append_kernel(AppendArgs a) {
     krows[t] = reinterpret_cast<const uint16_t*>(win + ((size_t)2 * S + slot) * D * 2);
     vrows[t] = reinterpret_cast<const uint16_t*>(win + ((size_t)2 * S + ring + slot) * D * 2);
   }
-  if (warp == 0) stage_kinv<D>(sm, stream_norm(a.buf, hd, a.g, b), lane);
+  if (warp == 0) stage_kinv<D>(sm.kinv, stream_norm(a.buf, hd, a.g, b), lane);
   // rows were just written through global memory by this block: plain loads
 #pragma unroll 4
   for (int j = tid; j < kTile * kChunks; j += 64) {
     const int t = j / kChunks, c = j % kChunks;
-    *reinterpret_cast<uint4*>(&sm.k[t][c * 4]) = reinterpret_cast<const uint4*>(krows[t])[c];
-    *reinterpret_cast<uint4*>(&sm.v[t][c * 4]) = reinterpret_cast<const uint4*>(vrows[t])[c];
+    *reinterpret_cast<uint4*>(&sm.k.x[t][c * 4]) = reinterpret_cast<const uint4*>(krows[t])[c];
+    *reinterpret_cast<uint4*>(&sm.v.x[t][c * 4]) = reinterpret_cast<const uint4*>(vrows[t])[c];
   }
   __syncthreads();
   uint8_t* rec = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)a.flush_tile * hd.rec_bytes;
   if (warp == 0) {
-    switch (hd.k_bits) {
-      case 2: pack_k<D, 2>(sm, rec, lane); break;
-      case 3: pack_k<D, 3>(sm, rec, lane); break;
-      case 4: pack_k<D, 4>(sm, rec, lane); break;
-      default: pack_k<D, 8>(sm, rec, lane); break;
-    }
+    pack_k_dispatch<D, true>(sm.k, sm.kinv, hd.k_bits, rec, lane);
   } else {
-    uint8_t* vrec = rec + blob_bytes(hd.k_bits, D) + 4 * D;
-    switch (hd.v_bits) {
-      case 2: pack_v<D, 2>(sm, vrec, lane); break;
-      case 3: pack_v<D, 3>(sm, vrec, lane); break;
-      case 4: pack_v<D, 4>(sm, vrec, lane); break;
-      default: pack_v<D, 8>(sm, vrec, lane); break;
-    }
+    pack_v_dispatch<D>(sm.v, hd.v_bits, rec + blob_bytes(hd.k_bits, D) + 4 * D, lane);
   }
 }
 
@@ -426,6 +249,18 @@ __global__ void norm_finalize_kernel(QuantizeArgs a) {
   }
 }
 
+template <int D>
+void launch_tiles(const QuantizeArgs& a, dim3 grid, cudaStream_t st) {
+  const int smem = kQuantWarps * (int)sizeof(PrefillSmem<D>);
+  if (a.k_norm) {
+    cudaFuncSetAttribute(quantize_tiles_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    quantize_tiles_kernel<D, true><<<grid, kQuantWarps * 32, smem, st>>>(a);
+  } else {
+    cudaFuncSetAttribute(quantize_tiles_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    quantize_tiles_kernel<D, false><<<grid, kQuantWarps * 32, smem, st>>>(a);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_norm_reset(uint8_t* buf, const HeadDesc* desc, const Geom& g, cudaStream_t st) {
@@ -450,18 +285,21 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t st) {
   if (n_tiles > 0) {
     dim3 grid((n_tiles + kQuantWarps - 1) / kQuantWarps, streams);
     if (a.g.D == 128) {
-      const int smem = kQuantWarps * (int)sizeof(TileSmem<128>);
-      cudaFuncSetAttribute(quantize_tiles_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      quantize_tiles_kernel<128><<<grid, kQuantWarps * 32, smem, st>>>(a);
+      launch_tiles<128>(a, grid, st);
     } else {
-      const int smem = kQuantWarps * (int)sizeof(TileSmem<64>);
-      cudaFuncSetAttribute(quantize_tiles_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      quantize_tiles_kernel<64><<<grid, kQuantWarps * 32, smem, st>>>(a);
+      launch_tiles<64>(a, grid, st);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (a.T > 0) copy_window_kernel<<<streams, 128, 0, st>>>(a);
+  if (a.T > 0) {
+    const int n_sink = a.T < a.g.S ? a.T : a.g.S;
+    const int rows = n_sink + (a.T - n_sink - a.Tq);
+    const int items = rows * (a.g.D / 8) * 2;
+    int y = (items + 127) / 128;
+    y = y < 1 ? 1 : (y > 65535 ? 65535 : y);  // the loop strides over any remainder
+    copy_window_kernel<<<dim3(streams, y), 128, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 
