@@ -386,11 +386,16 @@ rq_status rq_decode_step(rq_cache* c, int layer, const void* q, const void* k_ne
   // present now; with n_recent >= 2 the token appended here is not among them.
   const int T = T_old + 1;
   const int Tq = rq::quantized_tokens(T, S, R);
-  const int n_pack =
-      (R >= 2 && T + 1 <= c->max_tokens && rq::quantized_tokens(T + 1, S, R) != Tq) ? 1 : 0;
+  int n_pack = (R >= 2 && T + 1 <= c->max_tokens && rq::quantized_tokens(T + 1, S, R) != Tq) ? 1 : 0;
   rq::DecodeArgs a;
   int smem = 0;
   rq_status st = fill_decode(c, l0, nl, T, q, out, softmax_scale, n_splits, workspace, ws_bytes, a, smem, n_pack);
+  if (n_pack && (st == RQ_ERR_WORKSPACE || st == RQ_ERR_UNSUPPORTED)) {
+    // no room for the extra item (a workspace sized without it, or an
+    // explicit split count at the item limit): the next step flushes itself
+    n_pack = 0;
+    st = fill_decode(c, l0, nl, T, q, out, softmax_scale, n_splits, workspace, ws_bytes, a, smem, 0);
+  }
   if (st != RQ_OK) return st;
   a.k_new = static_cast<const uint16_t*>(k_new);
   a.v_new = static_cast<const uint16_t*>(v_new);

@@ -195,6 +195,37 @@ def test_decode_step_equals_append_then_decode(S, R, context):
     assert QuantizedKVCache.rq_decode_read_status(ws) == 0
 
 
+def test_decode_step_without_room_for_the_pack_item():
+    """A workspace sized for the decode items only: the step before a tile
+    flush cannot add the pack-ahead item, so it skips it and the flush step
+    takes the two-launch path.  Outputs and bytes as the oracle's."""
+    wl = _small(n_layers=1, batch=1, context=4 + 32 * 3 + 32 + 20)
+    kb, vb = _bits_grid(1, wl.n_kv_heads)
+    steps, splits = 16, 2
+    cache, st, (k, v, f) = _build(wl, kb, vb, extra=steps)
+    q, kn, vn = workloads.step_inputs(wl, steps, f, "cuda")
+    knp, vnp, qnp = to_f32(kn), to_f32(vn), to_f32(q).astype(np.float64)
+    # layout: [status, counters: 64 u32 per stream][partials: streams x items x (G*D + 2G) floats];
+    # the full size holds splits + 3 window items + 1 pack item, every window here needs one item
+    streams = wl.batch * wl.n_kv_heads
+    offset = 256 + streams * 64 * 4
+    part = (wl.group * wl.head_dim + 2 * wl.group) * 4
+    assert cache.rq_decode_workspace_bytes(splits) == offset + streams * (splits + 3 + 1) * part
+    ws = torch.zeros(offset + streams * (splits + 1) * part, dtype=torch.uint8, device="cuda")
+    flushes = 0
+    for t in range(steps):
+        for (l, b, h), s in st.items():
+            flushes += s.append(knp[t, l, b, h], vnp[t, l, b, h])
+        out = cache.rq_decode_step(0, q[t, 0].contiguous(), kn[t, 0].contiguous(), vn[t, 0].contiguous(),
+                                   n_splits=splits, workspace=ws).cpu().numpy()
+        exp = oracle_decode(wl, st, qnp[t], [(0, 0)])[(0, 0)]
+        assert_close(out[0], exp, f"step {t}")
+    assert flushes > 0
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_k_norm_prefill_decode_and_steps(d):
     """Per-channel K normalization: factors, tile records and window rows bit
