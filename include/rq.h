@@ -253,7 +253,9 @@ rq_status rq_decode_attention(rq_cache* cache, int layer, const void* q, float* 
  *   rq_append_token, or any step when n_recent < 2 -- quantizes the tile
  *   first and decodes after (two launches).  Results are those of the two
  *   calls in every case.  Workspace: rq_decode_workspace_bytes includes the
- *   extra item.  On an error nothing is launched and the length is
+ *   extra item; a workspace (or an explicit n_splits at the item limit) with
+ *   no room for it makes the step skip the pack-ahead, and the next step
+ *   flushes with two launches.  On an error nothing is launched and the length is
  *   unchanged; otherwise the length grows by one.  The pages have no
  *   separate counterpart: it is the two operations above, fused. */
 rq_status rq_decode_step(rq_cache* cache, int layer, const void* q, const void* k_new, const void* v_new,
