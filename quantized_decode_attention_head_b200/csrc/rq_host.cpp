@@ -401,6 +401,17 @@ rq_status rq_decode_step(rq_cache* c, int layer, const void* q, const void* k_ne
   a.v_new = static_cast<const uint16_t*>(v_new);
   a.pack_pos = S + Tq;
   a.pack_tile = Tq / rq::kTile;
+  if (packed && Tq != rq::quantized_tokens(T_old, S, R)) {
+    // This launch reads the tile the previous decode launch packed ahead.  A
+    // decode launch may start before its predecessor ends (programmatic
+    // dependent launch) and fetches its first tile records before waiting on
+    // it, so it must not follow the packing launch directly: a 4-byte memset
+    // of the workspace's padding (bytes 4..7, unused) in between makes it a
+    // plain stream dependency -- the packing launch completes first.  This
+    // holds in stream capture too (a memset node, not a kernel edge).
+    st = cuda_status(cudaMemsetAsync(static_cast<uint8_t*>(workspace) + 4, 0, 4, stream));
+    if (st != RQ_OK) return st;
+  }
   st = cuda_status(rq::launch_decode(a, smem, stream));
   if (st != RQ_OK) return st;
   for (int l = l0; l < l0 + nl; ++l) {
