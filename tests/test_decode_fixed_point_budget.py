@@ -31,19 +31,23 @@ def _bf16_to_f64(t):
     return qz.bf16_bits_to_f32(t.contiguous().view(torch.int16).numpy().view(np.uint16)).astype(np.float64)
 
 
-def _emulated_decode(q, kh, vh, S, Tq, n_splits, n_warps=4, rounding=True):
+def _emulated_decode(q, kh, vh, S, Tq, n_splits, n_warps=4, rounding=True, nrm=None):
     """Output [G, D] of the kernel's arithmetic model for one stream
-    (rounding=False: q_int and p_int left unrounded)."""
+    (rounding=False: q_int and p_int left unrounded).  nrm: the K
+    normalization factors of a normalized cache -- the tiles hold K / n and
+    the tile products use q * n (exact: powers of two), whose fixed point
+    then spans the channels' whole range."""
     rint = np.rint if rounding else (lambda x: x)
     G, D = q.shape
     scale = 1.0 / np.sqrt(D)
-    q32 = q.astype(np.float32)
+    n = np.ones(D) if nrm is None else np.asarray(nrm, dtype=np.float64)
+    q32 = (q * n).astype(np.float32)
     mx = np.abs(q32).max(axis=1, keepdims=True)
     inv = np.where(mx > 0, np.float32(QMAX) / mx, np.float32(0)).astype(np.float32)
     q_int = np.clip(rint((q32 * inv).astype(np.float64)), -QMAX, QMAX)
     sq = (mx.astype(np.float64) / QMAX)[:, 0]
     n_tiles = Tq // 32
-    x_tiles = (kh[S:S + Tq] @ q_int.T) * sq * scale * LOG2E  # base-2 logits [Tq, G]
+    x_tiles = ((kh[S:S + Tq] / n) @ q_int.T) * sq * scale * LOG2E  # base-2 logits [Tq, G]
     parts = []  # (m [G], l [G], o [G, D])
     for item in range(n_splits):
         t0, t1 = item * n_tiles // n_splits, (item + 1) * n_tiles // n_splits
@@ -74,12 +78,12 @@ def _emulated_decode(q, kh, vh, S, Tq, n_splits, n_warps=4, rounding=True):
     return O / L[:, None]
 
 
-def _stream(name, bits):
-    wl = workloads.CONFIGS[name]
+def _stream(name, bits, k_norm=False, **over):
+    wl = workloads.CONFIGS[name].with_(**over)
     one = wl.with_(n_layers=1, batch=1, n_kv_heads=1, n_q_heads=wl.group)
     k, v, f = workloads.kv_inputs(one, "cpu")
     q, _, _ = workloads.step_inputs(one, 1, f, "cpu")
-    st = ca.StreamCache(wl.head_dim, bits, bits, wl.n_sink, wl.n_recent)
+    st = ca.StreamCache(wl.head_dim, bits, bits, wl.n_sink, wl.n_recent, k_norm=k_norm)
     st.prefill(_bf16_to_f64(k)[0, 0, 0].astype(np.float32), _bf16_to_f64(v)[0, 0, 0].astype(np.float32))
     kh, vh = st.dequantized()
     return wl, _bf16_to_f64(q)[0, 0, 0], kh, vh, st
@@ -109,3 +113,16 @@ def test_fixed_point_model_is_exact_without_rounding():
     # and the roundings are what moves it: rounded, the error is orders larger
     err = np.abs(_emulated_decode(q, kh, vh, S, Tq, n_splits=6) - exp).max()
     assert 1e-6 < err < 1e-3
+
+
+def test_k_norm_fixed_point_error_budget():
+    """A normalized cache (K / n in the tiles, q * n in the tile products) at
+    outlier sigma = 1.0, the setting of the GPU parity test for normalized
+    caches: the query's 16-bit fixed point now spans every channel's
+    magnitude, and the error still stays under half the tolerance."""
+    wl, q, kh, vh, st = _stream("long_128k", 2, k_norm=True, k_sigma=1.0)
+    got = _emulated_decode(q, kh, vh, wl.n_sink, st.n_tiles * 32, n_splits=66, nrm=st.nrm)
+    exp = at.attend(q, kh, vh)
+    err = np.abs(got - exp).max()
+    rel = np.linalg.norm(got - exp) / np.linalg.norm(exp)
+    assert err < 1e-3 and rel < 5e-4, (err, rel)
