@@ -13,7 +13,7 @@ Rate-Distortion Theory" (paperlayer.ai summary of arXiv 2605.06675v2).
   b_min, repeatedly give one bit to the head with the largest weighted
   marginal gain (max-heap), optimal because the gains decrease in b.
 
-Readings taken where the page is silent (each also listed in the design doc):
+Readings taken where the page is silent:
 
 * The stationary point of the Lagrangian of sum w a beta^-b + lambda*(sum b)
   gives b_h(lambda) = log_beta_h(w_h alpha_h ln(beta_h) / lambda); it is

@@ -11,7 +11,7 @@ precision windows for the most recent tokens and for the attention-sink tokens;
 NOVA-KV review page ("Spend Bits Where Queries Look"), assumptions list: sink
 and recent bands kept apart from the quantized body.
 
-Readings where the pages are silent (also listed in the design doc):
+Readings where the pages are silent:
 
 * Tq = 32 * floor((T - S - R) / 32) when T >= S + R, else 0, so the recent
   window length r = T - S - Tq lies in [R, R + 32) (InnerQ gives no rule for a
