@@ -66,9 +66,10 @@ def ring_slot(pos: int, n_sink: int, n_recent: int) -> int:
 class StreamCache:
     """Quantized cache of one stream, built token by token or by prefill."""
 
-    def __init__(self, head_dim, k_bits, v_bits, n_sink, n_recent, k_norm=False):
+    def __init__(self, head_dim, k_bits, v_bits, n_sink, n_recent, k_norm=False, hybrid=False):
         self.d = head_dim
         self.k_norm = k_norm
+        self.hybrid = hybrid  # per-group symmetric / asymmetric choice (quantize.quantize_groups)
         self.nrm = np.ones(head_dim, dtype=np.float32)  # per-channel K normalization n_d
         self.kb = k_bits
         self.vb = v_bits
@@ -93,7 +94,8 @@ class StreamCache:
         n = tq // TILE
         if n:
             d = self.d
-            qb = qz.quantize_tiles(kn[s : s + tq].reshape(n, TILE, d), v[s : s + tq].reshape(n, TILE, d), self.kb, self.vb)
+            qb = qz.quantize_tiles(kn[s : s + tq].reshape(n, TILE, d), v[s : s + tq].reshape(n, TILE, d), self.kb, self.vb,
+                                   self.hybrid)
             self.tiles = [{key: val[i] for key, val in qb.items()} for i in range(n)]
         self.recent = [(p, k[p].copy(), v[p].copy()) for p in range(s + tq, T)]
         self.T = T
@@ -112,7 +114,7 @@ class StreamCache:
             self.recent = self.recent[TILE:]
             kt = (np.stack([o[1] for o in old]) / self.nrm).astype(np.float32)
             vt = np.stack([o[2] for o in old])
-            self.tiles.append(qz.quantize_tile(kt, vt, self.kb, self.vb))
+            self.tiles.append(qz.quantize_tile(kt, vt, self.kb, self.vb, self.hybrid))
             return True
         return False
 

@@ -15,7 +15,15 @@ high precision.
 The rounding rule (every step IEEE fp32, round-to-nearest-even, no FMA):
 
     x  = bf16 input widened to fp32 (exact)
-    mn, mx = min, max over the group
+    mn, mx = min, max over the group, each + 0.0 (a -0.0 extreme is stored
+             as +0.0: the pages fix no sign for a zero extreme)
+    hybrid option only (InnerQ technique (i), a symmetric or asymmetric
+    quantizer per group chosen from the group's own statistics; the page
+    prints no rule, this is the reading): a group that is nearly centred on
+    zero, |mx + mn| <= TAU * (mx - mn) in fp32 with TAU = 1/8, is quantized
+    on the symmetric interval [-M, M], M = max(|mn|, |mx|):
+               mn, mx = -M, M     (exact: M is a bf16 value)
+    and every other group on [mn, mx]; the rest of the rule is the same
     s32 = (mx - mn) / (2**b - 1)             fp32 subtract, fp32 divide
     s16 = fp16_rne(min(s32, 65504))           stored scale (fp16)
     s   = fp32(s16)
@@ -77,6 +85,9 @@ import numpy as np
 
 TILE = 32  # tokens per quantized tile == group size g
 CPW = {2: 16, 3: 10, 4: 8, 8: 4}
+# hybrid option: a group with |max + min| <= TAU * (max - min) is quantized on
+# the symmetric interval [-M, M] (power of two, so TAU * w is exact in fp32)
+TAU = np.float32(0.125)
 
 
 # ---------------------------------------------------------------- bf16 helpers
@@ -94,18 +105,38 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
 
 
 # ------------------------------------------------------------------ quantizer
-def quantize_groups(x: np.ndarray, b: int, axis: int):
+def symmetric_groups(mn: np.ndarray, mx: np.ndarray) -> np.ndarray:
+    """Hybrid rule: True where a group with extremes (mn, mx) is nearly
+    centred on zero, |mx + mn| <= TAU * (mx - mn), each side one fp32
+    operation rounded to nearest even."""
+    mn = np.asarray(mn, dtype=np.float32)
+    mx = np.asarray(mx, dtype=np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        centre = np.abs((mx + mn).astype(np.float32))
+        width = ((mx - mn).astype(np.float32) * TAU).astype(np.float32)
+    return centre <= width
+
+
+def quantize_groups(x: np.ndarray, b: int, axis: int, hybrid: bool = False):
     """Quantize float32 (bf16-valued) data in groups that run along ``axis``.
 
     Returns (codes uint8 same shape as x, s16 float16, z float32) where s16 and
-    z have ``axis`` removed.
+    z have ``axis`` removed.  hybrid: centred groups on [-M, M] (see above).
     """
     if b not in CPW:
         raise ValueError(f"unsupported bit width {b}")
     x = np.asarray(x, dtype=np.float32)
     qmax = np.float32((1 << b) - 1)
-    mn = np.min(x, axis=axis)
-    mx = np.max(x, axis=axis)
+    # min and max as real numbers: a -0.0 extreme becomes +0.0 (x + 0 in IEEE
+    # round-to-nearest), so which of two equal zeros a reduction returns does
+    # not matter
+    mn = (np.min(x, axis=axis) + np.float32(0.0)).astype(np.float32)
+    mx = (np.max(x, axis=axis) + np.float32(0.0)).astype(np.float32)
+    if hybrid:
+        sym = symmetric_groups(mn, mx)
+        m = np.maximum(np.abs(mn), np.abs(mx)).astype(np.float32)
+        mn = np.where(sym, (-m + np.float32(0.0)).astype(np.float32), mn).astype(np.float32)
+        mx = np.where(sym, m, mx).astype(np.float32)
     with np.errstate(over="ignore", invalid="ignore"):
         s32 = (mx - mn).astype(np.float32) / qmax
     s32 = np.minimum(s32, np.float32(65504.0)).astype(np.float32)
@@ -122,25 +153,25 @@ def quantize_groups(x: np.ndarray, b: int, axis: int):
     return c, s16, mn.astype(np.float32)
 
 
-def quantize_tile(k_tile: np.ndarray, v_tile: np.ndarray, kb: int, vb: int):
+def quantize_tile(k_tile: np.ndarray, v_tile: np.ndarray, kb: int, vb: int, hybrid: bool = False):
     """Quantize one 32-token tile.  k_tile, v_tile: float32 [32, D] (bf16 values).
 
     K groups: per token, 32 consecutive channels.  V groups: per channel, the
     tile's 32 tokens.  Returns dict with codes [32, D] (token-major) for K and
     V, K scale/zero [32, D/32], V scale/zero [D].
     """
-    q = quantize_tiles(k_tile[None], v_tile[None], kb, vb)
+    q = quantize_tiles(k_tile[None], v_tile[None], kb, vb, hybrid)
     return {key: val[0] for key, val in q.items()}
 
 
-def quantize_tiles(k_tiles: np.ndarray, v_tiles: np.ndarray, kb: int, vb: int):
+def quantize_tiles(k_tiles: np.ndarray, v_tiles: np.ndarray, kb: int, vb: int, hybrid: bool = False):
     """The same rule applied to n tiles at once: inputs [n, 32, D]; outputs
     carry a leading tile axis."""
     n, t, d = k_tiles.shape
     assert t == TILE and d % 32 == 0
     kx = np.asarray(k_tiles, dtype=np.float32).reshape(n, TILE, d // 32, 32)
-    kc, ks, kz = quantize_groups(kx, kb, axis=3)
-    vc, vs, vz = quantize_groups(np.asarray(v_tiles, dtype=np.float32), vb, axis=1)
+    kc, ks, kz = quantize_groups(kx, kb, axis=3, hybrid=hybrid)
+    vc, vs, vz = quantize_groups(np.asarray(v_tiles, dtype=np.float32), vb, axis=1, hybrid=hybrid)
     return {
         "k_codes": kc.reshape(n, TILE, d),
         "k_s": ks,  # [n, 32 tokens, D/32 groups]

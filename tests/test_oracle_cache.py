@@ -47,17 +47,18 @@ def test_flush_schedule_of_append_run():
     assert flushed == [4, 36]
 
 
+@pytest.mark.parametrize("hybrid", [False, True])
 @pytest.mark.parametrize("T0,T1,S,R", [(100, 230, 4, 32), (36, 99, 4, 32), (0, 80, 4, 32), (2, 70, 4, 0), (40, 200, 0, 16)])
-def test_prefill_then_append_equals_prefill(T0, T1, S, R):
+def test_prefill_then_append_equals_prefill(T0, T1, S, R, hybrid):
     rng = np.random.default_rng(T0 + T1)
     d = 64
     k = qz.bf16_bits_to_f32(rng.integers(0x3C00, 0x4100, size=(T1, d), dtype=np.uint16) ^ rng.integers(0, 2, size=(T1, d), dtype=np.uint16) << 15)
     v = qz.bf16_bits_to_f32(rng.integers(0x3C00, 0x4100, size=(T1, d), dtype=np.uint16))
-    a = ca.StreamCache(d, 3, 2, S, R)
+    a = ca.StreamCache(d, 3, 2, S, R, hybrid=hybrid)
     a.prefill(k[:T0], v[:T0])
     for t in range(T0, T1):
         a.append(k[t], v[t])
-    b = ca.StreamCache(d, 3, 2, S, R)
+    b = ca.StreamCache(d, 3, 2, S, R, hybrid=hybrid)
     b.prefill(k, v)
     assert a.T == b.T == T1 and a.n_tiles == b.n_tiles
     for i in range(a.n_tiles):

@@ -106,6 +106,104 @@ def test_constant_group_is_exact():
         assert np.all(c == 0) and np.all(s == 0) and np.all(z == np.float32(-2.375))
 
 
+def _signed_zero_groups():
+    """Groups of 32 whose extremes are zeros of either sign: all +0, all -0,
+    mixed zeros, a -0 minimum under positives, a -0 maximum over negatives."""
+    rows = [np.zeros(32), -np.zeros(32), np.where(np.arange(32) % 3 == 0, -0.0, 0.0)]
+    r = np.linspace(0.25, 8.0, 32)
+    r[[0, 17]] = [-0.0, 0.0]
+    rows.append(r)
+    r = -np.linspace(0.5, 3.0, 32)
+    r[[5, 30]] = [0.0, -0.0]
+    rows.append(r)
+    return np.asarray(rows, dtype=np.float32)
+
+
+def test_signed_zero_extremes_are_order_free():
+    """min and max are taken as real numbers, so the stored zero and scale of
+    a group do not depend on the order of its elements (a group's extremes
+    are a property of the set); a zero extreme is stored as +0.0 and an
+    all-zero group dequantizes to exactly zero."""
+    x = _signed_zero_groups()
+    rng = np.random.default_rng(5)
+    for b in BITS:
+        c0, s0, z0 = qz.quantize_groups(x, b, axis=1)
+        assert not np.any(np.signbit(z0)[:4]) and not np.any(np.signbit(s0))
+        assert np.all(c0[:3] == 0) and np.all(s0[:3] == 0) and np.all(z0[:3] == 0)
+        assert z0[3] == 0 and s0[3] == np.float16(np.float32(8.0) / np.float32((1 << b) - 1))
+        assert z0[4] == np.float32(-3.0)
+        for _ in range(8):
+            perm = rng.permutation(32)
+            c, s, z = qz.quantize_groups(x[:, perm], b, axis=1)
+            assert np.array_equal(c, c0[:, perm])
+            assert np.array_equal(s.view(np.uint16), s0.view(np.uint16))
+            assert np.array_equal(z.view(np.uint32), z0.view(np.uint32))
+        xh = c0.astype(np.float64) * s0.astype(np.float64)[:, None] + z0.astype(np.float64)[:, None]
+        assert np.all(xh[:3] == 0)
+
+
+def _centred_and_offset_groups(rng, n=64):
+    """Groups of 32 bf16 values: the first half centred on zero (a symmetric
+    law), the second half shifted well away from zero."""
+    x = rng.normal(size=(n, 32)).astype(np.float32) * np.exp(rng.normal(size=(n, 1))).astype(np.float32)
+    x[n // 2:] += (3.0 * np.abs(x[n // 2:]).max(axis=1, keepdims=True)).astype(np.float32)
+    return _bf16(x)
+
+
+@pytest.mark.parametrize("b", BITS)
+def test_hybrid_chooses_by_centring(b):
+    """Hybrid rule (InnerQ technique (i), reading: centred groups are quantized
+    on the symmetric interval [-M, M]): a group with |max + min| <= (max - min)/8
+    gets z = -M and s = fp16(2M / (2^b - 1)); any other group is quantized
+    exactly as without the option."""
+    rng = np.random.default_rng(100 + b)
+    x = _centred_and_offset_groups(rng)
+    c_a, s_a, z_a = qz.quantize_groups(x, b, axis=1)
+    c_h, s_h, z_h = qz.quantize_groups(x, b, axis=1, hybrid=True)
+    mn, mx = x.min(axis=1), x.max(axis=1)
+    sym = np.abs(mx.astype(np.float64) + mn) <= (mx.astype(np.float64) - mn) / 8
+    assert sym[:32].sum() >= 8 and not sym[32:].any()  # the generator gives both kinds
+    m = np.maximum(np.abs(mn), np.abs(mx))
+    assert np.array_equal(z_h[sym], -m[sym])
+    assert np.array_equal(s_h[sym], (np.float32(2.0) * m[sym] / np.float32((1 << b) - 1)).astype(np.float16))
+    for arr_h, arr_a in ((c_h, c_a), (s_h, s_a), (z_h, z_a)):
+        assert np.array_equal(arr_h[~sym], arr_a[~sym])
+    # the half-step bound holds on either interval
+    xh = c_h * s_h.astype(np.float64)[:, None] + z_h.astype(np.float64)[:, None]
+    assert np.all(np.abs(xh - x) <= s_h.astype(np.float64)[:, None] * 0.5 * (1 + 2**-10))
+
+
+@pytest.mark.parametrize("b", BITS)
+def test_hybrid_symmetric_group_equals_the_group_widened_to_plus_minus_m(b):
+    """A symmetric group is quantized as the asymmetric rule quantizes the same
+    group with -M and +M added to it (its extremes become exactly -M, M): an
+    independent statement of 'the interval is [-M, M]'."""
+    rng = np.random.default_rng(200 + b)
+    x = _centred_and_offset_groups(rng)[:32]
+    c_h, s_h, z_h = qz.quantize_groups(x, b, axis=1, hybrid=True)
+    m = np.maximum(np.abs(x.min(axis=1)), np.abs(x.max(axis=1)))
+    sym = qz.symmetric_groups(x.min(axis=1), x.max(axis=1))
+    wide = np.concatenate([x, -m[:, None], m[:, None]], axis=1)
+    c_w, s_w, z_w = qz.quantize_groups(wide, b, axis=1)
+    assert sym.sum() >= 8
+    assert np.array_equal(c_h[sym], c_w[sym, :32])
+    assert np.array_equal(s_h[sym], s_w[sym]) and np.array_equal(z_h[sym], z_w[sym])
+
+
+def test_hybrid_threshold_is_inclusive():
+    """|max + min| = (max - min) / 8 exactly is centred; a hair more is not."""
+    g_on = np.full((1, 32), 1.0, dtype=np.float32)
+    g_on[0, 0], g_on[0, 1] = -7.0, 9.0          # |2| = 16 / 8
+    g_off = g_on.copy()
+    g_off[0, 1] = 9.0625                       # |2.0625| > 16.0625 / 8 (bf16 value)
+    assert qz.symmetric_groups(g_on.min(axis=1), g_on.max(axis=1))[0]
+    assert not qz.symmetric_groups(g_off.min(axis=1), g_off.max(axis=1))[0]
+    _, s, z = qz.quantize_groups(g_on, 2, axis=1, hybrid=True)
+    assert z[0] == -9.0 and s[0] == np.float16(6.0)
+    _, s, z = qz.quantize_groups(g_off, 2, axis=1, hybrid=True)
+    assert z[0] == -7.0
+
+
 @pytest.mark.parametrize("role", ["K", "V"])
 @pytest.mark.parametrize("b", BITS)
 @pytest.mark.parametrize("d", [64, 128])
