@@ -59,6 +59,8 @@
  *            entry i = channel 16*mb + 8*rr + gid, gid = i/(D/8),
  *            mb = (i%(D/8))/2, rr = i%2.
  *   Quantization rule per group (IEEE fp32, round to nearest even):
+ *     max, min = the group's extremes, each + 0 (a -0.0 extreme becomes +0.0),
+ *       replaced by M, -M + 0 for a centred group of a hybrid cache (config),
  *     s = fp16(min((max - min) / (2^b - 1), 65504)), z = min (bf16),
  *     c = clamp(rint((x - z) * (s > 0 ? 1/s : 0)), 0, 2^b - 1).
  *   Windows per stream: sink K [S][D], sink V [S][D], recent ring K [R+32][D],
@@ -164,6 +166,13 @@ typedef struct {
                         n_d = smallest power of two >= max_t |K[t, d]| per stream and channel
                         over the prefill tokens, tiles hold K / n, queries are multiplied by n
                         for the quantized tokens; 0: n = 1.  Windows keep K as is. */
+  int hybrid;        /* 1: symmetric or asymmetric quantizer per group (InnerQ abstract,
+                        technique (i); this library's rule): a group with
+                        |max + min| <= (max - min) / 8 (fp32) is quantized on [-M, M],
+                        M = max(|min|, |max|), i.e. min := -M, max := M in the rule below;
+                        other groups on [min, max].  The record format and the decode are
+                        the same either way (every group stores its own scale and zero).
+                        0: every group asymmetric. */
 } rq_cache_config;
 
 typedef struct rq_cache rq_cache; /* opaque host handle */
@@ -172,10 +181,12 @@ typedef struct rq_cache rq_cache; /* opaque host handle */
 rq_status rq_cache_bytes(const rq_cache_config* cfg, size_t* bytes);
 
 /* Bind a caller-owned device buffer (>= rq_cache_bytes, 256-byte aligned) to
- * a new host handle with length 0.  Writes the buffer's descriptor header with
- * a synchronous cudaMemcpy on the current device and sets every stream's K
- * normalization factors to 1, waiting for both (the only blocking call
- * besides rq_decode_read_status).  *out receives the handle. */
+ * a new host handle with length 0.  Writes the buffer's descriptor header and
+ * sets every stream's K normalization factors to 1 on a private non-blocking
+ * stream of the current device and waits for that stream only (a blocking
+ * call, like rq_decode_read_status; other streams are not serialised behind
+ * it).  The buffer must not be in use by other streams meanwhile.  *out
+ * receives the handle. */
 rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes, rq_cache** out);
 
 /* Free the host handle (never the device buffer).  NULL is ignored. */
@@ -268,6 +279,17 @@ rq_status rq_decode_step(rq_cache* cache, int layer, const void* q, const void* 
  * without writing its outputs). */
 rq_status rq_decode_read_status(const void* workspace, int* device_status);
 
+/* rq_selftest_device_timeout -- exercises the device timeout path without a
+ *   fault: one thread waits on an mbarrier that nothing completes, using the
+ *   bounded wait of the decode pipeline with the given limit (limit_ns <= 1e9),
+ *   gives up and records RQ_ERR_DEVICE_TIMEOUT in the workspace status word as
+ *   a decode kernel would; rq_decode_read_status then reports it.  Clear the
+ *   word again with rq_decode_workspace_init.  The pages have no counterpart.
+ * Errors: RQ_ERR_INVALID_ARG (null or too small workspace, limit above 1 s),
+ *   RQ_ERR_CUDA. */
+rq_status rq_selftest_device_timeout(void* workspace, size_t ws_bytes, unsigned long long limit_ns,
+                                     cudaStream_t stream);
+
 /* rq_decode_attention_noalloc -- the same decode step as rq_decode_attention,
  *   for callers that cannot allocate device memory: code running where
  *   cudaMalloc is unavailable or forbidden (inside a custom allocator or
@@ -285,15 +307,27 @@ rq_status rq_decode_read_status(const void* workspace, int* device_status);
  * All calls share the one array, which keeps the last call's contents: calls
  *   that overlap on the GPU (other streams, other threads, other handles)
  *   race and corrupt each other's results; serialise them.
- * Arguments as rq_decode_attention, minus the workspace.  The device status
- *   word is not readable through the C ABI for this variant.
+ * Arguments as rq_decode_attention, minus the workspace.  The call returns
+ *   before the kernel runs, so a pipeline wait that gives up on the device
+ *   (the kernel then leaves out untouched) shows only in the array's status
+ *   word: read it with rq_decode_noalloc_read_status.
  * n_splits = 0 takes the automatic plan, reduced to the most splits whose
- *   partials fit the array when the plan needs more.
+ *   partials fit the array (in the plan's own cluster size) when the plan
+ *   needs more.
  * Errors: RQ_ERR_INVALID_ARG; RQ_ERR_WORKSPACE when the split partials of the
  *   call (about (n_splits + 2) * streams * (G*D + 2G) * 4 bytes) exceed the
  *   array -- reduce n_splits or decode fewer layers per call; RQ_ERR_CUDA. */
 rq_status rq_decode_attention_noalloc(rq_cache* cache, int layer, const void* q, float* out,
                                       float softmax_scale, int n_splits, cudaStream_t stream);
+
+/* rq_decode_noalloc_read_status -- blocking read of the status word of the
+ *   scratch array behind rq_decode_attention_noalloc on the current device
+ *   (waits for the device's work queued before it): 0 when the last call on
+ *   this device completed normally, RQ_ERR_DEVICE_TIMEOUT in the low byte
+ *   when a pipeline wait of that call gave up.  Each call clears the word, so
+ *   it reflects the LAST call made on the device (from any thread).
+ * Errors: RQ_ERR_INVALID_ARG (null pointer), RQ_ERR_CUDA. */
+rq_status rq_decode_noalloc_read_status(int* device_status);
 
 /* Library build description (static string). */
 const char* rq_build_info(void);

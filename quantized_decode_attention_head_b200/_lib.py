@@ -45,6 +45,7 @@ class CacheConfig(ctypes.Structure):
         ("k_bits", ctypes.POINTER(ctypes.c_int)),
         ("v_bits", ctypes.POINTER(ctypes.c_int)),
         ("k_norm", ctypes.c_int),
+        ("hybrid", ctypes.c_int),
     ]
 
 
@@ -74,7 +75,9 @@ SIGNATURES = {
     "rq_decode_attention": (_I, [_P, _I, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "rq_decode_step": (_I, [_P, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "rq_decode_read_status": (_I, [_P, _IP]),
+    "rq_selftest_device_timeout": (_I, [_P, _SZ, ctypes.c_ulonglong, _P]),
     "rq_decode_attention_noalloc": (_I, [_P, _I, _P, _P, ctypes.c_float, _I, _P]),
+    "rq_decode_noalloc_read_status": (_I, [_IP]),
 }
 
 _lib = None

@@ -109,13 +109,13 @@ def rq_cap_weights(w, factor=5.0):
 
 
 def _config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, n_sink, n_recent, max_tokens, k_bits, v_bits, group=32,
-            k_norm=False):
+            k_norm=False, hybrid=False):
     kb = np.ascontiguousarray(np.asarray(k_bits, dtype=np.int32).reshape(-1))
     vb = np.ascontiguousarray(np.asarray(v_bits, dtype=np.int32).reshape(-1))
     ip = ctypes.POINTER(ctypes.c_int)
     cfg = CacheConfig(
         n_layers, batch, n_q_heads, n_kv_heads, head_dim, group, n_sink, n_recent, max_tokens,
-        kb.ctypes.data_as(ip), vb.ctypes.data_as(ip), int(bool(k_norm)),
+        kb.ctypes.data_as(ip), vb.ctypes.data_as(ip), int(bool(k_norm)), int(bool(hybrid)),
     )
     return cfg, (kb, vb)
 
@@ -131,7 +131,7 @@ class QuantizedKVCache:
     """Owns a device buffer (torch uint8 tensor) and the library's host handle."""
 
     def __init__(self, n_layers, batch, n_q_heads, n_kv_heads, head_dim, n_sink, n_recent, max_tokens,
-                 k_bits, v_bits, device="cuda", group=32, k_norm=False):
+                 k_bits, v_bits, device="cuda", group=32, k_norm=False, hybrid=False):
         import torch
 
         self.n_layers, self.batch = n_layers, batch
@@ -140,8 +140,9 @@ class QuantizedKVCache:
         self.k_bits = np.asarray(k_bits, dtype=np.int32).reshape(n_layers, n_kv_heads)
         self.v_bits = np.asarray(v_bits, dtype=np.int32).reshape(n_layers, n_kv_heads)
         cfg, keep = _config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, n_sink, n_recent, max_tokens,
-                            self.k_bits, self.v_bits, group, k_norm)
+                            self.k_bits, self.v_bits, group, k_norm, hybrid)
         self.k_norm = bool(k_norm)
+        self.hybrid = bool(hybrid)
         nbytes = ctypes.c_size_t(0)
         check("rq_cache_bytes", lib().rq_cache_bytes(ctypes.byref(cfg), ctypes.byref(nbytes)))
         self.nbytes = nbytes.value

@@ -15,7 +15,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "librq.so")
-SOURCES = ["rq_alloc.cpp", "rq_host.cpp", "rq_quantize.cu", "rq_decode.cu"]
+# the decode kernel is instantiated once per (head_dim, GQA group) pair in its
+# own translation unit, so the units compile in parallel
+SOURCES = ["rq_alloc.cpp", "rq_host.cpp", "rq_quantize.cu", "rq_decode.cu"] + [
+    f"rq_decode_{d}x{g}.cu" for d in (128, 64) for g in (1, 2, 4, 8)]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -50,7 +53,7 @@ def _compile(src, ptxas_verbose):
 
 def build(ptxas_verbose: bool = False, quiet: bool = True) -> str:
     os.makedirs(OBJ, exist_ok=True)
-    with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+    with ThreadPoolExecutor(max_workers=min(len(SOURCES), os.cpu_count() or 4)) as ex:
         results = list(ex.map(lambda s: _compile(s, ptxas_verbose), SOURCES))
     objs = [o for o, _ in results]
     logs = "".join(l for _, l in results)

@@ -105,13 +105,19 @@ void knapsack(int n, const double* w, const double* alpha, const double* beta, c
   // g[h][u]: least distortion of heads h..n-1 using at most u bits
   std::vector<double> g((size_t)(n + 1) * (cap + 1), inf);
   auto G = [&](int h, long u) -> double& { return g[(size_t)h * (cap + 1) + u]; };
+  // distortion of head h at width S[j], computed once per (h, j)
+  const int ns = (int)S.size();
+  std::vector<double> dist((size_t)n * ns);
+  for (int h = 0; h < n; ++h)
+    for (int j = 0; j < ns; ++j) dist[(size_t)h * ns + j] = w[h] * alpha[h] * std::pow(beta[h], -S[j]);
   for (long u = 0; u <= cap; ++u) G(n, u) = 0.0;
   for (int h = n - 1; h >= 0; --h)
     for (long u = 0; u <= cap; ++u) {
       double best = inf;
-      for (int b : S) {
+      for (int j = 0; j < ns; ++j) {
+        const int b = S[j];
         if (b > u) continue;
-        const double v = G(h + 1, u - b) + w[h] * alpha[h] * std::pow(beta[h], -b);
+        const double v = G(h + 1, u - b) + dist[(size_t)h * ns + j];
         if (v < best) best = v;
       }
       G(h, u) = best;
@@ -122,7 +128,7 @@ void knapsack(int n, const double* w, const double* alpha, const double* beta, c
     for (int j = (int)S.size() - 1; j >= 0; --j) {
       const int b = S[j];
       if (b > u) continue;
-      const double v = G(h + 1, u - b) + w[h] * alpha[h] * std::pow(beta[h], -b);
+      const double v = G(h + 1, u - b) + dist[(size_t)h * ns + j];
       if (v <= target * (1.0 + 1e-12) + 1e-300) {
         out[h] = b;
         u -= b;

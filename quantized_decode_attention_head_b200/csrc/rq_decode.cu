@@ -1,1025 +1,11 @@
-// Split-K decode attention over the packed cache (sm_100a).
-//
-// One CTA = one work item of one (layer, batch, kv-head) stream: either a
-// contiguous range of packed tiles (items 0..n_splits-1) or the bf16 sink +
-// recent window (items n_splits..).  Four warps process tiles; lane 0 of each
-// streams the warp's own tile records into a private ring of shared-memory
-// stages with 1-D bulk copies (cp.async.bulk, TMA engine) completing on
-// mbarriers.  Consecutive items of a stream form thread-block clusters; the
-// first CTA of each cluster merges its cluster's partial softmax states
-// (log-sum-exp) from distributed shared memory, and the CTAs of the stream's
-// last cluster to finish merge the cluster partials and write the output --
-// no second launch.
-//
-// Per tile (32 tokens), with the G query heads that share the kv head:
-//   q.K^T  : integer tensor-core MMA (mma.sync m16n8k32, u8 x s8 -> s32).
-//            A = the packed K codes, masked in registers to one code class
-//            per byte (a byte then reads code * 2^(b j), exact), B = q in
-//            16-bit fixed point per head split into two s8 terms
-//            (q_int = 256 q1 + q2, one column each).  One MMA per 32-channel
-//            K group, so the group's fp16 scale and bf16 zero factor out of
-//            the exact integer sum (InnerQ grouping):
-//              score = sum_grp s_grp * sum_d q_d c_d + z_grp * sum_d q_d.
-//   softmax: online, base 2, running max per head; P in 16-bit fixed point
-//            relative to the running max, split into two u8 terms.
-//   P.V    : MMA (u8 x u8 -> s32) with A = V codes (channel x token), B = P;
-//            the V scale/zero are per channel for the whole tile:
-//              o_d += s_d * sum_t p_t c_td + z_d * sum_t p_t,
-//            where sum_t p_t comes from the same MMA with A = 1.
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-
-#include <cooperative_groups.h>
-
-#include <cfloat>
-#include <map>
+// Decode dispatchers: shared-memory sizing, the (head_dim, GQA group)
+// dispatch of launches and occupancy queries, and the device scratch array
+// of rq_decode_attention_noalloc.  The kernel itself is in rq_decode.cuh.
 #include <mutex>
-#include <tuple>
 
-#include "rq_device.cuh"
-#include "rq_internal.h"
-#include "rq_pack.cuh"
+#include "rq_decode.cuh"
 
 namespace rq {
-namespace {
-
-constexpr int NW = kDecodeConsumerWarps;
-constexpr int kMaxStages = 8;                // per-warp ring depth limit
-constexpr uint32_t kBiasBits = 0x4B400000u;  // bits of 1.5 * 2^23
-constexpr float kBias = 12582912.0f;         // 1.5 * 2^23
-constexpr float kPScale = 65535.0f;          // P in 16-bit fixed point: p_int = rint(p * 65535)
-constexpr float kQMax = 32639.0f;            // q_int in [-32639, 32639] = 256 * q1 + q2, q1, q2 in s8
-
-template <int D, int G>
-struct Cfg {
-  static constexpr int NG = D / 32;                  // K groups per token (one k32 MMA each)
-  static constexpr int NB = (G + 3) / 4;             // 8-column blocks: 4 heads x 2 terms
-  static constexpr int HB = G < 4 ? G : 4;           // heads per block
-  static constexpr int PART = G * D + 2 * G;         // floats per partial state
-  static constexpr int KMW = NG;                     // K meta words converted per lane
-  static constexpr int VMW = D / 32;                 // V meta words converted per lane
-  static constexpr int KSTR = NG * 8 + 4;            // floats per gid row of the K scale scratch
-  static constexpr int VSTR = (D / 8) * 2 + 4;       // floats per gid row of the V scale scratch
-  static constexpr int SCRATCH = 8 * (KSTR + VSTR);  // floats per warp
-};
-
-// Per-warp state.  Thread (gid, tig) owns, in block nb, head 4nb + tig of the
-// MMA results (columns 2 tig, 2 tig + 1 = the two terms of that head).
-template <int D, int G>
-struct WarpState {
-  using C = Cfg<D, G>;
-  uint32_t qb[C::NB][C::NG][2];  // q B-fragments: column n = 2 h + term, bytes = s8 terms
-  float qz[C::NB][C::NG];        // sum of q_int over group g -- zero-point term
-  float xs[C::NB];               // sq * softmax scale * log2(e)
-  float m[C::NB], l[C::NB];      // running max (log2 units) and sum of p (x 65535)
-  float o[C::NB][D / 16][2];     // channel 16 mb + 8 rh + gid (x 65535)
-  float kf[C::KMW], vf[C::VMW];  // class factors 2^(-b j) of the meta words this lane converts
-};
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
-
-// q of the G heads -> per-head 16-bit fixed point (sq = max|q_h| / 32639)
-// split into two s8 terms q_int = 256 q1 + q2, laid out as the k32 x n8
-// B-fragments of the q.K^T MMA (column n = 2 * head + term).
-template <int D, int G, int KB, int VB>
-__device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, const float* nrm, float scale_log2, int lane) {
-  using C = Cfg<D, G>;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int hl = gid >> 1, tau = gid & 1;
-#pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb) {
-    const bool hv = hl < C::HB;
-    const uint16_t* qp = qh + (size_t)(4 * nb + hl) * D;
-    float qv[C::NG][8];
-    float mx = 0.0f, ps[C::NG];
-#pragma unroll
-    for (int g = 0; g < C::NG; ++g) {
-      ps[g] = 0.0f;
-#pragma unroll
-      for (int kh = 0; kh < 2; ++kh) {
-        uint2 u = make_uint2(0u, 0u);
-        if (hv) u = __ldg(reinterpret_cast<const uint2*>(qp + 32 * g + 16 * kh + 4 * tig));
-        const uint32_t w[2] = {u.x, u.y};
-        // K normalization folded into q for the packed tiles: q_d * n_d (exact, powers of two)
-        const float4 nv = *reinterpret_cast<const float4*>(nrm + 32 * g + 16 * kh + 4 * tig);
-        const float nn[4] = {nv.x, nv.y, nv.z, nv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x = bf16_bits_to_float(e & 1 ? w[e >> 1] >> 16 : w[e >> 1] & 0xFFFFu) * nn[e];
-          qv[g][4 * kh + e] = x;
-          mx = fmaxf(mx, fabsf(x));
-        }
-      }
-    }
-    // the four lanes of a quad hold all D channels of one head
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float inv = mx > 0.0f ? kQMax / mx : 0.0f;
-    const float sq = mx * (1.0f / kQMax);
-#pragma unroll
-    for (int g = 0; g < C::NG; ++g)
-#pragma unroll
-      for (int kh = 0; kh < 2; ++kh) {
-        uint32_t packed = 0u;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          int qi = __float2int_rn(qv[g][4 * kh + e] * inv);
-          qi = qi > 32639 ? 32639 : (qi < -32639 ? -32639 : qi);
-          const int q1 = (qi + 128) >> 8;  // floor((qi + 128) / 256)
-          const int q2 = qi - (q1 << 8);   // in [-128, 127]
-          packed |= ((uint32_t)(tau ? q2 : q1) & 0xFFu) << (8 * e);
-          ps[g] += (float)qi;
-        }
-        st.qb[nb][g][kh] = hv ? packed : 0u;
-      }
-    // zero-point term: sum of the SAME rounded q_int over each group, so the
-    // code and zero terms together are exactly (s c + z) . q_int and the large
-    // cancellation between them (z = group minimum) leaves no rounding residue
-#pragma unroll
-    for (int g = 0; g < C::NG; ++g) {
-      ps[g] += __shfl_xor_sync(0xffffffffu, ps[g], 1);
-      ps[g] += __shfl_xor_sync(0xffffffffu, ps[g], 2);
-    }
-    // the result columns of thread (gid, tig) belong to head 4nb + tig, whose
-    // statistics live in lane 8 tig (gid = 2 tig, term 0)
-    const float sq_c = __shfl_sync(0xffffffffu, sq, 8 * tig);
-#pragma unroll
-    for (int g = 0; g < C::NG; ++g) st.qz[nb][g] = __shfl_sync(0xffffffffu, ps[g], 8 * tig);
-    st.xs[nb] = sq_c * scale_log2;
-    st.m[nb] = -INFINITY;
-    st.l[nb] = 0.0f;
-#pragma unroll
-    for (int mb = 0; mb < D / 16; ++mb) st.o[nb][mb][0] = st.o[nb][mb][1] = 0.0f;
-  }
-  // class factors of the metadata words this lane converts (see convert_meta)
-#pragma unroll
-  for (int k = 0; k < C::KMW; ++k) {
-    const int w = C::KMW * lane + k, g = w / 32, i = (w % 32) % 4;
-    st.kf[k] = pow2i(-KB * reg_class(KB, i * C::NG + g));
-  }
-#pragma unroll
-  for (int k = 0; k < C::VMW; ++k) {
-    const int w = C::VMW * lane + k, rho = w % (D / 8);
-    st.vf[k] = pow2i(-VB * reg_class(VB, rho));
-  }
-}
-
-template <int W>
-__device__ __forceinline__ void load_words(uint32_t (&w)[W], const uint8_t* blob, int lane) {
-#pragma unroll
-  for (int c = 0; c < W / 4; ++c) {
-    const uint4 u = *reinterpret_cast<const uint4*>(blob + word_offset(W, lane, 4 * c));
-    w[4 * c] = u.x;
-    w[4 * c + 1] = u.y;
-    w[4 * c + 2] = u.z;
-    w[4 * c + 3] = u.w;
-  }
-#pragma unroll
-  for (int k = 4 * (W / 4); k < W; ++k) w[k] = *reinterpret_cast<const uint32_t*>(blob + word_offset(W, lane, k));
-}
-
-__device__ __forceinline__ float half_lo_to_float(uint32_t m) {
-  return __half2float(__ushort_as_half((unsigned short)(m & 0xFFFFu)));
-}
-
-// Metadata of one tile -> (scale * 2^(-b j), zero) float pairs in the warp's
-// scratch, each entry converted once.  K: scratch[gid][g][i] for token
-// gid + 8 i; V: scratch[gid][rho] for channel 16 (rho/2) + 8 (rho%2) + gid.
-template <int D, int G, int KB, int VB>
-__device__ __forceinline__ void convert_meta(const uint8_t* rec, const WarpState<D, G>& st, float* ks, float* vs,
-                                             int lane) {
-  using C = Cfg<D, G>;
-  const uint32_t* kmeta = reinterpret_cast<const uint32_t*>(rec + blob_bytes(KB, D));
-  const uint32_t* vmeta = reinterpret_cast<const uint32_t*>(rec + blob_bytes(KB, D) + 4 * D + blob_bytes(VB, D));
-  uint32_t km[C::KMW], vm[C::VMW];
-  if constexpr (C::KMW == 4) {
-    const uint4 u = *reinterpret_cast<const uint4*>(kmeta + 4 * lane);
-    km[0] = u.x, km[1] = u.y, km[2] = u.z, km[3] = u.w;
-  } else {
-    const uint2 u = *reinterpret_cast<const uint2*>(kmeta + 2 * lane);
-    km[0] = u.x, km[1] = u.y;
-  }
-  if constexpr (C::VMW == 4) {
-    const uint4 u = *reinterpret_cast<const uint4*>(vmeta + 4 * lane);
-    vm[0] = u.x, vm[1] = u.y, vm[2] = u.z, vm[3] = u.w;
-  } else {
-    const uint2 u = *reinterpret_cast<const uint2*>(vmeta + 2 * lane);
-    vm[0] = u.x, vm[1] = u.y;
-  }
-  float kv[2 * C::KMW], vv[2 * C::VMW];
-#pragma unroll
-  for (int k = 0; k < C::KMW; ++k) {
-    kv[2 * k] = half_lo_to_float(km[k]) * st.kf[k];
-    kv[2 * k + 1] = __uint_as_float(km[k] & 0xFFFF0000u);
-  }
-#pragma unroll
-  for (int k = 0; k < C::VMW; ++k) {
-    vv[2 * k] = half_lo_to_float(vm[k]) * st.vf[k];
-    vv[2 * k + 1] = __uint_as_float(vm[k] & 0xFFFF0000u);
-  }
-  // word w = KMW * lane + k: group w / 32, gid (w % 32) / 4, i = w % 4
-  {
-    const int w0 = C::KMW * lane;
-    float* dst = ks + ((w0 % 32) / 4) * C::KSTR + ((w0 / 32) * 4 + (w0 % 4)) * 2;
-#pragma unroll
-    for (int c = 0; c < C::KMW / 2; ++c)
-      *reinterpret_cast<float4*>(dst + 4 * c) = make_float4(kv[4 * c], kv[4 * c + 1], kv[4 * c + 2], kv[4 * c + 3]);
-  }
-  // word w = VMW * lane + k: gid w / (D/8), rho = w % (D/8)
-  {
-    const int w0 = C::VMW * lane;
-    float* dst = vs + (w0 / (D / 8)) * C::VSTR + (w0 % (D / 8)) * 2;
-#pragma unroll
-    for (int c = 0; c < C::VMW / 2; ++c)
-      *reinterpret_cast<float4*>(dst + 4 * c) = make_float4(vv[4 * c], vv[4 * c + 1], vv[4 * c + 2], vv[4 * c + 3]);
-  }
-}
-
-// q.K^T of one tile: raw scores acc[nb][i] (units sq, without the softmax
-// scale) for token gid + 8 i and head 4 nb + tig.  One k32 MMA per (token
-// half, group); its two term columns combine exactly in int32, and the
-// group's scale/zero apply to that exact integer sum.
-template <int D, int G, int KB>
-__device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G>& st, const float* ks,
-                                        float (&acc)[Cfg<D, G>::NB][4], int lane) {
-  using C = Cfg<D, G>;
-  constexpr int W = words_per_lane(KB, D);
-  const int gid = lane >> 2;
-  uint32_t kw[W];
-  load_words<W>(kw, rec, lane);
-#pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[nb][i] = 0.0f;
-#pragma unroll
-  for (int g = 0; g < C::NG; ++g)
-#pragma unroll
-    for (int mb = 0; mb < 2; ++mb) {
-      const float4 sz = *reinterpret_cast<const float4*>(ks + gid * C::KSTR + (g * 4 + 2 * mb) * 2);
-      uint32_t a[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) a[r] = code_reg<KB, W>(kw, (2 * mb + (r & 1)) * C::NG + g, r >> 1);
-#pragma unroll
-      for (int nb = 0; nb < C::NB; ++nb) {
-        uint32_t c[4];
-        imma_u8s8(c, a, st.qb[nb][g][0], st.qb[nb][g][1], 0u);
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-          // |256 hi + lo| < 2^31: exact in int32, one rounding to fp32
-          const float v = (float)((int)c[2 * rh] * 256 + (int)c[2 * rh + 1]);
-          const float s = rh ? sz.z : sz.x, z = rh ? sz.w : sz.y;
-          acc[nb][2 * mb + rh] = fmaf(s, v, fmaf(z, st.qz[nb][g], acc[nb][2 * mb + rh]));
-        }
-      }
-    }
-}
-
-// Online softmax of one tile.  The probabilities are taken relative to the
-// running maximum m (p <= 1, 16-bit fixed point p_int = rint(65535 p)); m
-// moves -- and the state is rescaled -- only when a score of the tile exceeds
-// it, which after the first tiles is rare.  Returns the P B-fragments pb
-// (column n = 2 * head + term, term 0 = high byte).
-template <int D, int G>
-__device__ __forceinline__ void softmax_tile(WarpState<D, G>& st, const float (&acc)[Cfg<D, G>::NB][4],
-                                             uint32_t (&pb)[Cfg<D, G>::NB][2], int lane) {
-  using C = Cfg<D, G>;
-  const int gid = lane >> 2, tig = lane & 3;
-  float x[C::NB][4];
-  bool grow = false;
-#pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[nb][i] = acc[nb][i] * st.xs[nb];
-    grow |= fmaxf(fmaxf(x[nb][0], x[nb][1]), fmaxf(x[nb][2], x[nb][3])) > st.m[nb];
-  }
-  if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb) {
-      float v = fmaxf(fmaxf(x[nb][0], x[nb][1]), fmaxf(x[nb][2], x[nb][3]));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      const float mn = fmaxf(st.m[nb], v);
-      const float alpha = ex2(st.m[nb] - mn);  // 0 while m = -inf
-      st.m[nb] = mn;
-      st.l[nb] *= alpha;
-#pragma unroll
-      for (int mb = 0; mb < D / 16; ++mb) {
-        st.o[nb][mb][0] *= alpha;
-        st.o[nb][mb][1] *= alpha;
-      }
-    }
-  }
-  const int hl = gid >> 1;
-  const int src0 = 4 * tig + hl, src1 = 16 + 4 * tig + hl;
-#pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb) {
-    uint32_t y[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) y[i] = __float_as_uint(fmaf(ex2(x[nb][i] - st.m[nb]), kPScale, kBias));
-    // low 16 bits of y = p_int; byte e of hi/lo = token gid + 8e
-    const uint32_t u0 = __byte_perm(y[0], y[1], 0x5410), u1 = __byte_perm(y[2], y[3], 0x5410);
-    const uint32_t hi = __byte_perm(u0, u1, 0x7531), lo = __byte_perm(u0, u1, 0x6420);
-    // B element (k, n = gid): token 4 (k >> 4) + ((k >> 2) & 3) + 8 (k & 3),
-    // held by lane 4 * gid_src + head with gid_src = tig (k < 16) or tig + 4
-    const uint32_t h0 = __shfl_sync(0xffffffffu, hi, src0), l0 = __shfl_sync(0xffffffffu, lo, src0);
-    const uint32_t h1 = __shfl_sync(0xffffffffu, hi, src1), l1 = __shfl_sync(0xffffffffu, lo, src1);
-    const bool hv = hl < C::HB;
-    pb[nb][0] = hv ? ((gid & 1) ? l0 : h0) : 0u;
-    pb[nb][1] = hv ? ((gid & 1) ? l1 : h1) : 0u;
-  }
-}
-
-// P.V of one tile into the running state.  One k32 MMA per 16 channels; the
-// channel's scale/zero apply to the exact integer sum, and the zero term
-// needs sum_t p_t, which one more MMA with A = 1 delivers in the same layout.
-template <int D, int G, int VB>
-__device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st, const float* vs,
-                                        const uint32_t (&pb)[Cfg<D, G>::NB][2], int lane) {
-  using C = Cfg<D, G>;
-  constexpr int W = words_per_lane(VB, D);
-  const int gid = lane >> 2;
-  float ps[C::NB];
-  const uint32_t ones[4] = {0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u};
-#pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb) {
-    uint32_t c[4];
-    imma_u8u8(c, ones, pb[nb][0], pb[nb][1], kBiasBits);
-    ps[nb] = fmaf(256.0f, __uint_as_float(c[0]) - kBias, __uint_as_float(c[1]) - kBias);
-    st.l[nb] += ps[nb];
-  }
-  uint32_t vw[W];
-  load_words<W>(vw, vrec, lane);
-#pragma unroll
-  for (int mb = 0; mb < D / 16; ++mb) {
-    const float4 sz = *reinterpret_cast<const float4*>(vs + gid * C::VSTR + 4 * mb);
-    uint32_t a[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) a[r] = code_reg<VB, W>(vw, 2 * mb + (r & 1), r >> 1);
-#pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb) {
-      uint32_t c[4];
-      imma_u8u8(c, a, pb[nb][0], pb[nb][1], 0u);
-#pragma unroll
-      for (int rh = 0; rh < 2; ++rh) {
-        const float v = (float)((int)c[2 * rh] * 256 + (int)c[2 * rh + 1]);
-        const float s = rh ? sz.z : sz.x, z = rh ? sz.w : sz.y;
-        st.o[nb][mb][rh] = fmaf(s, v, fmaf(z, ps[nb], st.o[nb][mb][rh]));
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
-  *abort_flag = 1;
-  atomicCAS(status, 0, kDeviceTimeout);
-}
-
-// Consumer warp w owns tiles w, w + NW, w + 2 NW, ... of the CTA's range and a
-// private ring of `stages` shared-memory slots.  Lane 0 streams the warp's
-// own tile records into the ring with 1-D bulk copies (TMA) and re-arms a
-// slot as soon as the warp has read it, so the warp never waits on another
-// warp and every warp keeps `stages` records in flight.
-template <int D, int G, int KB, int VB>
-__device__ void consume(WarpState<D, G>& st, const uint16_t* qh, const float* nrm, float scale_log2, uint8_t* ring,
-                        int stages,
-                        int stage_bytes, uint64_t* bars, float* scratch, const uint8_t* src, int rec, int n_my,
-                        int warp, int lane, volatile int* abort_flag, int* status) {
-  using C = Cfg<D, G>;
-  const int n_w = n_my > warp ? (n_my - warp + NW - 1) / NW : 0;
-  // Packed tiles are written only by kernels that complete before a decode
-  // launch may start (prefill, tile flush), never by the decode launch this
-  // one may overlap, so the first records can be fetched before waiting on
-  // it; the query, the window and the workspace are read after the wait.
-  const uint64_t policy = l2_evict_first_policy();  // tile records are read once per launch
-  if (lane == 0) {
-    for (int j = 0; j < stages && j < n_w; ++j) {
-      mbar_arrive_expect_tx(&bars[j], (uint32_t)rec);
-      bulk_g2s_hint(ring + (size_t)j * stage_bytes, src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec, &bars[j],
-                    policy);
-    }
-  }
-  griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
-  setup_query<D, G, KB, VB>(st, qh, nrm, scale_log2, lane);
-  float* ks = scratch;
-  float* vs = scratch + 8 * C::KSTR;
-  const int VOFF = blob_bytes(KB, D) + 4 * D;
-  int j = 0, slot = 0, parity = 0;  // ring position of tile j, advanced without division
-  uint8_t* cur = ring;               // slot address of tile j
-  const uint8_t* nsrc = src + (int64_t)(warp + stages * NW) * rec;  // record of tile j + stages
-  bool ok = true;
-  for (; j < n_w; ++j) {
-    ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], (uint32_t)parity));
-    if (!ok) break;
-    convert_meta<D, G, KB, VB>(cur, st, ks, vs, lane);
-    __syncwarp();
-    float acc[C::NB][4];
-    qk_tile<D, G, KB>(cur, st, ks, acc, lane);
-    uint32_t pb[C::NB][2];
-    softmax_tile<D, G>(st, acc, pb, lane);
-    pv_tile<D, G, VB>(cur + VOFF, st, vs, pb, lane);
-    __syncwarp();  // every lane has finished reading the slot and the scratch
-    if (lane == 0 && j + stages < n_w) {
-      fence_proxy_async_smem();  // generic-proxy reads of the slot precede the async refill
-      mbar_arrive_expect_tx(&bars[slot], (uint32_t)rec);
-      bulk_g2s_hint(cur, nsrc, (uint32_t)rec, &bars[slot], policy);
-    }
-    nsrc += (int64_t)NW * rec;
-    cur += stage_bytes;
-    if (++slot == stages) {
-      slot = 0;
-      parity ^= 1;
-      cur = ring;
-    }
-    if ((j & 3) == 3 && *abort_flag) {  // another warp gave up: stop within four tiles
-      ok = false;
-      break;
-    }
-  }
-  if (!ok) {
-    if (lane == 0) {
-      raise_abort(abort_flag, status);
-      // let the copies in flight land before the CTA exits
-      for (int k = j; k < n_w && k < j + stages; ++k) (void)mbar_wait_bounded(&bars[k % stages], (k / stages) & 1);
-    }
-  }
-}
-
-template <int D, int G>
-__device__ __forceinline__ void consume_dispatch(int kb, int vb, WarpState<D, G>& st, const uint16_t* qh,
-                                                 const float* nrm, float scale_log2, uint8_t* ring, int stages, int stage_bytes,
-                                                 uint64_t* bars, float* scratch, const uint8_t* src, int rec,
-                                                 int n_my, int warp, int lane, volatile int* abort_flag,
-                                                 int* status) {
-#define RQ_C(KBV, VBV)                                                                                       \
-  consume<D, G, KBV, VBV>(st, qh, nrm, scale_log2, ring, stages, stage_bytes, bars, scratch, src, rec, n_my, warp, \
-                          lane, abort_flag, status)
-#define RQ_V(KBV)                  \
-  switch (vb) {                    \
-    case 2: RQ_C(KBV, 2); break;   \
-    case 3: RQ_C(KBV, 3); break;   \
-    case 4: RQ_C(KBV, 4); break;   \
-    default: RQ_C(KBV, 8); break;  \
-  }
-  switch (kb) {
-    case 2: RQ_V(2) break;
-    case 3: RQ_V(3) break;
-    case 4: RQ_V(4) break;
-    default: RQ_V(8) break;
-  }
-#undef RQ_V
-#undef RQ_C
-}
-
-// Canonical partial of one warp in shared memory: o[G][D], m[G], l[G], with
-// o and l back in units of p (the tile path keeps them x 65535).
-template <int D, int G>
-__device__ void dump_tile_state(const WarpState<D, G>& st, float* slot, int lane) {
-  using C = Cfg<D, G>;
-  const int gid = lane >> 2, tig = lane & 3;
-  constexpr float inv = 1.0f / kPScale;
-#pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb) {
-    const int h = 4 * nb + tig;
-    if (tig < C::HB) {
-#pragma unroll
-      for (int mb = 0; mb < D / 16; ++mb)
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh) slot[h * D + 16 * mb + 8 * rh + gid] = st.o[nb][mb][rh] * inv;
-      if (gid == 0) {
-        slot[G * D + h] = st.m[nb];
-        slot[G * D + G + h] = st.l[nb] * inv;
-      }
-    }
-  }
-}
-
-// bf16 sink + recent window on CUDA cores.  The window is split into chunks
-// of 32 tokens, kWinChunksPerItem consecutive chunks per work item.  For each
-// chunk thread 0 stages its K and V rows in shared memory with at most six
-// 1-D bulk copies (the rows of a chunk form at most three contiguous runs:
-// sink, ring, ring after wrap); warp w then takes heads w, w + 4, ...:
-// lane = token for q.k (K row words read in a lane-rotated order so the 32
-// rows hit 32 banks), lane = channel for p.v, and merges the chunk into its
-// running (m, l, o).
-constexpr int kWinChunk = 32;
-
-__host__ __device__ inline int window_tokens(int T, int S, int Tq) { return (T < S ? T : S) + (T - (T < S ? T : S) - Tq); }
-
-template <int D>
-__device__ __forceinline__ void window_issue_chunk(const DecodeArgs& a, const uint8_t* win, uint32_t* kbuf,
-                                                   uint32_t* vbuf, uint64_t* bar, int j0, int cnt,
-                                                   const uint16_t* knew, const uint16_t* vnew) {
-  const int S = a.g.S, ring = a.g.R + kTile;
-  const int n_sink = a.T < S ? a.T : S;
-  mbar_arrive_expect_tx(bar, (uint32_t)(cnt * D * 2 * 2));
-  // appended in the same call: the newest token comes from the caller's rows
-  const int n_cache = knew ? cnt - 1 : cnt;
-  if (knew) {
-    bulk_g2s(kbuf + (size_t)n_cache * (D / 2), knew, (uint32_t)(D * 2), bar);
-    bulk_g2s(vbuf + (size_t)n_cache * (D / 2), vnew, (uint32_t)(D * 2), bar);
-  }
-  int t = 0;
-  while (t < n_cache) {
-    const int j = j0 + t;
-    size_t row;  // K row inside the window block; its V row follows its block's K rows
-    int run;
-    size_t v_off;
-    if (j < n_sink) {
-      row = j;
-      run = min(n_cache - t, n_sink - j);
-      v_off = S;
-    } else {
-      const int slot = (a.Tq + (j - n_sink)) % ring;
-      row = (size_t)2 * S + slot;
-      run = min(n_cache - t, ring - slot);
-      v_off = ring;
-    }
-    bulk_g2s(kbuf + (size_t)t * (D / 2), win + row * D * 2, (uint32_t)(run * D * 2), bar);
-    bulk_g2s(vbuf + (size_t)t * (D / 2), win + (row + v_off) * D * 2, (uint32_t)(run * D * 2), bar);
-    t += run;
-  }
-}
-
-template <int D, int G>
-__device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* qh, size_t knew_off, int witem,
-                            float* scratch, uint64_t* bar, float* slot, int warp, int lane,
-                            volatile int* abort_flag) {
-  constexpr int RW = D / 2;  // words per bf16 row
-  constexpr int HW = (G + NW - 1) / NW;
-  const int tid = warp * 32 + lane;
-  const int n_tok = window_tokens(a.T, a.g.S, a.Tq);
-  const int n_chunks = (n_tok + kWinChunk - 1) / kWinChunk;
-  const int c0 = witem * kWinChunksPerItem;
-  const int c1 = min(c0 + kWinChunksPerItem, n_chunks);
-  float* qs = scratch;                                              // [G][D]
-  uint32_t* kbuf = reinterpret_cast<uint32_t*>(qs + G * D);         // [32][RW]
-  uint32_t* vbuf = kbuf + kWinChunk * RW;                           // [32][RW]
-  for (int i = tid; i < G * D; i += NW * 32) qs[i] = bf16_bits_to_float(qh[i]);
-  // running state of this warp's heads over the item's chunks
-  float m[HW], l[HW], o[HW][D / 32];
-#pragma unroll
-  for (int jh = 0; jh < HW; ++jh) {
-    m[jh] = -INFINITY;
-    l[jh] = 0.0f;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) o[jh][c] = 0.0f;
-  }
-  int parity = 0;
-  for (int ch = c0; ch < c1; ++ch, parity ^= 1) {
-    const int j0 = ch * kWinChunk;
-    const int cnt = min(kWinChunk, n_tok - j0);
-    // a fused append delivers the newest token (window index n_tok - 1) itself
-    const bool newest = a.k_new != nullptr && j0 + cnt == n_tok;
-    if (ch > c0) {
-      __syncthreads();  // every thread has finished reading the previous chunk
-      if (tid == 0) fence_proxy_async_smem();
-    }
-    if (tid == 0)
-      window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt, newest ? a.k_new + knew_off : nullptr,
-                            newest ? a.v_new + knew_off : nullptr);
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, (uint32_t)parity));
-    if (!__syncthreads_and(ok)) {
-      if (tid == 0) {
-        raise_abort(abort_flag, a.status);
-        (void)mbar_wait_bounded(bar, (uint32_t)parity);  // let the copies land before the CTA exits
-      }
-      return;
-    }
-    if (newest && tid < 2 * (D / 8)) {
-      // the appended token enters the cache (sink row, or its ring slot) for
-      // later calls; no other work item of this call reads that row
-      const int S = a.g.S, ring = a.g.R + kTile;
-      const int n_sink = a.T < S ? a.T : S;
-      const int j = n_tok - 1;
-      size_t krow, vrow;
-      if (j < n_sink) {
-        krow = j;
-        vrow = (size_t)S + j;
-      } else {
-        const int rs = (a.Tq + (j - n_sink)) % ring;
-        krow = (size_t)2 * S + rs;
-        vrow = (size_t)2 * S + ring + rs;
-      }
-      const int c = tid % (D / 8);
-      const bool isv = tid >= D / 8;
-      const uint4 x = reinterpret_cast<const uint4*>((isv ? vbuf : kbuf) + (size_t)(cnt - 1) * RW)[c];
-      reinterpret_cast<uint4*>(win + (isv ? vrow : krow) * D * 2)[c] = x;
-    }
-#pragma unroll
-    for (int jh = 0; jh < HW; ++jh) {
-      const int h = warp + NW * jh;
-      if (h >= G) continue;
-      float acc = 0.0f;
-      if (lane < cnt) {
-#pragma unroll 8
-        for (int w = 0; w < RW; ++w) {
-          const int wr = (w + lane) & (RW - 1);
-          const uint32_t kk = kbuf[lane * RW + wr];
-          acc = fmaf(qs[h * D + 2 * wr], bf16_bits_to_float(kk & 0xFFFFu),
-                     fmaf(qs[h * D + 2 * wr + 1], bf16_bits_to_float(kk >> 16), acc));
-        }
-      }
-      const float x = lane < cnt ? acc * a.scale_log2 : -INFINITY;
-      const float mc = warp_max(x);
-      const float mn = fmaxf(m[jh], mc);
-      const float a_old = ex2(m[jh] - mn);  // 0 while m = -inf
-      const float p = ex2(x - mn);
-      l[jh] = l[jh] * a_old + warp_sum(p);
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) o[jh][c] *= a_old;
-      for (int t = 0; t < cnt; ++t) {
-        const float pt = __shfl_sync(0xffffffffu, p, t);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const int d = lane + 32 * c;
-          const uint32_t vv = vbuf[t * RW + d / 2];
-          o[jh][c] = fmaf(pt, (d & 1) ? bf16_bits_to_float(vv >> 16) : bf16_bits_to_float(vv & 0xFFFFu), o[jh][c]);
-        }
-      }
-      m[jh] = mn;
-    }
-  }
-#pragma unroll
-  for (int jh = 0; jh < HW; ++jh) {
-    const int h = warp + NW * jh;
-    if (h < G) {
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) slot[h * D + lane + 32 * c] = o[jh][c];
-      if (lane == 0) {
-        slot[G * D + h] = m[jh];
-        slot[G * D + G + h] = l[jh];
-      }
-    }
-  }
-  // heads of the other warps: empty partial states
-  for (int h = 0; h < G; ++h) {
-    if (h % NW == warp) continue;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) slot[h * D + lane + 32 * c] = 0.0f;
-    if (lane == 0) {
-      slot[G * D + h] = -INFINITY;
-      slot[G * D + G + h] = 0.0f;
-    }
-  }
-}
-
-// Pack-ahead item (a fused step whose next append completes a tile): the 32
-// oldest ring tokens -- exactly the tile that append will flush -- are
-// quantized and packed into tile slot a.pack_tile, which no item of this
-// launch reads, so the next step needs no separate flush launch.  The rows
-// it reads are not the one this launch's window item writes (n_recent >= 2).
-// Warp 0 packs K, warp 1 V.  Leaves empty partial states in the warp slots.
-template <int D, int G>
-__device__ void pack_item(const DecodeArgs& a, const HeadDesc& hd, int b, uint8_t* area, float* merge, int tid) {
-  using C = Cfg<D, G>;
-  const int warp = tid >> 5, lane = tid & 31;
-  TileSmem<D>& sm = *reinterpret_cast<TileSmem<D>*>(area);
-  uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
-  const int S = a.g.S, ring = a.g.R + kTile;
-  griddep_wait();
-  if (warp == 0) stage_kinv<D>(sm.kinv, stream_norm(a.buf, hd, a.g, b), lane);
-  constexpr int kChunks = D / 8;
-  for (int j = tid; j < kTile * kChunks; j += blockDim.x) {
-    const int t = j / kChunks, c = j % kChunks;
-    const int slot = (a.pack_pos + t - S) % ring;
-    const uint4* krow = reinterpret_cast<const uint4*>(win + ((size_t)2 * S + slot) * D * 2);
-    const uint4* vrow = reinterpret_cast<const uint4*>(win + ((size_t)2 * S + ring + slot) * D * 2);
-    *reinterpret_cast<uint4*>(&sm.k.x[t][c * 4]) = __ldg(krow + c);
-    *reinterpret_cast<uint4*>(&sm.v.x[t][c * 4]) = __ldg(vrow + c);
-  }
-  __syncthreads();
-  uint8_t* rec = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)a.pack_tile * hd.rec_bytes;
-  if (warp == 0) {
-    pack_k_dispatch<D, true>(sm.k, sm.kinv, hd.k_bits, rec, lane);
-  } else if (warp == 1) {
-    pack_v_dispatch<D>(sm.v, hd.v_bits, rec + blob_bytes(hd.k_bits, D) + 4 * D, lane);
-  }
-  __syncthreads();  // the staged tile is dead; its memory becomes the warp slots
-  float* slot = merge + warp * C::PART;
-  for (int i = lane; i < G * D; i += 32) slot[i] = 0.0f;
-  if (lane < G) {
-    slot[G * D + lane] = -INFINITY;
-    slot[G * D + G + lane] = 0.0f;
-  }
-}
-
-// Final log-sum-exp merge of n partial states (o[G][D], m[G], l[G] each,
-// stride PART floats) into the normalised output, for the slice of outputs
-// owned by cluster rank `part` (of CL): one output per thread, all of its loads for
-// up to 24 partials in flight at once (a stream of the long-context cache has
-// 17 cluster partials, so one round trip to L2 covers them).
-template <int D, int G, int CL>
-__device__ void merge_outputs(const float* base, int n, float* outp, int part, int tid) {
-  using C = Cfg<D, G>;
-  constexpr int PER = (G * D + CL - 1) / CL;  // outputs of one CTA
-  constexpr int U = 24;
-  for (int idx = part * PER + tid; idx < (part + 1) * PER && idx < G * D; idx += kDecodeThreads) {
-    const int hh = idx / D;
-    float M = -INFINITY, O = 0.0f, L = 0.0f;
-    for (int i0 = 0; i0 < n; i0 += U) {
-      float ov[U], mv[U], lv[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const bool ok = i0 + u < n;
-        const float* pp = base + (size_t)(i0 + u) * C::PART;
-        ov[u] = ok ? __ldcg(pp + idx) : 0.0f;
-        mv[u] = ok ? __ldcg(pp + G * D + hh) : -INFINITY;
-        lv[u] = ok ? __ldcg(pp + G * D + G + hh) : 0.0f;
-      }
-      float nm = M;
-#pragma unroll
-      for (int u = 0; u < U; ++u) nm = fmaxf(nm, mv[u]);
-      if (nm == -INFINITY) continue;
-      const float sc = ex2(M - nm);  // 0 while M = -inf
-      O *= sc;
-      L *= sc;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const float f = ex2(mv[u] - nm);
-        O = fmaf(ov[u], f, O);
-        L = fmaf(lv[u], f, L);
-      }
-      M = nm;
-    }
-    outp[idx] = L > 0.0f ? O / L : 0.0f;
-  }
-}
-
-// CL = CTAs per thread-block cluster (kDecodeCluster, or 1: no cluster); the
-// cluster shape is given at launch.
-template <int D, int G, int CL>
-__global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_kernel(DecodeArgs a) {
-  using C = Cfg<D, G>;
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ uint64_t bars[NW * kMaxStages];
-  __shared__ volatile int abort_flag;
-  __shared__ int is_last;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int srel = blockIdx.y, item = blockIdx.x;
-  const int NI = a.n_splits + a.n_win + a.n_pack;  // work items of this stream
-  const int h = srel % a.g.Hkv, b = (srel / a.g.Hkv) % a.g.B, lrel = srel / (a.g.Hkv * a.g.B);
-  const int l = a.layer0 + lrel;
-  const HeadDesc hd = a.desc[l * a.g.Hkv + h];
-  const uint16_t* qh = a.q + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  // dynamic shared memory: [per-warp scale scratch][stages | merge + window]
-  uint8_t* area = smem + (size_t)NW * C::SCRATCH * 4;
-  float* merge = reinterpret_cast<float*>(area);  // aliases the stages after the main loop
-
-  // programmatic dependent launch: the next kernel of the stream may be
-  // scheduled now; it waits below for this grid's memory before reading any
-  // input, so only its launch and prologue overlap our tail
-  griddep_launch_dependents();
-  if (tid == 0) {
-    abort_flag = 0;
-    for (int s = 0; s < NW * kMaxStages; ++s) mbar_init(&bars[s], 1);
-    mbar_fence_init();
-  }
-  __syncthreads();
-
-  WarpState<D, G> st;
-  const bool tiles_item = item < a.n_splits;
-  if (tiles_item) {
-    const int t0 = (int)(((int64_t)item * a.n_tiles) / a.n_splits);
-    const int t1 = (int)(((int64_t)(item + 1) * a.n_tiles) / a.n_splits);
-    const int rec = hd.rec_bytes;
-    const uint8_t* src = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)t0 * rec;
-    if (warp < NW)
-      consume_dispatch<D, G>(hd.k_bits, hd.v_bits, st, qh,
-                             reinterpret_cast<const float*>(a.buf + hd.win_base + (int64_t)b * a.g.win_bytes +
-                                                            window_rows_bytes(a.g.S, a.g.R, D)),
-                             a.scale_log2,
-                             area + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
-                             bars + warp * kMaxStages, reinterpret_cast<float*>(smem) + warp * C::SCRATCH, src, rec,
-                             t1 - t0, warp, lane, &abort_flag, a.status);
-  } else if (a.n_pack && item == a.n_splits + a.n_win) {
-    pack_item<D, G>(a, hd, b, area, merge, tid);
-  } else {
-    griddep_wait();  // the window rows and the query may come from the previous kernel
-    // 32-token chunks of the bf16 sink + recent window
-    uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
-    const size_t knew_off = ((size_t)(lrel * a.g.B + b) * a.g.Hkv + h) * D;
-    window_item<D, G>(a, win, qh, knew_off, item - a.n_splits, merge + NW * C::PART, &bars[0],
-                      merge + warp * C::PART, warp, lane, &abort_flag);
-  }
-  __syncthreads();  // every stage read has completed; merge may now alias the stages
-  if (tiles_item && warp < NW && !abort_flag) dump_tile_state<D, G>(st, merge + warp * C::PART, lane);
-  __syncthreads();
-  const bool valid = !abort_flag;
-
-  // merge the warps' partial states into this item's partial (shared memory)
-  float* mypart = merge + NW * C::PART;
-  for (int idx = tid; idx < G * D; idx += blockDim.x) {
-    const int hh = idx / D;
-    float M = -INFINITY;
-    if (valid) {
-#pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, merge[w * C::PART + G * D + hh]);
-    }
-    float O = 0.0f, L = 0.0f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const float f = ex2(merge[w * C::PART + G * D + hh] - M);
-        O = fmaf(merge[w * C::PART + idx], f, O);
-        L = fmaf(merge[w * C::PART + G * D + G + hh], f, L);
-      }
-    }
-    mypart[idx] = O;
-    if (idx % D == 0) {
-      mypart[G * D + hh] = M;
-      mypart[G * D + G + hh] = L;
-    }
-  }
-  // Level 1: the CL items of a thread-block cluster (consecutive items of one
-  // stream) are merged by the cluster's first CTA straight from the others'
-  // shared memory (CL = 1: the CTA stores its own partial).  Every CTA passes
-  // both cluster barriers on every path (no early exit before them).
-  namespace cg = cooperative_groups;
-  float* ps = a.partials + (size_t)srel * NI * C::PART;
-  const int ncl = (int)gridDim.x / CL;
-  int crank = 0;
-  if constexpr (CL > 1) {
-    cg::cluster_group cluster = cg::this_cluster();
-    crank = (int)cluster.block_rank();
-    cluster.sync();  // all partials of the cluster are in shared memory
-    if (crank == 0) {
-      const float* rp[CL];
-#pragma unroll
-      for (int r = 0; r < CL; ++r) rp[r] = cluster.map_shared_rank(mypart, r);
-      float* cp = ps + (size_t)(item / CL) * C::PART;
-      for (int idx = tid; idx < G * D; idx += blockDim.x) {
-        const int hh = idx / D;
-        float mv[CL];
-        float M = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < CL; ++r) {
-          mv[r] = rp[r][G * D + hh];
-          M = fmaxf(M, mv[r]);
-        }
-        float O = 0.0f, L = 0.0f;
-        if (M != -INFINITY) {
-#pragma unroll
-          for (int r = 0; r < CL; ++r) {
-            const float f = ex2(mv[r] - M);
-            O = fmaf(rp[r][idx], f, O);
-            L = fmaf(rp[r][G * D + G + hh], f, L);
-          }
-        }
-        cp[idx] = O;
-        if (idx % D == 0) {
-          cp[G * D + hh] = M;
-          cp[G * D + G + hh] = L;
-        }
-      }
-    }
-  } else {
-    __syncthreads();  // the item partial is complete in shared memory
-    float* cp = ps + (size_t)item * C::PART;
-    for (int idx = tid; idx < C::PART; idx += blockDim.x) cp[idx] = mypart[idx];
-  }
-  // the first CTA publishes the cluster partial and learns whether its
-  // cluster is the stream's last; it tells every CTA of the cluster
-  if (crank == 0) {
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      const int last = atomicAdd(&a.counters[(size_t)srel * kCountersPerStream], 1u) == (unsigned)(ncl - 1);
-      if constexpr (CL > 1) {
-        cg::cluster_group cluster = cg::this_cluster();
-#pragma unroll
-        for (int r = 0; r < CL; ++r) *cluster.map_shared_rank(&is_last, r) = last;
-      } else {
-        is_last = last;
-      }
-    }
-  }
-  if constexpr (CL > 1) {
-    cg::this_cluster().sync();  // remote partial reads and the is_last stores are complete
-  } else {
-    __syncthreads();
-  }
-  if (!is_last) return;
-  // Level 2: the CTAs of the last cluster merge the cluster partials, each a
-  // slice of the outputs
-  __threadfence();
-  float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  merge_outputs<D, G, CL>(ps, ncl, outp, crank, tid);
-  if (crank == 0 && tid == 0) a.counters[(size_t)srel * kCountersPerStream] = 0u;
-}
-
-// Host-side caches (per device) of the decode kernel's shared-memory
-// attribute and of its resident capacity: both are fixed for a given
-// (device, D, G, cluster, size), and querying them on every call costs more
-// host time than a decode step.
-std::mutex g_attr_mu;
-std::map<std::tuple<int, int, int, int>, int> g_smem_set;        // (dev, D, G, CL) -> largest size set
-std::map<std::tuple<int, int, int, int, int>, int> g_resident;   // (dev, D, G, CL, smem) -> CTAs
-
-template <int D, int G, int CL>
-cudaError_t ensure_smem(int smem) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(g_attr_mu);
-  int& cur = g_smem_set[std::make_tuple(dev, D, G, CL)];
-  if (cur >= smem) return cudaSuccess;
-  e = cudaFuncSetAttribute(decode_kernel<D, G, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) cur = smem;
-  return e;
-}
-
-template <int D, int G, int CL>
-cudaError_t launch_dgc(const DecodeArgs& a, int smem, cudaStream_t st) {
-  cudaError_t e = ensure_smem<D, G, CL>(smem);
-  if (e != cudaSuccess) return e;
-  const int streams = a.n_layers * a.g.B * a.g.Hkv;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cluster_items(a.n_splits + a.n_win + a.n_pack, CL), streams, 1);
-  cfg.blockDim = dim3(kDecodeThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = RQ_DECODE_PDL;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (CL > 1) {
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = CL;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.numAttrs = 2;
-  }
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G, CL>, a);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
-}
-
-template <int D, int G>
-cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
-  if (a.cluster == 1) return launch_dgc<D, G, 1>(a, smem, st);
-  if (a.cluster == kDecodeCluster) return launch_dgc<D, G, kDecodeCluster>(a, smem, st);
-  return cudaErrorInvalidValue;
-}
-
-// CTAs of the decode kernel that the device holds at once, in whole clusters.
-template <int D, int G, int CL>
-int resident_ctas_dgc(int smem) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return CL;
-  {
-    std::lock_guard<std::mutex> lock(g_attr_mu);
-    auto it = g_resident.find(std::make_tuple(dev, D, G, CL, smem));
-    if (it != g_resident.end()) return it->second;
-  }
-  if (ensure_smem<D, G, CL>(smem) != cudaSuccess) return CL;
-  int n = 0;
-  if (CL > 1) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CL * 64, 1, 1);
-    cfg.blockDim = dim3(kDecodeThreads, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<D, G, CL>, &cfg) != cudaSuccess || n < 1) return CL;
-    n *= CL;
-  } else {
-    int per_sm = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<D, G, CL>, kDecodeThreads, smem) !=
-            cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || per_sm < 1 || sms < 1)
-      return 1;
-    n = per_sm * sms;
-  }
-  std::lock_guard<std::mutex> lock(g_attr_mu);
-  g_resident[std::make_tuple(dev, D, G, CL, smem)] = n;
-  return n;
-}
-
-template <int D, int G>
-int resident_ctas_dg(int cluster, int smem) {
-  return cluster == 1 ? resident_ctas_dgc<D, G, 1>(smem) : resident_ctas_dgc<D, G, kDecodeCluster>(smem);
-}
-
-}  // namespace
 
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   const int part = G * D + 2 * G;
@@ -1038,17 +24,34 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
 
 int decode_resident_ctas(int D, int G, int cluster, int smem) {
 #define RQ_DG(DD, GG) \
-  if (D == DD && G == GG) return resident_ctas_dg<DD, GG>(cluster, smem);
+  if (D == DD && G == GG) return decode_resident_ctas_dg<DD, GG>(cluster, smem);
   RQ_DG(128, 1) RQ_DG(128, 2) RQ_DG(128, 4) RQ_DG(128, 8)
   RQ_DG(64, 1) RQ_DG(64, 2) RQ_DG(64, 4) RQ_DG(64, 8)
 #undef RQ_DG
   return 1;
 }
 
+// Self-test of the device timeout path: one thread waits on an mbarrier that
+// nothing ever completes, with the same bounded wait the decode pipeline uses,
+// gives up after limit_ns and records the timeout in the status word the way
+// a decode kernel does.
+__global__ void wait_timeout_selftest_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  mbar_fence_init();
+  if (!mbar_wait_bounded(&bar, 0u, limit_ns)) atomicCAS(status, 0, kDeviceTimeout);
+}
+
+cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, int smem, cudaStream_t st) {
   const int D = a.g.D, G = a.g.G;
 #define RQ_DG(DD, GG) \
-  if (D == DD && G == GG) return launch_dg<DD, GG>(a, smem, st);
+  if (D == DD && G == GG) return launch_decode_dg<DD, GG>(a, smem, st);
   RQ_DG(128, 1) RQ_DG(128, 2) RQ_DG(128, 4) RQ_DG(128, 8)
   RQ_DG(64, 1) RQ_DG(64, 2) RQ_DG(64, 4) RQ_DG(64, 8)
 #undef RQ_DG

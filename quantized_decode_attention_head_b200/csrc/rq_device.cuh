@@ -1,5 +1,5 @@
-// Device-side helpers: packed-format tables, tensor-core MMA, fragment
-// transpose, mbarrier and bulk-copy primitives (sm_100a).
+// Device-side helpers: packed-format tables, integer tensor-core MMA,
+// mbarrier and bulk-copy primitives (sm_100a).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -61,15 +61,6 @@ __device__ __forceinline__ void put_code(uint32_t* words, int rho, int kh, int e
 }
 
 // ------------------------------------------------------------ tensor cores
-// D = A(16x16 f16, row) * B(16x8 f16, col) + C, fp32 accumulate.
-__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // D = A(16x32 u8, row) * B(32x8 s8 / u8, col) + C, s32 accumulate; every C
 // element is the same value c.  Results are returned as raw 32-bit words.
 __device__ __forceinline__ void imma_u8s8(uint32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
@@ -87,18 +78,6 @@ __device__ __forceinline__ void imma_u8u8(uint32_t (&d)[4], const uint32_t (&a)[
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};\n"
       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c), "r"(c), "r"(c), "r"(c));
-}
-
-// Transpose an 8x8 b16 matrix held one row-pair per thread (m8n8 fragment).
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -149,13 +128,14 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
   return t;
 }
-// Bounded wait: gives up after ~1 s and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+// Bounded wait: gives up after limit_ns (default ~1 s) and returns false.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > 1000000000ull) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 // Orders this thread's earlier generic-proxy shared-memory accesses before

@@ -59,6 +59,7 @@ size_t layout(const rq_cache_config* c, rq::Geom& g, std::vector<HeadDesc>& desc
   g.S = c->n_sink;
   g.R = c->n_recent;
   g.max_tiles = rq::quantized_tokens(c->max_tokens, g.S, g.R) / rq::kTile;
+  g.hybrid = c->hybrid ? 1 : 0;
   g.win_bytes = rq::window_bytes(g.S, g.R, g.D);
   const int nh = g.L * g.Hkv;
   desc.assign(nh, HeadDesc{});
@@ -134,9 +135,12 @@ rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_
 
 // Decode arguments for layers [l0, l0 + nl) of a cache holding T tokens, with
 // the workspace checked and partitioned; the fused-append pointers are null.
+// a.cluster is set before the workspace check, so a caller whose workspace
+// was too small for the automatic plan can retry with fewer splits and the
+// same cluster size (cluster_override != 0 replaces the plan's choice).
 rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, float* out, float softmax_scale,
                       int n_splits, void* workspace, size_t ws_bytes, rq::DecodeArgs& a, int& smem,
-                      int n_pack = 0) {
+                      int n_pack = 0, int cluster_override = 0) {
   const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
   const int n_tiles = Tq / rq::kTile;
   const int streams = nl * c->g.B * c->g.Hkv;
@@ -146,6 +150,8 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   int cluster = rq::kDecodeCluster;  // explicit split counts run in clusters
   int splits =
       n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win + n_pack, &cluster) : n_splits;
+  if (cluster_override != 0) cluster = cluster_override;
+  a.cluster = cluster;
   if (splits > n_tiles) splits = n_tiles;
   if (n_tiles > 0 && splits < 1) splits = 1;
   const int items = splits + n_win + n_pack;
@@ -170,7 +176,6 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   a.pack_pos = 0;
   a.pack_tile = 0;
   a.n_streams = streams;
-  a.cluster = cluster;
   a.stages = rq::decode_stages(stage_bytes);
   a.stage_bytes = stage_bytes;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -242,10 +247,19 @@ rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes,
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) c->sm_count = n;
   }
   c->k_norm = cfg->k_norm ? 1 : 0;
-  cudaError_t e = cudaMemcpy(c->buf, c->desc.data(), c->desc.size() * sizeof(HeadDesc), cudaMemcpyHostToDevice);
-  // normalization factors start at 1 (a cache built by appends only)
-  if (e == cudaSuccess) e = rq::launch_norm_reset(c->buf, reinterpret_cast<const HeadDesc*>(c->buf), c->g, 0);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(0);
+  // The header copy and the reset of the normalization factors (to 1: a cache
+  // built by appends only) run on a private non-blocking stream that only
+  // this call waits for, so other streams of the process are not serialised
+  // behind it (the legacy default stream would be).
+  cudaStream_t s = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+  if (e == cudaSuccess) {
+    e = cudaMemcpyAsync(c->buf, c->desc.data(), c->desc.size() * sizeof(HeadDesc), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = rq::launch_norm_reset(c->buf, reinterpret_cast<const HeadDesc*>(c->buf), c->g, s);
+    const cudaError_t e2 = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = e2;
+    cudaStreamDestroy(s);
+  }
   if (e != cudaSuccess) {
     delete c;
     return RQ_ERR_CUDA;
@@ -344,6 +358,12 @@ rq_status rq_decode_workspace_bytes(const rq_cache* c, int n_splits, size_t* byt
 rq_status rq_decode_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream) {
   if (!workspace || ws_bytes < rq::ws_counter_offset()) return RQ_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(workspace, 0, ws_bytes, stream));
+}
+
+rq_status rq_selftest_device_timeout(void* workspace, size_t ws_bytes, unsigned long long limit_ns,
+                                     cudaStream_t stream) {
+  if (!workspace || ws_bytes < rq::ws_counter_offset() || limit_ns > 1000000000ull) return RQ_ERR_INVALID_ARG;
+  return cuda_status(rq::launch_wait_timeout_selftest(static_cast<int*>(workspace), limit_ns, stream));
 }
 
 rq_status rq_decode_read_status(const void* workspace, int* device_status) {
@@ -453,14 +473,19 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
                              rq::kNoAllocScratchBytes, a, smem);
   if (st == RQ_ERR_WORKSPACE && n_splits == 0) {
     // the automatic plan needs more partials than the array holds: take the
-    // most splits whose partials fit
+    // most splits whose partials fit, in the plan's own cluster size (with
+    // clusters the items are padded to whole clusters)
+    const int cluster = a.cluster;
     const int64_t streams = (int64_t)nl * c->g.B * c->g.Hkv;
-    const int64_t items = (int64_t)(rq::kNoAllocScratchBytes - rq::ws_partial_offset(all_streams)) /
-                          (streams * (int64_t)(c->g.G * c->g.D + 2 * c->g.G) * 4);
+    const size_t avail = rq::kNoAllocScratchBytes > rq::ws_partial_offset(all_streams)
+                             ? rq::kNoAllocScratchBytes - rq::ws_partial_offset(all_streams)
+                             : 0;
+    int64_t items = (int64_t)avail / (streams * (int64_t)(c->g.G * c->g.D + 2 * c->g.G) * 4);
+    items = items / cluster * cluster;
     const int64_t s = items - rq::window_items(c->length[l0], c->g.S, c->g.R);
     if (s >= 1)
       st = fill_decode(c, l0, nl, c->length[l0], q, out, softmax_scale, (int)s, scratch, rq::kNoAllocScratchBytes,
-                       a, smem);
+                       a, smem, 0, cluster);
   }
   if (st == RQ_ERR_WORKSPACE) return RQ_ERR_WORKSPACE;  // more split partials than the fixed array holds
   if (st != RQ_OK) return st;
@@ -468,4 +493,13 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
   // whatever the previous call (on any stream) left in it
   if (cudaMemsetAsync(scratch, 0, rq::ws_partial_offset(all_streams), stream) != cudaSuccess) return RQ_ERR_CUDA;
   return cuda_status(rq::launch_decode(a, smem, stream));
+}
+
+// Status word of the scratch array behind rq_decode_attention_noalloc on the
+// current device (see include/rq.h).
+extern "C" rq_status rq_decode_noalloc_read_status(int* device_status) {
+  if (!device_status) return RQ_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if (rq::noalloc_scratch(&scratch) != cudaSuccess) return RQ_ERR_CUDA;
+  return cuda_status(cudaMemcpy(device_status, scratch, sizeof(int), cudaMemcpyDeviceToHost));
 }

@@ -27,6 +27,7 @@ static_assert(sizeof(HeadDesc) == 40, "HeadDesc layout");
 struct Geom {
   int L, B, Hq, Hkv, D, G, S, R;
   int max_tiles;
+  int hybrid;          // per-group symmetric / asymmetric choice (group_params)
   int64_t win_bytes;   // bytes of one stream's window block
 };
 
@@ -160,6 +161,10 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D);
 // CTAs of the decode kernel resident on the device at once, in whole clusters
 // of `cluster` CTAs
 int decode_resident_ctas(int D, int G, int cluster, int smem_bytes);
+
+// One-thread kernel whose bounded mbarrier wait runs out after limit_ns and
+// records kDeviceTimeout in *status (self-test of the timeout path).
+cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t s);
 
 // Size of the device array behind rq_decode_attention_noalloc (bytes).
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;

@@ -55,9 +55,25 @@ __device__ __forceinline__ void stage_kinv(float* kinv, const float* nrm, int la
 __device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Scale/zero of one group from its min and max; returns the meta word.
+// Hybrid option (InnerQ, technique (i): a symmetric or an asymmetric
+// quantizer per group, chosen from the group's statistics; this library's
+// rule): a group nearly centred on zero, |max + min| <= (max - min) / 8, is
+// quantized on the symmetric interval [-M, M], M = max(|min|, |max|).
+constexpr float kHybridTau = 0.125f;
+
+// Scale/zero of one group from its min and max; returns the meta word and
+// leaves in mn the zero the codes are taken from.  The extremes are real
+// numbers: x + 0 turns a -0.0 extreme into +0.0, so the stored zero and scale
+// do not depend on which of two equal zeros fminf / fmaxf returned.
 template <int B>
-__device__ __forceinline__ uint32_t group_params(float mn, float mx, float& r) {
+__device__ __forceinline__ uint32_t group_params(float& mn, float mx, float& r, bool hybrid) {
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  if (hybrid && fabsf(__fadd_rn(mx, mn)) <= __fmul_rn(__fsub_rn(mx, mn), kHybridTau)) {
+    const float m = fmaxf(fabsf(mn), fabsf(mx));
+    mn = __fadd_rn(-m, 0.0f);
+    mx = m;
+  }
   float s32 = __fdiv_rn(__fsub_rn(mx, mn), (float)((1 << B) - 1));
   s32 = fminf(s32, 65504.0f);
   const __half h = __float2half_rn(s32);
@@ -76,7 +92,7 @@ __device__ __forceinline__ uint32_t code_of(float x, float z, float r) {
 
 // KN: multiply by the K normalization factors 1/n (false: n = 1, skipped).
 template <int D, int KB, bool KN>
-__device__ void pack_k(HalfTile<D>& sm, const float* kinv, uint8_t* rec, int lane) {
+__device__ void pack_k(HalfTile<D>& sm, const float* kinv, uint8_t* rec, int lane, bool hybrid) {
   constexpr int NG = D / 32;
   constexpr int W = words_per_lane(KB, D);
   // statistics: lane = token, rotated word order spreads smem banks
@@ -95,7 +111,7 @@ __device__ void pack_k(HalfTile<D>& sm, const float* kinv, uint8_t* rec, int lan
         mx = fmaxf(mx, fmaxf(x0, x1));
       }
       float r;
-      const uint32_t meta = group_params<KB>(mn, mx, r);
+      const uint32_t meta = group_params<KB>(mn, mx, r, hybrid);
       sm.r[t * NG + grp] = r;
       sm.z[t * NG + grp] = mn;
       const int i = (t & 7) * 4 + (t >> 4) * 2 + ((t >> 3) & 1);
@@ -130,7 +146,7 @@ __device__ void pack_k(HalfTile<D>& sm, const float* kinv, uint8_t* rec, int lan
 }
 
 template <int D, int VB>
-__device__ void pack_v(HalfTile<D>& sm, uint8_t* vrec, int lane) {
+__device__ void pack_v(HalfTile<D>& sm, uint8_t* vrec, int lane, bool hybrid) {
   constexpr int W = words_per_lane(VB, D);
   // statistics: each lane owns channel pairs (2w, 2w+1)
 #pragma unroll
@@ -147,10 +163,10 @@ __device__ void pack_v(HalfTile<D>& sm, uint8_t* vrec, int lane) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int d = 2 * w + h;
-      float r;
-      const uint32_t meta = group_params<VB>(h ? mn1 : mn0, h ? mx1 : mx0, r);
+      float r, z = h ? mn1 : mn0;
+      const uint32_t meta = group_params<VB>(z, h ? mx1 : mx0, r, hybrid);
       sm.r[d] = r;
-      sm.z[d] = h ? mn1 : mn0;
+      sm.z[d] = z;
       const int i = (d & 7) * (D / 8) + (d >> 4) * 2 + ((d >> 3) & 1);
       reinterpret_cast<uint32_t*>(vrec + blob_bytes(VB, D))[i] = meta;
     }
@@ -183,22 +199,23 @@ __device__ void pack_v(HalfTile<D>& sm, uint8_t* vrec, int lane) {
 }
 
 template <int D, bool KN>
-__device__ __forceinline__ void pack_k_dispatch(HalfTile<D>& sm, const float* kinv, int kb, uint8_t* rec, int lane) {
+__device__ __forceinline__ void pack_k_dispatch(HalfTile<D>& sm, const float* kinv, int kb, uint8_t* rec, int lane,
+                                                bool hybrid) {
   switch (kb) {
-    case 2: pack_k<D, 2, KN>(sm, kinv, rec, lane); break;
-    case 3: pack_k<D, 3, KN>(sm, kinv, rec, lane); break;
-    case 4: pack_k<D, 4, KN>(sm, kinv, rec, lane); break;
-    default: pack_k<D, 8, KN>(sm, kinv, rec, lane); break;
+    case 2: pack_k<D, 2, KN>(sm, kinv, rec, lane, hybrid); break;
+    case 3: pack_k<D, 3, KN>(sm, kinv, rec, lane, hybrid); break;
+    case 4: pack_k<D, 4, KN>(sm, kinv, rec, lane, hybrid); break;
+    default: pack_k<D, 8, KN>(sm, kinv, rec, lane, hybrid); break;
   }
 }
 
 template <int D>
-__device__ __forceinline__ void pack_v_dispatch(HalfTile<D>& sm, int vb, uint8_t* vrec, int lane) {
+__device__ __forceinline__ void pack_v_dispatch(HalfTile<D>& sm, int vb, uint8_t* vrec, int lane, bool hybrid) {
   switch (vb) {
-    case 2: pack_v<D, 2>(sm, vrec, lane); break;
-    case 3: pack_v<D, 3>(sm, vrec, lane); break;
-    case 4: pack_v<D, 4>(sm, vrec, lane); break;
-    default: pack_v<D, 8>(sm, vrec, lane); break;
+    case 2: pack_v<D, 2>(sm, vrec, lane, hybrid); break;
+    case 3: pack_v<D, 3>(sm, vrec, lane, hybrid); break;
+    case 4: pack_v<D, 4>(sm, vrec, lane, hybrid); break;
+    default: pack_v<D, 8>(sm, vrec, lane, hybrid); break;
   }
 }
 

@@ -54,11 +54,11 @@ __global__ void __launch_bounds__(kQuantWarps * 32, kQuantMinBlocks) quantize_ti
   if (KN) stage_kinv<D>(sm.kinv, stream_norm(a.buf, hd, a.g, b), lane);
   __syncwarp();
   uint8_t* rec = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)tile * hd.rec_bytes;
-  pack_k_dispatch<D, KN>(sm.t, sm.kinv, hd.k_bits, rec, lane);
+  pack_k_dispatch<D, KN>(sm.t, sm.kinv, hd.k_bits, rec, lane, a.g.hybrid);
   __syncwarp();  // every lane has read the K rows and statistics
   stage_rows_contig<D>(sm.t.x, a.v + row0, lane);
   __syncwarp();
-  pack_v_dispatch<D>(sm.t, hd.v_bits, rec + blob_bytes(hd.k_bits, D) + 4 * D, lane);
+  pack_v_dispatch<D>(sm.t, hd.v_bits, rec + blob_bytes(hd.k_bits, D) + 4 * D, lane, a.g.hybrid);
 }
 
 // Copy sink tokens [0, min(S,T)) and recent tokens [S+Tq, T) into the window
@@ -144,9 +144,9 @@ __global__ void __launch_bounds__(64) append_kernel(AppendArgs a) {
   __syncthreads();
   uint8_t* rec = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)a.flush_tile * hd.rec_bytes;
   if (warp == 0) {
-    pack_k_dispatch<D, true>(sm.k, sm.kinv, hd.k_bits, rec, lane);
+    pack_k_dispatch<D, true>(sm.k, sm.kinv, hd.k_bits, rec, lane, a.g.hybrid);
   } else {
-    pack_v_dispatch<D>(sm.v, hd.v_bits, rec + blob_bytes(hd.k_bits, D) + 4 * D, lane);
+    pack_v_dispatch<D>(sm.v, hd.v_bits, rec + blob_bytes(hd.k_bits, D) + 4 * D, lane, a.g.hybrid);
   }
 }
 
@@ -164,7 +164,7 @@ __device__ double group_sse(float x) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
   float r;
-  const uint32_t meta = group_params<B>(mn, mx, r);
+  const uint32_t meta = group_params<B>(mn, mx, r, false);
   const double s = (double)__half2float(__ushort_as_half((unsigned short)(meta & 0xFFFFu)));
   const double z = (double)__uint_as_float(meta & 0xFFFF0000u);
   const double xh = __dadd_rn(__dmul_rn((double)code_of<B>(x, mn, r), s), z);
@@ -271,12 +271,14 @@ cudaError_t launch_norm_reset(uint8_t* buf, const HeadDesc* desc, const Geom& g,
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t st) {
   const int streams = a.g.L * a.g.B * a.g.Hkv;
   // the prefill fixes the K normalization factors before any tile is packed
+  // (a cache without normalization keeps the factors of 1 that
+  // rq_cache_init wrote: no launch)
   if (a.k_norm && a.T > 0) {
     norm_fill_kernel<<<streams, 128, 0, st>>>(a.buf, a.desc, a.g, 0.0f);
     const int tpb = 1024;
     norm_max_kernel<<<dim3((a.T + tpb - 1) / tpb, streams), 128, 0, st>>>(a, tpb);
     norm_finalize_kernel<<<streams, 128, 0, st>>>(a);
-  } else {
+  } else if (a.k_norm) {
     norm_fill_kernel<<<streams, 128, 0, st>>>(a.buf, a.desc, a.g, 1.0f);
   }
   cudaError_t e0 = cudaGetLastError();

@@ -46,17 +46,18 @@ def workload_bits(wl):
     return (lk, lv), (ok, ov)
 
 
-def make_cache(wl, k_bits, v_bits, max_tokens, k_norm=False):
+def make_cache(wl, k_bits, v_bits, max_tokens, k_norm=False, hybrid=False):
     return QuantizedKVCache(wl.n_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n_sink,
-                            wl.n_recent, max_tokens, k_bits, v_bits, k_norm=k_norm)
+                            wl.n_recent, max_tokens, k_bits, v_bits, k_norm=k_norm, hybrid=hybrid)
 
 
-def oracle_streams(wl, k_bits, v_bits, k_np, v_np, which, k_norm=False):
+def oracle_streams(wl, k_bits, v_bits, k_np, v_np, which, k_norm=False, hybrid=False):
     """Oracle StreamCache for each (l, b, h) in ``which`` from float32 inputs
     [L, B, H, T, D]."""
     out = {}
     for (l, b, h) in which:
-        st = ca.StreamCache(wl.head_dim, int(k_bits[l, h]), int(v_bits[l, h]), wl.n_sink, wl.n_recent, k_norm=k_norm)
+        st = ca.StreamCache(wl.head_dim, int(k_bits[l, h]), int(v_bits[l, h]), wl.n_sink, wl.n_recent, k_norm=k_norm,
+                            hybrid=hybrid)
         st.prefill(k_np[l, b, h], v_np[l, b, h])
         out[(l, b, h)] = st
     return out

@@ -12,6 +12,7 @@ import torch
 from gpu_helpers import (all_streams, assert_close, check_stream_bytes, make_cache, oracle_decode, oracle_streams,
                          to_f32, workload_bits)
 from oracle import cache as ca
+from oracle import quantize as qz
 from quantized_decode_attention_head_b200 import workloads
 from quantized_decode_attention_head_b200.api import QuantizedKVCache
 
@@ -48,6 +49,75 @@ def test_quantize_all_bit_pairs_bitexact(d):
     assert cache.length(0) == wl.context
     for key, s in st.items():
         check_stream_bytes(cache, s, *key)
+
+
+def _plant_signed_zeros(x, kind, rng):
+    """Overwrite groups of a bf16 [L, B, H, T, D] tensor with zeros of both
+    signs: K groups are 32 channels of a token, V groups a channel over the 32
+    tokens of a tile.  Patterns: all +0, all -0, mixed zeros, a -0 minimum
+    under positive values, a -0 maximum over negative values."""
+    L, B, H, T, D = x.shape
+    neg0 = torch.tensor(-0.0, dtype=torch.bfloat16)
+    x = x.cpu().clone()
+    tile0 = 4  # first tile token (n_sink = 4)
+    for l in range(L):
+        for b in range(B):
+            for h in range(H):
+                for p in range(5):
+                    t = tile0 + int(rng.integers(0, 32 * 3))  # a token of the first three tiles
+                    if kind == "K":
+                        g = int(rng.integers(0, D // 32))
+                        idx = (l, b, h, t, slice(32 * g, 32 * g + 32))
+                    else:
+                        tl = (t - tile0) // 32
+                        d0 = int(rng.integers(0, D))
+                        idx = (l, b, h, slice(tile0 + 32 * tl, tile0 + 32 * tl + 32), d0)
+                    grp = x[idx]
+                    if p == 0:
+                        grp.zero_()
+                    elif p == 1:
+                        grp.fill_(neg0)
+                    elif p == 2:
+                        grp.zero_()
+                        grp[::3] = neg0
+                    elif p == 3:
+                        grp.copy_(grp.abs() + 0.125)
+                        grp[int(rng.integers(0, 32))] = neg0
+                        grp[int(rng.integers(0, 32))] = 0.0
+                    else:
+                        grp.copy_(-grp.abs() - 0.25)
+                        grp[int(rng.integers(0, 32))] = neg0
+                        grp[int(rng.integers(0, 32))] = 0.0
+                    x[idx] = grp
+    return x.cuda()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_signed_zero_groups_bitexact(d):
+    """Groups whose extremes are +0 / -0 (and all-zero groups) pack to the
+    oracle's bytes: a zero extreme is stored as +0 with a +0 scale whatever
+    order the zeros come in."""
+    wl = _small(head_dim=d, n_layers=1, context=4 + 32 * 3 + 32 + 9)
+    kb, vb = _bits_grid(1, wl.n_kv_heads)
+    rng = np.random.default_rng(41)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    k = _plant_signed_zeros(k, "K", rng)
+    v = _plant_signed_zeros(v, "V", rng)
+    cache = make_cache(wl, kb, vb, wl.context + 8)
+    cache.rq_quantize_kv(k, v)
+    st = oracle_streams(wl, kb, vb, to_f32(k), to_f32(v), all_streams(wl))
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+        for rec in s.records():
+            q = qz.unpack_record(rec, s.kb, s.vb, s.d)
+            for name in ("k_z", "v_z", "k_s", "v_s"):
+                vals = q[name]
+                assert not np.any(np.signbit(vals) & (vals == 0)), f"{key} {name}: a -0.0 was stored"
+    q, _, _ = workloads.step_inputs(wl, 1, f, "cuda")
+    out = cache.rq_decode_attention(0, q[0, 0].contiguous()).cpu().numpy()
+    exp = oracle_decode(wl, st, to_f32(q[0]).astype(np.float64), [(0, b) for b in range(wl.batch)])
+    for b in range(wl.batch):
+        assert_close(out[b], exp[(0, b)], f"signed zeros b {b}")
 
 
 @pytest.mark.parametrize("d,g", [(64, 1), (64, 2), (64, 4), (64, 8), (128, 1), (128, 2), (128, 4), (128, 8)])
@@ -314,3 +384,40 @@ def test_tiny_workload_end_to_end():
     out = cache.rq_decode_attention(0, q[0, 0].contiguous()).cpu().numpy()
     exp = oracle_decode(wl, st, to_f32(q[0]).astype(np.float64), [(0, 0)])[(0, 0)]
     assert_close(out[0], exp, "tiny")
+
+
+@pytest.mark.parametrize("d,k_norm", [(64, False), (128, False), (128, True)])
+def test_hybrid_prefill_decode_and_steps(d, k_norm):
+    """Hybrid symmetric / asymmetric groups: tile records and window rows bit
+    for bit against the oracle after the prefill and after fused steps across
+    tile flushes, decoded outputs within the parity tolerance; both kinds of
+    group occur in the data."""
+    wl = _small(head_dim=d, n_q_heads=16, n_kv_heads=4, k_sigma=1.0, context=4 + 32 * 5 + 32 + 7)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    steps = 40
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, wl.context + steps, k_norm=k_norm, hybrid=True)
+    cache.rq_quantize_kv(k, v)
+    knp0, vnp0 = to_f32(k), to_f32(v)
+    st = oracle_streams(wl, kb, vb, knp0, vnp0, all_streams(wl), k_norm=k_norm, hybrid=True)
+    # V groups of the prefill's tiles: one channel over 32 tokens
+    vt = vnp0[:, :, :, wl.n_sink:wl.n_sink + 32 * 5].reshape(wl.n_layers, wl.batch, wl.n_kv_heads, 5, 32, d)
+    sym = qz.symmetric_groups(vt.min(axis=4), vt.max(axis=4))
+    assert 0 < sym.sum() < sym.size
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    q, kn, vn = workloads.step_inputs(wl, steps, f, "cuda")
+    knp, vnp, qnp = to_f32(kn), to_f32(vn), to_f32(q).astype(np.float64)
+    ws = cache.make_workspace()
+    for t in range(steps):
+        for (l, b, h), s in st.items():
+            s.append(knp[t, l, b, h], vnp[t, l, b, h])
+        out = cache.rq_decode_step(-1, q[t].contiguous(), kn[t].contiguous(), vn[t].contiguous(),
+                                   workspace=ws).cpu().numpy()
+        if t % 7 == 0 or t == steps - 1:
+            exp = oracle_decode(wl, st, qnp[t], [(l, b) for l in range(wl.n_layers) for b in range(wl.batch)])
+            for (l, b), e in exp.items():
+                assert_close(out[l, b], e, f"hybrid step {t} layer {l} b {b}")
+    for key, s in st.items():
+        check_stream_bytes(cache, s, *key)
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0

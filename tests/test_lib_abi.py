@@ -179,3 +179,12 @@ def test_cap_weights_matches_the_oracle():
     w = np.array([0.5, 1.0, 2.0, 300.0, 1.5])
     assert np.array_equal(rq_cap_weights(w), cal.cap_weights(w))
     assert np.array_equal(rq_cap_weights(w, 2.0), cal.cap_weights(w, 2.0))
+
+
+def test_timeout_selftest_rejects_bad_arguments_before_cuda():
+    """Argument checks happen on the host, before any CUDA call: no workspace,
+    a workspace smaller than its status block, or a limit above one second."""
+    L = _lib.lib()
+    assert L.rq_selftest_device_timeout(None, 4096, 1000, None) == 1
+    assert L.rq_selftest_device_timeout(ctypes.c_void_p(256), 16, 1000, None) == 1
+    assert L.rq_selftest_device_timeout(ctypes.c_void_p(256), 4096, 2_000_000_000, None) == 1
