@@ -8,7 +8,7 @@
 namespace rq {
 
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
-  const int part = G * D + 2 * G;
+  const int part = partial_floats(G, D);
   // merge slots + window scratch (q, one K and one V chunk)
   int merge = (NW * part + G * D) * 4 + 2 * kWinChunk * D * 2;
   if (merge < (NW + 1) * part * 4) merge = (NW + 1) * part * 4;  // warp slots + the item partial
@@ -22,9 +22,9 @@ int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   return (need + 127) / 128 * 128 + scratch;
 }
 
-int decode_resident_ctas(int D, int G, int cluster, int smem) {
+int decode_resident_ctas(int D, int G, int cluster, int smem, int q_terms) {
 #define RQ_DG(DD, GG) \
-  if (D == DD && G == GG) return decode_resident_ctas_dg<DD, GG>(cluster, smem);
+  if (D == DD && G == GG) return decode_resident_ctas_dg<DD, GG>(cluster, smem, q_terms);
   RQ_DG(128, 1) RQ_DG(128, 2) RQ_DG(128, 4) RQ_DG(128, 8)
   RQ_DG(64, 1) RQ_DG(64, 2) RQ_DG(64, 4) RQ_DG(64, 8)
 #undef RQ_DG

@@ -53,13 +53,15 @@ constexpr uint32_t kBiasBits = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kBias = 12582912.0f;         // 1.5 * 2^23
 constexpr float kPScale = 65535.0f;          // P in 16-bit fixed point: p_int = rint(p * 65535)
 constexpr float kQMax = 32639.0f;            // q_int in [-32639, 32639] = 256 * q1 + q2, q1, q2 in s8
+// normalized caches: q_int in [-8323072, 8323072] = 65536 q1 + 256 q2 + q3, all s8
+constexpr float kQMax3 = 8323072.0f;
 
 template <int D, int G>
 struct Cfg {
   static constexpr int NG = D / 32;                  // K groups per token (one k32 MMA each)
   static constexpr int NB = (G + 3) / 4;             // 8-column blocks: 4 heads x 2 terms
   static constexpr int HB = G < 4 ? G : 4;           // heads per block
-  static constexpr int PART = G * D + 2 * G;         // floats per partial state
+  static constexpr int PART = partial_floats(G, D);  // floats per partial state (16-byte multiple)
   static constexpr int KMW = NG;                     // K meta words converted per lane
   static constexpr int VMW = D / 32;                 // V meta words converted per lane
   static constexpr int KSTR = NG * 8 + 4;            // floats per gid row of the K scale scratch
@@ -69,10 +71,14 @@ struct Cfg {
 
 // Per-warp state.  Thread (gid, tig) owns, in block nb, head 4nb + tig of the
 // MMA results (columns 2 tig, 2 tig + 1 = the two terms of that head).
-template <int D, int G>
+// QT = 2: q in 16-bit fixed point (two s8 terms); QT = 3: 24-bit (three s8
+// terms, for caches whose K normalization factors are folded into q and
+// widen its range): terms 1, 2 in qb, term 3 in qb3 (column 2 h, 2 h + 1 = 0).
+template <int D, int G, int QT = 2>
 struct WarpState {
   using C = Cfg<D, G>;
   uint32_t qb[C::NB][C::NG][2];  // q B-fragments: column n = 2 h + term, bytes = s8 terms
+  uint32_t qb3[C::NB][C::NG][QT == 3 ? 2 : 1];  // third-term B-fragments (QT = 3)
   float2 qz[C::NB][C::NG];       // sum of q_int over group g (both halves) -- zero-point term
   float xs[C::NB];               // sq * softmax scale * log2(e)
   float m[C::NB], l[C::NB];      // running max (log2 units) and sum of p (x 65535)
@@ -85,6 +91,27 @@ struct WarpState {
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+#ifndef RQ_CVT_BIAS
+#define RQ_CVT_BIAS 0
+#endif
+// C operand of the two-term MMAs: 0 (int32 results) or the bits of 1.5 * 2^23
+// (each result, read as a float, is 1.5 * 2^23 + the exact integer sum).
+constexpr uint32_t kTermC = RQ_CVT_BIAS ? kBiasBits : 0u;
+
+// The two-term results (hi, lo) of rows gid and gid + 8 of one MMA -> the
+// pair (256 hi + lo) of both rows in fp32, each rounded once.
+__device__ __forceinline__ float2 combine_terms(const uint32_t (&c)[4]) {
+  if constexpr (RQ_CVT_BIAS) {
+    const float2 nb = make_float2(-kBias, -kBias);
+    const float2 r0 = fadd2(make_float2(__uint_as_float(c[0]), __uint_as_float(c[1])), nb);  // exact integers
+    const float2 r1 = fadd2(make_float2(__uint_as_float(c[2]), __uint_as_float(c[3])), nb);
+    return make_float2(fmaf(256.0f, r0.x, r0.y), fmaf(256.0f, r1.x, r1.y));
+  } else {
+    // |256 hi + lo| < 2^31: exact in int32, one rounding to fp32 per row
+    return make_float2((float)((int)c[0] * 256 + (int)c[1]), (float)((int)c[2] * 256 + (int)c[3]));
+  }
+}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -102,8 +129,9 @@ __device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) 
 // q of the G heads -> per-head 16-bit fixed point (sq = max|q_h| / 32639)
 // split into two s8 terms q_int = 256 q1 + q2, laid out as the k32 x n8
 // B-fragments of the q.K^T MMA (column n = 2 * head + term).
-template <int D, int G, int KB, int VB>
-__device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, const float* nrm, float scale_log2, int lane) {
+template <int D, int G, int KB, int VB, int QT>
+__device__ void setup_query(WarpState<D, G, QT>& st, const uint16_t* qh, const float* nrm, float scale_log2,
+                            int lane) {
   using C = Cfg<D, G>;
   const int gid = lane >> 2, tig = lane & 3;
   const int hl = gid >> 1, tau = gid & 1;
@@ -112,10 +140,11 @@ __device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, const float
     const bool hv = hl < C::HB;
     const uint16_t* qp = qh + (size_t)(4 * nb + hl) * D;
     float qv[C::NG][8];
-    float mx = 0.0f, ps[C::NG];
+    float mx = 0.0f;
+    int ps[C::NG];
 #pragma unroll
     for (int g = 0; g < C::NG; ++g) {
-      ps[g] = 0.0f;
+      ps[g] = 0;
 #pragma unroll
       for (int kh = 0; kh < 2; ++kh) {
         uint2 u = make_uint2(0u, 0u);
@@ -135,23 +164,36 @@ __device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, const float
     // the four lanes of a quad hold all D channels of one head
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float inv = mx > 0.0f ? kQMax / mx : 0.0f;
-    const float sq = mx * (1.0f / kQMax);
+    constexpr float QM = QT == 3 ? kQMax3 : kQMax;
+    constexpr int QI = (int)QM;
+    const float inv = mx > 0.0f ? QM / mx : 0.0f;
+    const float sq = mx * (1.0f / QM);
 #pragma unroll
     for (int g = 0; g < C::NG; ++g)
 #pragma unroll
       for (int kh = 0; kh < 2; ++kh) {
-        uint32_t packed = 0u;
+        uint32_t packed = 0u, packed3 = 0u;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           int qi = __float2int_rn(qv[g][4 * kh + e] * inv);
-          qi = qi > 32639 ? 32639 : (qi < -32639 ? -32639 : qi);
-          const int q1 = (qi + 128) >> 8;  // floor((qi + 128) / 256)
-          const int q2 = qi - (q1 << 8);   // in [-128, 127]
-          packed |= ((uint32_t)(tau ? q2 : q1) & 0xFFu) << (8 * e);
-          ps[g] += (float)qi;
+          qi = qi > QI ? QI : (qi < -QI ? -QI : qi);
+          if constexpr (QT == 3) {
+            // qi = 65536 q1 + 256 q2 + q3, every term in [-128, 127]
+            const int q3 = ((qi + 128) & 0xFF) - 128;
+            const int r = (qi - q3) >> 8;
+            const int q2 = ((r + 128) & 0xFF) - 128;
+            const int q1 = (r - q2) >> 8;
+            packed |= ((uint32_t)(tau ? q2 : q1) & 0xFFu) << (8 * e);
+            packed3 |= ((uint32_t)(tau ? 0 : q3) & 0xFFu) << (8 * e);
+          } else {
+            const int q1 = (qi + 128) >> 8;  // floor((qi + 128) / 256)
+            const int q2 = qi - (q1 << 8);   // in [-128, 127]
+            packed |= ((uint32_t)(tau ? q2 : q1) & 0xFFu) << (8 * e);
+          }
+          ps[g] += qi;  // exact: |sum| < 2^31
         }
         st.qb[nb][g][kh] = hv ? packed : 0u;
+        if constexpr (QT == 3) st.qb3[nb][g][kh] = hv ? packed3 : 0u;
       }
     // zero-point term: sum of the SAME rounded q_int over each group, so the
     // code and zero terms together are exactly (s c + z) . q_int and the large
@@ -166,7 +208,7 @@ __device__ void setup_query(WarpState<D, G>& st, const uint16_t* qh, const float
     const float sq_c = __shfl_sync(0xffffffffu, sq, 8 * tig);
 #pragma unroll
     for (int g = 0; g < C::NG; ++g) {
-      const float z = __shfl_sync(0xffffffffu, ps[g], 8 * tig);
+      const float z = (float)__shfl_sync(0xffffffffu, ps[g], 8 * tig);  // exact below 2^24 (QT = 2)
       st.qz[nb][g] = make_float2(z, z);
     }
     st.xs[nb] = sq_c * scale_log2;
@@ -212,8 +254,8 @@ __device__ __forceinline__ float half_lo_to_float(uint32_t m) {
 // zero pair of a packed epilogue.  K: pair (i = 2 mb, 2 mb + 1) of group g
 // for tokens gid + 8 i; V: pair (rho = 2 mb, 2 mb + 1) for channels
 // 16 mb + gid and 16 mb + 8 + gid.
-template <int D, int G, int KB, int VB>
-__device__ __forceinline__ void convert_meta(const uint8_t* rec, const WarpState<D, G>& st, float* ks, float* vs,
+template <int D, int G, int KB, int VB, int QT>
+__device__ __forceinline__ void convert_meta(const uint8_t* rec, const WarpState<D, G, QT>& st, float* ks, float* vs,
                                              int lane) {
   using C = Cfg<D, G>;
   const uint32_t* kmeta = reinterpret_cast<const uint32_t*>(rec + blob_bytes(KB, D));
@@ -277,8 +319,8 @@ __device__ __forceinline__ void convert_meta(const uint8_t* rec, const WarpState
 // group's scale/zero apply to that exact integer sum.
 // The epilogue runs on row pairs (tokens gid + 16 mb, gid + 16 mb + 8):
 // acc2[nb][mb] = (score of the first, score of the second).
-template <int D, int G, int KB>
-__device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G>& st, const float* ks,
+template <int D, int G, int KB, int QT>
+__device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G, QT>& st, const float* ks,
                                         float2 (&acc)[Cfg<D, G>::NB][2], int lane) {
   using C = Cfg<D, G>;
   constexpr int W = words_per_lane(KB, D);
@@ -300,9 +342,19 @@ __device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G
 #pragma unroll
       for (int nb = 0; nb < C::NB; ++nb) {
         uint32_t c[4];
-        imma_u8s8(c, a, st.qb[nb][g][0], st.qb[nb][g][1], 0u);
-        // |256 hi + lo| < 2^31: exact in int32, one rounding to fp32 per row
-        const float2 v = make_float2((float)((int)c[0] * 256 + (int)c[1]), (float)((int)c[2] * 256 + (int)c[3]));
+        float2 v;
+        if constexpr (QT == 3) {
+          // terms 1, 2 in one MMA, term 3 in another: 65536 t1 + (256 t2 + t3),
+          // the bracket exact in int32, two roundings in fp32
+          uint32_t c3[4];
+          imma_u8s8(c, a, st.qb[nb][g][0], st.qb[nb][g][1], 0u);
+          imma_u8s8(c3, a, st.qb3[nb][g][0], st.qb3[nb][g][1], 0u);
+          v = make_float2(fmaf(65536.0f, (float)(int)c[0], (float)((int)c[1] * 256 + (int)c3[0])),
+                          fmaf(65536.0f, (float)(int)c[2], (float)((int)c[3] * 256 + (int)c3[2])));
+        } else {
+          imma_u8s8(c, a, st.qb[nb][g][0], st.qb[nb][g][1], kTermC);
+          v = combine_terms(c);
+        }
         acc[nb][mb] = ffma2(make_float2(sz.x, sz.y), v, ffma2(make_float2(sz.z, sz.w), st.qz[nb][g], acc[nb][mb]));
       }
     }
@@ -313,8 +365,8 @@ __device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G
 // moves -- and the state is rescaled -- only when a score of the tile exceeds
 // it, which after the first tiles is rare.  Returns the P B-fragments pb
 // (column n = 2 * head + term, term 0 = high byte).
-template <int D, int G>
-__device__ __forceinline__ void softmax_tile(WarpState<D, G>& st, const float2 (&acc)[Cfg<D, G>::NB][2],
+template <int D, int G, int QT>
+__device__ __forceinline__ void softmax_tile(WarpState<D, G, QT>& st, const float2 (&acc)[Cfg<D, G>::NB][2],
                                              uint32_t (&pb)[Cfg<D, G>::NB][2], int lane) {
   using C = Cfg<D, G>;
   const int gid = lane >> 2, tig = lane & 3;
@@ -377,8 +429,8 @@ __device__ __forceinline__ void softmax_tile(WarpState<D, G>& st, const float2 (
 // P.V of one tile into the running state.  One k32 MMA per 16 channels; the
 // channel's scale/zero apply to the exact integer sum, and the zero term
 // needs sum_t p_t, which one more MMA with A = 1 delivers in the same layout.
-template <int D, int G, int VB>
-__device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st, const float* vs,
+template <int D, int G, int VB, int QT>
+__device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G, QT>& st, const float* vs,
                                         const uint32_t (&pb)[Cfg<D, G>::NB][2], int lane) {
   using C = Cfg<D, G>;
   constexpr int W = words_per_lane(VB, D);
@@ -404,8 +456,8 @@ __device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G>& st
 #pragma unroll
     for (int nb = 0; nb < C::NB; ++nb) {
       uint32_t c[4];
-      imma_u8u8(c, a, pb[nb][0], pb[nb][1], 0u);
-      const float2 v = make_float2((float)((int)c[0] * 256 + (int)c[1]), (float)((int)c[2] * 256 + (int)c[3]));
+      imma_u8u8(c, a, pb[nb][0], pb[nb][1], kTermC);
+      const float2 v = combine_terms(c);
       st.o[nb][mb] = ffma2(make_float2(sz.x, sz.y), v, ffma2(make_float2(sz.z, sz.w), ps[nb], st.o[nb][mb]));
     }
   }
@@ -421,8 +473,8 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
 // own tile records into the ring with 1-D bulk copies (TMA) and re-arms a
 // slot as soon as the warp has read it, so the warp never waits on another
 // warp and every warp keeps `stages` records in flight.
-template <int D, int G, int KB, int VB>
-__device__ void consume(WarpState<D, G>& st, const uint16_t* qh, const float* nrm, float scale_log2, uint8_t* ring,
+template <int D, int G, int KB, int VB, int QT>
+__device__ void consume(WarpState<D, G, QT>& st, const uint16_t* qh, const float* nrm, float scale_log2, uint8_t* ring,
                         int stages,
                         int stage_bytes, uint64_t* bars, float* scratch, const uint8_t* src, int rec, int n_my,
                         int warp, int lane, volatile int* abort_flag, int* status) {
@@ -441,7 +493,7 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, const float* nr
     }
   }
   griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
-  setup_query<D, G, KB, VB>(st, qh, nrm, scale_log2, lane);
+  setup_query<D, G, KB, VB, QT>(st, qh, nrm, scale_log2, lane);
   float* ks = scratch;
   float* vs = scratch + 8 * C::KSTR;
   const int VOFF = blob_bytes(KB, D) + 4 * D;
@@ -452,13 +504,13 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, const float* nr
   for (; j < n_w; ++j) {
     ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], (uint32_t)parity));
     if (!ok) break;
-    convert_meta<D, G, KB, VB>(cur, st, ks, vs, lane);
+    convert_meta<D, G, KB, VB, QT>(cur, st, ks, vs, lane);
     __syncwarp();
     float2 acc[C::NB][2];
-    qk_tile<D, G, KB>(cur, st, ks, acc, lane);
+    qk_tile<D, G, KB, QT>(cur, st, ks, acc, lane);
     uint32_t pb[C::NB][2];
-    softmax_tile<D, G>(st, acc, pb, lane);
-    pv_tile<D, G, VB>(cur + VOFF, st, vs, pb, lane);
+    softmax_tile<D, G, QT>(st, acc, pb, lane);
+    pv_tile<D, G, VB, QT>(cur + VOFF, st, vs, pb, lane);
     __syncwarp();  // every lane has finished reading the slot and the scratch
     if (lane == 0 && j + stages < n_w) {
       fence_proxy_async_smem();  // generic-proxy reads of the slot precede the async refill
@@ -486,14 +538,14 @@ __device__ void consume(WarpState<D, G>& st, const uint16_t* qh, const float* nr
   }
 }
 
-template <int D, int G>
-__device__ __forceinline__ void consume_dispatch(int kb, int vb, WarpState<D, G>& st, const uint16_t* qh,
+template <int D, int G, int QT>
+__device__ __forceinline__ void consume_dispatch(int kb, int vb, WarpState<D, G, QT>& st, const uint16_t* qh,
                                                  const float* nrm, float scale_log2, uint8_t* ring, int stages, int stage_bytes,
                                                  uint64_t* bars, float* scratch, const uint8_t* src, int rec,
                                                  int n_my, int warp, int lane, volatile int* abort_flag,
                                                  int* status) {
 #define RQ_C(KBV, VBV)                                                                                       \
-  consume<D, G, KBV, VBV>(st, qh, nrm, scale_log2, ring, stages, stage_bytes, bars, scratch, src, rec, n_my, warp, \
+  consume<D, G, KBV, VBV, QT>(st, qh, nrm, scale_log2, ring, stages, stage_bytes, bars, scratch, src, rec, n_my, warp, \
                           lane, abort_flag, status)
 #define RQ_V(KBV)                  \
   switch (vb) {                    \
@@ -514,8 +566,8 @@ __device__ __forceinline__ void consume_dispatch(int kb, int vb, WarpState<D, G>
 
 // Canonical partial of one warp in shared memory: o[G][D], m[G], l[G], with
 // o and l back in units of p (the tile path keeps them x 65535).
-template <int D, int G>
-__device__ void dump_tile_state(const WarpState<D, G>& st, float* slot, int lane) {
+template <int D, int G, int QT>
+__device__ void dump_tile_state(const WarpState<D, G, QT>& st, float* slot, int lane) {
   using C = Cfg<D, G>;
   const int gid = lane >> 2, tig = lane & 3;
   constexpr float inv = 1.0f / kPScale;
@@ -788,10 +840,82 @@ __device__ void merge_outputs(const float* base, int n, float* outp, int part, i
   }
 }
 
+// Merge of n partial states (stride PART floats) with four consecutive
+// outputs of one head per thread and the loads of up to U partials in flight:
+// into one more partial state at dst (outp null), or into the normalised
+// outputs at outp.
+template <int D, int G, int U>
+__device__ void merge_quads(const float* base, int n, float* dst, float* outp, int tid) {
+  using C = Cfg<D, G>;
+  for (int qd = tid; qd < G * D / 4; qd += kDecodeThreads) {
+    const int idx = 4 * qd, hh = idx / D;
+    float M = -INFINITY, L = 0.0f;
+    float4 O = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int i0 = 0; i0 < n; i0 += U) {
+      float4 ov[U];
+      float mv[U], lv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const bool ok = i0 + u < n;
+        const float* pp = base + (size_t)(i0 + u) * C::PART;
+        ov[u] = ok ? __ldcg(reinterpret_cast<const float4*>(pp + idx)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        mv[u] = ok ? __ldcg(pp + G * D + hh) : -INFINITY;
+        lv[u] = ok ? __ldcg(pp + G * D + G + hh) : 0.0f;
+      }
+      float nm = M;
+#pragma unroll
+      for (int u = 0; u < U; ++u) nm = fmaxf(nm, mv[u]);
+      if (nm == -INFINITY) continue;
+      const float sc = ex2(M - nm);  // 0 while M = -inf
+      O.x *= sc, O.y *= sc, O.z *= sc, O.w *= sc;
+      L *= sc;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float f = ex2(mv[u] - nm);
+        O.x = fmaf(ov[u].x, f, O.x), O.y = fmaf(ov[u].y, f, O.y);
+        O.z = fmaf(ov[u].z, f, O.z), O.w = fmaf(ov[u].w, f, O.w);
+        L = fmaf(lv[u], f, L);
+      }
+      M = nm;
+    }
+    if (outp != nullptr) {
+      const bool any = L > 0.0f;
+      *reinterpret_cast<float4*>(outp + idx) =
+          make_float4(any ? O.x / L : 0.0f, any ? O.y / L : 0.0f, any ? O.z / L : 0.0f, any ? O.w / L : 0.0f);
+    } else {
+      *reinterpret_cast<float4*>(dst + idx) = O;
+      if (idx % D == 0) {
+        dst[G * D + hh] = M;
+        dst[G * D + G + hh] = L;
+      }
+    }
+  }
+}
+
+// Tile work item: the warps stream and process their tiles, then (after every
+// stage read has completed, so the merge area may alias the stages) leave
+// their partial states in the warp slots.
+template <int D, int G, int QT>
+__device__ __forceinline__ void tile_item(const DecodeArgs& a, const HeadDesc& hd, const uint16_t* qh,
+                                          const float* nrm, uint8_t* area, uint8_t* smem, float* merge,
+                                          uint64_t* bars, const uint8_t* src, int rec, int n_my, int warp, int lane,
+                                          volatile int* abort_flag) {
+  using C = Cfg<D, G>;
+  WarpState<D, G, QT> st;
+  consume_dispatch<D, G, QT>(hd.k_bits, hd.v_bits, st, qh, nrm, a.scale_log2,
+                             area + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
+                             bars + warp * kMaxStages, reinterpret_cast<float*>(smem) + warp * C::SCRATCH, src, rec,
+                             n_my, warp, lane, abort_flag, a.status);
+  __syncthreads();
+  if (!*abort_flag) dump_tile_state<D, G, QT>(st, merge + warp * C::PART, lane);
+}
+
 // CL = CTAs per thread-block cluster (kDecodeCluster, or 1: no cluster); the
 // cluster shape is given at launch.
-template <int D, int G, int CL>
-__global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_kernel(DecodeArgs a) {
+// QT: s8 terms of the fixed-point query (2, or 3 for K-normalized caches); a
+// separate instantiation so that the 16-bit path keeps its register budget.
+template <int D, int G, int CL, int QT>
+__global__ void __launch_bounds__(kDecodeThreads, QT == 3 ? 3 : RQ_DECODE_MIN_BLOCKS) decode_kernel(DecodeArgs a) {
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[NW * kMaxStages];
@@ -820,21 +944,15 @@ __global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_k
   }
   __syncthreads();
 
-  WarpState<D, G> st;
   const bool tiles_item = item < a.n_splits;
   if (tiles_item) {
     const int t0 = (int)(((int64_t)item * a.n_tiles) / a.n_splits);
     const int t1 = (int)(((int64_t)(item + 1) * a.n_tiles) / a.n_splits);
     const int rec = hd.rec_bytes;
     const uint8_t* src = a.buf + hd.tile_base + (int64_t)b * hd.tile_stride + (int64_t)t0 * rec;
-    if (warp < NW)
-      consume_dispatch<D, G>(hd.k_bits, hd.v_bits, st, qh,
-                             reinterpret_cast<const float*>(a.buf + hd.win_base + (int64_t)b * a.g.win_bytes +
-                                                            window_rows_bytes(a.g.S, a.g.R, D)),
-                             a.scale_log2,
-                             area + (size_t)warp * a.stages * a.stage_bytes, a.stages, a.stage_bytes,
-                             bars + warp * kMaxStages, reinterpret_cast<float*>(smem) + warp * C::SCRATCH, src, rec,
-                             t1 - t0, warp, lane, &abort_flag, a.status);
+    const float* nrm = reinterpret_cast<const float*>(a.buf + hd.win_base + (int64_t)b * a.g.win_bytes +
+                                                      window_rows_bytes(a.g.S, a.g.R, D));
+    tile_item<D, G, QT>(a, hd, qh, nrm, area, smem, merge, bars, src, rec, t1 - t0, warp, lane, &abort_flag);
   } else if (a.n_pack && item == a.n_splits + a.n_win) {
     pack_item<D, G>(a, hd, b, area, merge, tid);
   } else {
@@ -845,8 +963,6 @@ __global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_k
     window_item<D, G>(a, win, qh, knew_off, item - a.n_splits, merge + NW * C::PART, &bars[0],
                       merge + warp * C::PART, warp, lane, &abort_flag);
   }
-  __syncthreads();  // every stage read has completed; merge may now alias the stages
-  if (tiles_item && warp < NW && !abort_flag) dump_tile_state<D, G>(st, merge + warp * C::PART, lane);
   __syncthreads();
   const bool valid = !abort_flag;
 
@@ -879,7 +995,7 @@ __global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_k
   // shared memory (CL = 1: the CTA stores its own partial).  Every CTA passes
   // both cluster barriers on every path (no early exit before them).
   namespace cg = cooperative_groups;
-  float* ps = a.partials + (size_t)srel * NI * C::PART;
+  float* ps = a.partials + (size_t)srel * partial_slots(NI) * C::PART;
   const int ncl = (int)gridDim.x / CL;
   int crank = 0;
   if constexpr (CL > 1) {
@@ -920,6 +1036,37 @@ __global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_k
     __syncthreads();  // the item partial is complete in shared memory
     float* cp = ps + (size_t)item * C::PART;
     for (int idx = tid; idx < C::PART; idx += blockDim.x) cp[idx] = mypart[idx];
+    const int ngr = merge_groups(NI);
+    if (ngr > 0) {
+      // two levels: the last item of each group of kMergeGroup merges the
+      // group into partial slot NI + group; the last group merger merges the
+      // group partials into the output
+      const int grp = item / kMergeGroup;
+      const int gsize = min(kMergeGroup, NI - grp * kMergeGroup);
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {
+        uint32_t* gc = &a.counters[(size_t)srel * kCountersPerStream + 1 + grp];
+        const int last_g = atomicAdd(gc, 1u) == (unsigned)(gsize - 1);
+        if (last_g) *gc = 0u;  // every item of the group has counted: reset for the next call
+        is_last = last_g;
+      }
+      __syncthreads();
+      if (!is_last) return;
+      __threadfence();
+      merge_quads<D, G, kMergeGroup>(ps + (size_t)grp * kMergeGroup * C::PART, gsize, ps + (size_t)(NI + grp) * C::PART,
+                                     nullptr, tid);
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) is_last = atomicAdd(&a.counters[(size_t)srel * kCountersPerStream], 1u) == (unsigned)(ngr - 1);
+      __syncthreads();
+      if (!is_last) return;
+      __threadfence();
+      float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
+      merge_quads<D, G, 12>(ps + (size_t)NI * C::PART, ngr, nullptr, outp, tid);
+      if (tid == 0) a.counters[(size_t)srel * kCountersPerStream] = 0u;
+      return;
+    }
   }
   // the first CTA publishes the cluster partial and learns whether its
   // cluster is the stream's last; it tells every CTA of the cluster
@@ -947,7 +1094,11 @@ __global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_k
   // slice of the outputs
   __threadfence();
   float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
-  merge_outputs<D, G, CL>(ps, ncl, outp, crank, tid);
+  if constexpr (CL > 1) {
+    merge_outputs<D, G, CL>(ps, ncl, outp, crank, tid);
+  } else {
+    merge_quads<D, G, kMergeGroup>(ps, ncl, nullptr, outp, tid);
+  }
   if (crank == 0 && tid == 0) a.counters[(size_t)srel * kCountersPerStream] = 0u;
 }
 
@@ -956,25 +1107,25 @@ __global__ void __launch_bounds__(kDecodeThreads, RQ_DECODE_MIN_BLOCKS) decode_k
 // (device, D, G, cluster, size), and querying them on every call costs more
 // host time than a decode step.
 std::mutex g_attr_mu;
-std::map<std::tuple<int, int, int, int>, int> g_smem_set;        // (dev, D, G, CL) -> largest size set
-std::map<std::tuple<int, int, int, int, int>, int> g_resident;   // (dev, D, G, CL, smem) -> CTAs
+std::map<std::tuple<int, int, int, int, int>, int> g_smem_set;       // (dev, D, G, CL, QT) -> largest size set
+std::map<std::tuple<int, int, int, int, int, int>, int> g_resident;  // (dev, D, G, CL, QT, smem) -> CTAs
 
-template <int D, int G, int CL>
+template <int D, int G, int CL, int QT>
 cudaError_t ensure_smem(int smem) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_attr_mu);
-  int& cur = g_smem_set[std::make_tuple(dev, D, G, CL)];
+  int& cur = g_smem_set[std::make_tuple(dev, D, G, CL, QT)];
   if (cur >= smem) return cudaSuccess;
-  e = cudaFuncSetAttribute(decode_kernel<D, G, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(decode_kernel<D, G, CL, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) cur = smem;
   return e;
 }
 
-template <int D, int G, int CL>
+template <int D, int G, int CL, int QT>
 cudaError_t launch_dgc(const DecodeArgs& a, int smem, cudaStream_t st) {
-  cudaError_t e = ensure_smem<D, G, CL>(smem);
+  cudaError_t e = ensure_smem<D, G, CL, QT>(smem);
   if (e != cudaSuccess) return e;
   const int streams = a.n_layers * a.g.B * a.g.Hkv;
   cudaLaunchConfig_t cfg = {};
@@ -994,29 +1145,31 @@ cudaError_t launch_dgc(const DecodeArgs& a, int smem, cudaStream_t st) {
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G, CL>, a);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G, CL, QT>, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int smem, cudaStream_t st) {
-  if (a.cluster == 1) return launch_dgc<D, G, 1>(a, smem, st);
-  if (a.cluster == kDecodeCluster) return launch_dgc<D, G, kDecodeCluster>(a, smem, st);
+  const bool q3 = a.q_terms == 3;
+  if (a.cluster == 1) return q3 ? launch_dgc<D, G, 1, 3>(a, smem, st) : launch_dgc<D, G, 1, 2>(a, smem, st);
+  if (a.cluster == kDecodeCluster)
+    return q3 ? launch_dgc<D, G, kDecodeCluster, 3>(a, smem, st) : launch_dgc<D, G, kDecodeCluster, 2>(a, smem, st);
   return cudaErrorInvalidValue;
 }
 
 // CTAs of the decode kernel that the device holds at once, in whole clusters.
-template <int D, int G, int CL>
+template <int D, int G, int CL, int QT>
 int resident_ctas_dgc(int smem) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return CL;
   {
     std::lock_guard<std::mutex> lock(g_attr_mu);
-    auto it = g_resident.find(std::make_tuple(dev, D, G, CL, smem));
+    auto it = g_resident.find(std::make_tuple(dev, D, G, CL, QT, smem));
     if (it != g_resident.end()) return it->second;
   }
-  if (ensure_smem<D, G, CL>(smem) != cudaSuccess) return CL;
+  if (ensure_smem<D, G, CL, QT>(smem) != cudaSuccess) return CL;
   int n = 0;
   if (CL > 1) {
     cudaLaunchConfig_t cfg = {};
@@ -1030,24 +1183,26 @@ int resident_ctas_dgc(int smem) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<D, G, CL>, &cfg) != cudaSuccess || n < 1) return CL;
+    if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<D, G, CL, QT>, &cfg) != cudaSuccess || n < 1) return CL;
     n *= CL;
   } else {
     int per_sm = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<D, G, CL>, kDecodeThreads, smem) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<D, G, CL, QT>, kDecodeThreads, smem) !=
             cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || per_sm < 1 || sms < 1)
       return 1;
     n = per_sm * sms;
   }
   std::lock_guard<std::mutex> lock(g_attr_mu);
-  g_resident[std::make_tuple(dev, D, G, CL, smem)] = n;
+  g_resident[std::make_tuple(dev, D, G, CL, QT, smem)] = n;
   return n;
 }
 
 template <int D, int G>
-int resident_ctas_dg(int cluster, int smem) {
-  return cluster == 1 ? resident_ctas_dgc<D, G, 1>(smem) : resident_ctas_dgc<D, G, kDecodeCluster>(smem);
+int resident_ctas_dg(int cluster, int smem, int q_terms) {
+  if (q_terms == 3)
+    return cluster == 1 ? resident_ctas_dgc<D, G, 1, 3>(smem) : resident_ctas_dgc<D, G, kDecodeCluster, 3>(smem);
+  return cluster == 1 ? resident_ctas_dgc<D, G, 1, 2>(smem) : resident_ctas_dgc<D, G, kDecodeCluster, 2>(smem);
 }
 
 }  // namespace
@@ -1057,7 +1212,7 @@ int resident_ctas_dg(int cluster, int smem) {
 template <int D, int G>
 cudaError_t launch_decode_dg(const DecodeArgs& a, int smem, cudaStream_t st);
 template <int D, int G>
-int decode_resident_ctas_dg(int cluster, int smem);
+int decode_resident_ctas_dg(int cluster, int smem, int q_terms);
 
 }  // namespace rq
 
@@ -1068,7 +1223,7 @@ int decode_resident_ctas_dg(int cluster, int smem);
     return launch_dg<DD, GG>(a, smem, st);                                                 \
   }                                                                                        \
   template <>                                                                              \
-  int decode_resident_ctas_dg<DD, GG>(int cluster, int smem) {                             \
-    return resident_ctas_dg<DD, GG>(cluster, smem);                                        \
+  int decode_resident_ctas_dg<DD, GG>(int cluster, int smem, int q_terms) {                \
+    return resident_ctas_dg<DD, GG>(cluster, smem, q_terms);                               \
   }                                                                                        \
   }

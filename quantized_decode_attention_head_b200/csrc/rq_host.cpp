@@ -108,11 +108,25 @@ int max_record(const rq_cache* c, int l0, int nl) {
 // stream's last cluster.  Several waves: single-CTA items of about
 // kWaveTilesPerItem tiles (more when the slots allow), so that no CTA holds
 // a slot at a cluster barrier while the others of its cluster still work.
+#ifndef RQ_BALANCED
+#define RQ_BALANCED 0
+#endif
 int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win, int* cluster) {
   *cluster = rq::kDecodeCluster;
   if (n_tiles <= 0) return 0;
   const int smem = rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes), stage_bytes, c->g.G, c->g.D);
-  const long slots = rq::decode_resident_ctas(c->g.D, c->g.G, rq::kDecodeCluster, smem);
+  if (RQ_BALANCED) {
+    // one wave of single-CTA items filling every resident slot
+    const long slots1 = rq::decode_resident_ctas(c->g.D, c->g.G, 1, smem, c->k_norm ? 3 : 2);
+    if (slots1 / streams >= 2 + n_win) {
+      *cluster = 1;
+      long s = slots1 / streams - n_win;
+      if (s > n_tiles) s = n_tiles;
+      if (s > rq::kMaxItems - n_win) s = rq::kMaxItems - n_win;
+      return (int)s;
+    }
+  }
+  const long slots = rq::decode_resident_ctas(c->g.D, c->g.G, rq::kDecodeCluster, smem, c->k_norm ? 3 : 2);
   const long per = (slots / streams) / rq::kDecodeCluster * rq::kDecodeCluster;
   const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;  // keep a CTA's pipeline busy
   long s;
@@ -120,7 +134,7 @@ int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, in
     s = per - n_win;
   } else {
     *cluster = 1;
-    const long slots1 = rq::decode_resident_ctas(c->g.D, c->g.G, 1, smem);
+    const long slots1 = rq::decode_resident_ctas(c->g.D, c->g.G, 1, smem, c->k_norm ? 3 : 2);
     s = (n_tiles + rq::kWaveTilesPerItem - 1) / rq::kWaveTilesPerItem;
     if (slots1 / streams - n_win > s) s = slots1 / streams - n_win;
   }
@@ -176,6 +190,9 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   a.pack_pos = 0;
   a.pack_tile = 0;
   a.n_streams = streams;
+  // K-normalized caches fold the channel factors into the query, which widens
+  // its range: 24-bit fixed point there, 16-bit otherwise
+  a.q_terms = c->k_norm ? 3 : 2;
   a.stages = rq::decode_stages(stage_bytes);
   a.stage_bytes = stage_bytes;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -480,7 +497,9 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
     const size_t avail = rq::kNoAllocScratchBytes > rq::ws_partial_offset(all_streams)
                              ? rq::kNoAllocScratchBytes - rq::ws_partial_offset(all_streams)
                              : 0;
-    int64_t items = (int64_t)avail / (streams * (int64_t)(c->g.G * c->g.D + 2 * c->g.G) * 4);
+    const int64_t slots = (int64_t)avail / (streams * (int64_t)rq::partial_floats(c->g.G, c->g.D) * 4);
+    int64_t items = slots;
+    while (items > 0 && rq::partial_slots((int)items) > slots) --items;
     items = items / cluster * cluster;
     const int64_t s = items - rq::window_items(c->length[l0], c->g.S, c->g.R);
     if (s >= 1)

@@ -91,6 +91,7 @@ struct DecodeArgs {
   int pack_tile;
   int n_streams;          // streams of this call
   int cluster;            // CTAs per thread-block cluster: kDecodeCluster or 1
+  int q_terms;            // s8 terms of the fixed-point query: 2 (16 bits) or 3 (24 bits, K-normalized caches)
   int stages;             // per-warp ring depth (2..8)
   int stage_bytes;        // bytes per stage (max record size in the call)
   float* partials;        // [streams][n_splits+1][G*D + 2G]
@@ -125,17 +126,31 @@ __host__ __device__ inline int cluster_items(int items, int cluster) {
   return (items + cluster - 1) / cluster * cluster;
 }
 
+// Floats of one partial softmax state (o[G][D], m[G], l[G]), padded to a
+// multiple of four so that every partial starts on a 16-byte boundary.
+__host__ __device__ constexpr int partial_floats(int G, int D) { return (G * D + 2 * G + 3) / 4 * 4; }
+// Single-CTA items (cluster 1) of a stream merge in groups of kMergeGroup:
+// the last item of a group to finish merges the group into one more partial,
+// the last group merger merges the group partials into the output.
+constexpr int kMergeGroup = 8;
+__host__ __device__ inline int merge_groups(int items) {
+  return items > kMergeGroup ? (items + kMergeGroup - 1) / kMergeGroup : 0;
+}
+// partial slots of one stream: one per item plus one per merge group
+__host__ __device__ inline int partial_slots(int items) { return items + merge_groups(items); }
+
 // Workspace layout (bytes): [status int32, pad to 256][kCountersPerStream u32
-// counters per stream of the whole cache (L*B*Hkv)][partials of one call:
-// [stream][item][G*D + 2G] floats = o, m, l (cluster partials use the first
-// items' slots)].  The counter region is sized for every stream so calls
-// with different layer arguments never overlap.
+// counters per stream of the whole cache (L*B*Hkv): [0] items or groups
+// merged, [1 + group] items of a merge group finished][partials of one call:
+// [stream][partial_slots(items)][partial_floats(G, D)] = o, m, l (cluster
+// partials use the first items' slots)].  The counter region is sized for
+// every stream so calls with different layer arguments never overlap.
 inline size_t ws_counter_offset() { return 256; }
 inline size_t ws_partial_offset(int64_t all_streams) {
   return ws_counter_offset() + (size_t)all_streams * kCountersPerStream * 4;
 }
 inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int items, int G, int D) {
-  return ws_partial_offset(all_streams) + (size_t)call_streams * items * (size_t)(G * D + 2 * G) * 4;
+  return ws_partial_offset(all_streams) + (size_t)call_streams * partial_slots(items) * (size_t)partial_floats(G, D) * 4;
 }
 // bf16 window tokens of a T-token cache and the number of window work items
 // (kWinChunksPerItem chunks of 32 tokens each; at least one item)
@@ -160,7 +175,7 @@ cudaError_t launch_decode(const DecodeArgs& a, int smem_bytes, cudaStream_t s);
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D);
 // CTAs of the decode kernel resident on the device at once, in whole clusters
 // of `cluster` CTAs
-int decode_resident_ctas(int D, int G, int cluster, int smem_bytes);
+int decode_resident_ctas(int D, int G, int cluster, int smem_bytes, int q_terms);
 
 // One-thread kernel whose bounded mbarrier wait runs out after limit_ns and
 // records kDeviceTimeout in *status (self-test of the timeout path).

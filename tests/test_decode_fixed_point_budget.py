@@ -22,7 +22,8 @@ from oracle import cache as ca
 from oracle import quantize as qz
 from quantized_decode_attention_head_b200 import workloads
 
-QMAX = 32639.0
+QMAX = 32639.0        # 16-bit query (two s8 terms)
+QMAX3 = 8323072.0     # 24-bit query of K-normalized caches (three s8 terms)
 PSCALE = 65535.0
 LOG2E = 1.4426950408889634
 
@@ -31,7 +32,7 @@ def _bf16_to_f64(t):
     return qz.bf16_bits_to_f32(t.contiguous().view(torch.int16).numpy().view(np.uint16)).astype(np.float64)
 
 
-def _emulated_decode(q, kh, vh, S, Tq, n_splits, n_warps=4, rounding=True, nrm=None):
+def _emulated_decode(q, kh, vh, S, Tq, n_splits, n_warps=4, rounding=True, nrm=None, qmax=QMAX):
     """Output [G, D] of the kernel's arithmetic model for one stream
     (rounding=False: q_int and p_int left unrounded).  nrm: the K
     normalization factors of a normalized cache -- the tiles hold K / n and
@@ -43,9 +44,9 @@ def _emulated_decode(q, kh, vh, S, Tq, n_splits, n_warps=4, rounding=True, nrm=N
     n = np.ones(D) if nrm is None else np.asarray(nrm, dtype=np.float64)
     q32 = (q * n).astype(np.float32)
     mx = np.abs(q32).max(axis=1, keepdims=True)
-    inv = np.where(mx > 0, np.float32(QMAX) / mx, np.float32(0)).astype(np.float32)
-    q_int = np.clip(rint((q32 * inv).astype(np.float64)), -QMAX, QMAX)
-    sq = (mx.astype(np.float64) / QMAX)[:, 0]
+    inv = np.where(mx > 0, np.float32(qmax) / mx, np.float32(0)).astype(np.float32)
+    q_int = np.clip(rint((q32 * inv).astype(np.float64)), -qmax, qmax)
+    sq = (mx.astype(np.float64) / qmax)[:, 0]
     n_tiles = Tq // 32
     x_tiles = ((kh[S:S + Tq] / n) @ q_int.T) * sq * scale * LOG2E  # base-2 logits [Tq, G]
     parts = []  # (m [G], l [G], o [G, D])
@@ -116,13 +117,19 @@ def test_fixed_point_model_is_exact_without_rounding():
 
 
 def test_k_norm_fixed_point_error_budget():
-    """A normalized cache (K / n in the tiles, q * n in the tile products) at
-    outlier sigma = 1.0, the setting of the GPU parity test for normalized
-    caches: the query's 16-bit fixed point now spans every channel's
-    magnitude, and the error still stays under half the tolerance."""
-    wl, q, kh, vh, st = _stream("long_128k", 2, k_norm=True, k_sigma=1.0)
-    got = _emulated_decode(q, kh, vh, wl.n_sink, st.n_tiles * 32, n_splits=66, nrm=st.nrm)
+    """A normalized cache (K / n in the tiles, q * n in the tile products) on
+    the long-context workload itself (outlier sigma = 1.5): the query's fixed
+    point now spans every channel's magnitude.  With the 24-bit query the
+    kernel uses for normalized caches the error stays far under half the
+    tolerance; a 16-bit query would lose more than ten times as much (the
+    reason normalized caches take the three-term query)."""
+    wl, q, kh, vh, st = _stream("long_128k", 2, k_norm=True)
+    assert wl.k_sigma == 1.5
     exp = at.attend(q, kh, vh)
+    got = _emulated_decode(q, kh, vh, wl.n_sink, st.n_tiles * 32, n_splits=66, nrm=st.nrm, qmax=QMAX3)
     err = np.abs(got - exp).max()
     rel = np.linalg.norm(got - exp) / np.linalg.norm(exp)
     assert err < 1e-3 and rel < 5e-4, (err, rel)
+    got16 = _emulated_decode(q, kh, vh, wl.n_sink, st.n_tiles * 32, n_splits=66, nrm=st.nrm, qmax=QMAX)
+    err16 = np.abs(got16 - exp).max()
+    assert err16 > 10 * err, (err16, err)

@@ -114,3 +114,41 @@ def test_long_context_named_split_counts():
     assert QuantizedKVCache.rq_decode_read_status(ws) == 0
     for h, s in streams.items():
         check_stream_bytes(cache, s, 0, 0, h)
+
+
+def test_long_context_k_norm():
+    """The long-context workload (outlier sigma 1.5) as a K-normalized cache:
+    the factors, sampled streams' records and windows bit for bit, and the
+    decoded heads of three streams within the parity tolerance after the
+    prefill and after a fused step (24-bit query)."""
+    wl = workloads.CONFIGS["long_128k"]
+    (kb, vb), (okb, ovb) = workload_bits(wl)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, wl.context + 1, k_norm=True)
+    cache.rq_quantize_kv(k, v)
+    q, kn, vn = workloads.step_inputs(wl, 2, f, "cuda")
+    heads = (0, 3, 7)
+    streams = {}
+    for h in heads:
+        s = ca.StreamCache(wl.head_dim, int(okb[0, h]), int(ovb[0, h]), wl.n_sink, wl.n_recent, k_norm=True)
+        s.prefill(to_f32(k[0, 0, h]), to_f32(v[0, 0, h]))
+        streams[h] = s
+    del k, v
+    torch.cuda.empty_cache()
+    G = wl.group
+    ws = cache.make_workspace()
+    out = cache.rq_decode_attention(0, q[0, 0].contiguous(), workspace=ws).cpu().numpy()
+    for h, s in streams.items():
+        kh, vh = s.dequantized()
+        e = at.attend(to_f32(q[0, 0, 0, h * G:(h + 1) * G]).astype(np.float64), kh, vh)
+        assert_close(out[0, h * G:(h + 1) * G], e, f"k_norm prefill, kv-head {h}")
+    out = cache.rq_decode_step(0, q[1, 0].contiguous(), kn[1, 0].contiguous(), vn[1, 0].contiguous(),
+                               workspace=ws).cpu().numpy()
+    for h, s in streams.items():
+        s.append(to_f32(kn[1, 0, 0, h]), to_f32(vn[1, 0, 0, h]))
+        kh, vh = s.dequantized()
+        e = at.attend(to_f32(q[1, 0, 0, h * G:(h + 1) * G]).astype(np.float64), kh, vh)
+        assert_close(out[0, h * G:(h + 1) * G], e, f"k_norm fused step, kv-head {h}")
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+    for h, s in streams.items():
+        check_stream_bytes(cache, s, 0, 0, h)
