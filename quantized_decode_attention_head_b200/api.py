@@ -13,11 +13,15 @@ import numpy as np
 from ._lib import CacheConfig, check, lib
 
 
-def _stream_ptr(stream=None):
+def _stream_ptr(stream=None, device=None):
+    """The raw cudaStream_t of `stream`, or of the current stream of `device`
+    (default: the current device)."""
     import torch
 
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
+    idx = torch.cuda.current_device() if device is None else device
+    return ctypes.c_void_p(torch._C._cuda_getCurrentRawStream(idx))
 
 
 def _dptr(t):
@@ -27,6 +31,10 @@ def _dptr(t):
 def _check_tensor(name, t, dtype, shape=None, device_type="cuda"):
     import torch
 
+    # one cheap test on the common path; the detailed message only on failure
+    if (isinstance(t, torch.Tensor) and t.dtype is dtype and t.is_cuda == (device_type == "cuda")
+            and t.is_contiguous() and (shape is None or t.shape == tuple(shape))):
+        return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
@@ -35,8 +43,7 @@ def _check_tensor(name, t, dtype, shape=None, device_type="cuda"):
         raise ValueError(f"{name} must be on {device_type}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if shape is not None and tuple(t.shape) != tuple(shape):
-        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
 def rq_allocate_bits(w, alpha, beta, avg_bits, allowed):
@@ -232,7 +239,7 @@ class QuantizedKVCache:
             workspace = self.make_workspace(n_splits, stream)
         check("rq_decode_attention", lib().rq_decode_attention(
             self.handle, layer, _dptr(q), _dptr(out), float(softmax_scale), int(n_splits), _dptr(workspace),
-            workspace.numel(), _stream_ptr(stream)))
+            workspace.numel(), _stream_ptr(stream, q.get_device())))
         return out
 
     def rq_decode_step(self, layer, q, k_new, v_new, out=None, softmax_scale=0.0, n_splits=0, workspace=None,
@@ -258,7 +265,7 @@ class QuantizedKVCache:
             workspace = self.make_workspace(n_splits, stream)
         check("rq_decode_step", lib().rq_decode_step(
             self.handle, layer, _dptr(q), _dptr(k_new), _dptr(v_new), _dptr(out), float(softmax_scale),
-            int(n_splits), _dptr(workspace), workspace.numel(), _stream_ptr(stream)))
+            int(n_splits), _dptr(workspace), workspace.numel(), _stream_ptr(stream, q.get_device())))
         return out
 
     @staticmethod

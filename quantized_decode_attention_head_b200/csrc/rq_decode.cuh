@@ -95,6 +95,11 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(
 #ifndef RQ_CVT_BIAS
 #define RQ_CVT_BIAS 0
 #endif
+// tile records per warp prefetched into L2 (beyond its ring) before the
+// launch waits for its predecessor
+#ifndef RQ_L2_AHEAD
+#define RQ_L2_AHEAD 0
+#endif
 // C operand of the two-term MMAs: 0 (int32 results) or the bits of 1.5 * 2^23
 // (each result, read as a float, is 1.5 * 2^23 + the exact integer sum).
 constexpr uint32_t kTermC = RQ_CVT_BIAS ? kBiasBits : 0u;
@@ -491,6 +496,12 @@ __device__ void consume(WarpState<D, G, QT>& st, const uint16_t* qh, const float
       bulk_g2s_hint(ring + (size_t)j * stage_bytes, src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec, &bars[j],
                     policy);
     }
+  }
+  // the next few records into L2 as well, so that while the previous launch
+  // finishes (its merge tail), this one keeps HBM busy
+  if (RQ_L2_AHEAD > 0 && lane < RQ_L2_AHEAD) {
+    const int j = stages + lane;
+    if (j < n_w) l2_prefetch(src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec);
   }
   griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
   setup_query<D, G, KB, VB, QT>(st, qh, nrm, scale_log2, lane);

@@ -90,25 +90,94 @@ __device__ __forceinline__ uint32_t code_of(float x, float z, float r) {
   return (uint32_t)c;
 }
 
+// The same rule on two elements at once: c = min(rint((x - z) * r), 2^B - 1)
+// with x - z and the product each one fp32 operation rounded to nearest
+// (packed pairs), and rint done by adding 1.5 * 2^23: for 0 <= y < 2^22 the
+// sum rounds to y's nearest integer (ties to even) + 1.5 * 2^23 exactly.
+// x >= z holds for every element of its group (z is the group minimum, or
+// -M), so y >= 0 and only the top clamp applies (it binds only for
+// subnormal or saturated fp16 scales; larger y round wrongly but clamp).
+// Returns the sums' bit patterns, the code in the low byte.
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+template <int B>
+__device__ __forceinline__ uint2 codes2(float2 x, float2 nz, float2 r) {
+  constexpr uint32_t kTop = 0x4B400000u + (1u << B) - 1u;
+  const float2 y = __fmul2_rn(__fadd2_rn(x, nz), r);
+  const float2 m = __fadd2_rn(y, make_float2(kRound, kRound));
+  return make_uint2(min(__float_as_uint(m.x), kTop), min(__float_as_uint(m.y), kTop));
+}
+
+// Four codes (low bytes of the code_of2 results) into the four bytes of one
+// register, byte e = code e.
+__device__ __forceinline__ uint32_t code_bytes(uint2 c01, uint2 c23) {
+  return __byte_perm(__byte_perm(c01.x, c01.y, 0x0040), __byte_perm(c23.x, c23.y, 0x0040), 0x5410);
+}
+
+// Places register (rho, kh) -- byte e holding code e -- into the lane's words.
+template <int B, int W>
+__device__ __forceinline__ void put_reg(uint32_t* words, int rho, int kh, uint32_t reg) {
+  const int j = reg_class(B, rho), sgm = reg_source(B, rho, kh);
+  if (B == 3 && sgm >= W) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) put_code<B, W>(words, rho, kh, e, (reg >> (8 * e)) & 0xFFu);
+  } else {
+    words[sgm] |= reg << (B * j);
+  }
+}
+
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) { return make_float2(lo_bf16(w), hi_bf16(w)); }
+
+// Minimum and maximum of a group of 32 bf16 values held as 16 pairs, compared
+// as bf16x2 (exact: widening bf16 to fp32 keeps the order).
+__device__ __forceinline__ void minmax_pairs(uint32_t& mnw, uint32_t& mxw, uint32_t w) {
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&w);
+  __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&mnw), hi = *reinterpret_cast<const __nv_bfloat162*>(&mxw);
+  lo = __hmin2(lo, a);
+  hi = __hmax2(hi, a);
+  mnw = *reinterpret_cast<const uint32_t*>(&lo);
+  mxw = *reinterpret_cast<const uint32_t*>(&hi);
+}
+__device__ __forceinline__ float min_of_pair(uint32_t w) { return fminf(lo_bf16(w), hi_bf16(w)); }
+__device__ __forceinline__ float max_of_pair(uint32_t w) { return fmaxf(lo_bf16(w), hi_bf16(w)); }
+
 // KN: multiply by the K normalization factors 1/n (false: n = 1, skipped).
 template <int D, int KB, bool KN>
 __device__ void pack_k(HalfTile<D>& sm, const float* kinv, uint8_t* rec, int lane, bool hybrid) {
   constexpr int NG = D / 32;
   constexpr int W = words_per_lane(KB, D);
-  // statistics: lane = token, rotated word order spreads smem banks
+  // statistics: lane = token; 16-byte row reads (the padded row stride puts
+  // the eight lanes of a phase on distinct banks)
   {
     const int t = lane;
 #pragma unroll
     for (int grp = 0; grp < NG; ++grp) {
-      float mn = INFINITY, mx = -INFINITY;
+      float mn, mx;
+      if constexpr (KN) {
+        mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int cw = grp * 16 + ((c + (t >> 3)) & 15);
-        const uint32_t w = sm.x[t][cw];
-        const float x0 = KN ? lo_bf16(w) * kinv[2 * cw] : lo_bf16(w);
-        const float x1 = KN ? hi_bf16(w) * kinv[2 * cw + 1] : hi_bf16(w);
-        mn = fminf(mn, fminf(x0, x1));
-        mx = fmaxf(mx, fmaxf(x0, x1));
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const uint4 u = *reinterpret_cast<const uint4*>(&sm.x[t][grp * 16 + 4 * c4]);
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int cw = grp * 16 + 4 * c4 + k;
+            const float x0 = lo_bf16(w4[k]) * kinv[2 * cw], x1 = hi_bf16(w4[k]) * kinv[2 * cw + 1];
+            mn = fminf(mn, fminf(x0, x1));
+            mx = fmaxf(mx, fmaxf(x0, x1));
+          }
+        }
+      } else {
+        uint32_t mnw = sm.x[t][grp * 16], mxw = mnw;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const uint4 u = *reinterpret_cast<const uint4*>(&sm.x[t][grp * 16 + 4 * c4]);
+          minmax_pairs(mnw, mxw, u.x);
+          minmax_pairs(mnw, mxw, u.y);
+          minmax_pairs(mnw, mxw, u.z);
+          minmax_pairs(mnw, mxw, u.w);
+        }
+        mn = min_of_pair(mnw);
+        mx = max_of_pair(mxw);
       }
       float r;
       const uint32_t meta = group_params<KB>(mn, mx, r, hybrid);
@@ -125,18 +194,23 @@ __device__ void pack_k(HalfTile<D>& sm, const float* kinv, uint8_t* rec, int lan
   for (int w = 0; w < W; ++w) words[w] = 0;
   // register (rho, kh), byte e: token gid + 8i, channel 32g + 16kh + 4tig + e
 #pragma unroll
-  for (int rho = 0; rho < D / 8; ++rho)
+  for (int rho = 0; rho < D / 8; ++rho) {
+    const int i = rho / NG, g = rho % NG;
+    const int t = gid + 8 * i;
+    const float r1 = sm.r[t * NG + g], z1 = sm.z[t * NG + g];
+    const float2 rr = make_float2(r1, r1), nz = make_float2(-z1, -z1);
 #pragma unroll
-    for (int kh = 0; kh < 2; ++kh)
-#pragma unroll
-      for (int e = 0; e < 4; e += 2) {
-        const int i = rho / NG, g = rho % NG;
-        const int t = gid + 8 * i, d0 = 32 * g + 16 * kh + 4 * tig + e;
-        const uint32_t x = sm.x[t][d0 / 2];
-        const float rr = sm.r[t * NG + g], z = sm.z[t * NG + g];
-        put_code<KB, W>(words, rho, kh, e, code_of<KB>(KN ? lo_bf16(x) * kinv[d0] : lo_bf16(x), z, rr));
-        put_code<KB, W>(words, rho, kh, e + 1, code_of<KB>(KN ? hi_bf16(x) * kinv[d0 + 1] : hi_bf16(x), z, rr));
+    for (int kh = 0; kh < 2; ++kh) {
+      const int d0 = 32 * g + 16 * kh + 4 * tig;
+      const uint2 xw = *reinterpret_cast<const uint2*>(&sm.x[t][d0 / 2]);
+      float2 x01 = bf16x2_to_float2(xw.x), x23 = bf16x2_to_float2(xw.y);
+      if constexpr (KN) {
+        x01 = __fmul2_rn(x01, make_float2(kinv[d0], kinv[d0 + 1]));
+        x23 = __fmul2_rn(x23, make_float2(kinv[d0 + 2], kinv[d0 + 3]));
       }
+      put_reg<KB, W>(words, rho, kh, code_bytes(codes2<KB>(x01, nz, rr), codes2<KB>(x23, nz, rr)));
+    }
+  }
 #pragma unroll
   for (int c = 0; c < W / 4; ++c)
     *reinterpret_cast<uint4*>(rec + word_offset(W, lane, 4 * c)) =
@@ -148,23 +222,17 @@ __device__ void pack_k(HalfTile<D>& sm, const float* kinv, uint8_t* rec, int lan
 template <int D, int VB>
 __device__ void pack_v(HalfTile<D>& sm, uint8_t* vrec, int lane, bool hybrid) {
   constexpr int W = words_per_lane(VB, D);
-  // statistics: each lane owns channel pairs (2w, 2w+1)
+  // statistics: each lane owns channel pairs (2w, 2w+1), compared as bf16x2
 #pragma unroll
   for (int w = lane; w < D / 2; w += 32) {
-    float mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY;
+    uint32_t mnw = sm.x[0][w], mxw = mnw;
 #pragma unroll 8
-    for (int t = 0; t < kTile; ++t) {
-      const uint32_t x = sm.x[t][w];
-      mn0 = fminf(mn0, lo_bf16(x));
-      mx0 = fmaxf(mx0, lo_bf16(x));
-      mn1 = fminf(mn1, hi_bf16(x));
-      mx1 = fmaxf(mx1, hi_bf16(x));
-    }
+    for (int t = 1; t < kTile; ++t) minmax_pairs(mnw, mxw, sm.x[t][w]);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int d = 2 * w + h;
-      float r, z = h ? mn1 : mn0;
-      const uint32_t meta = group_params<VB>(z, h ? mx1 : mx0, r, hybrid);
+      float r, z = h ? hi_bf16(mnw) : lo_bf16(mnw);
+      const uint32_t meta = group_params<VB>(z, h ? hi_bf16(mxw) : lo_bf16(mxw), r, hybrid);
       sm.r[d] = r;
       sm.z[d] = z;
       const int i = (d & 7) * (D / 8) + (d >> 4) * 2 + ((d >> 3) & 1);
@@ -173,6 +241,9 @@ __device__ void pack_v(HalfTile<D>& sm, uint8_t* vrec, int lane, bool hybrid) {
   }
   __syncwarp();
   const int gid = lane >> 2, tig = lane & 3;
+  // channels 16 mb + 8 rh + gid have the parity of gid: pick that bf16 half of
+  // a staged word into the high half of a float with one byte permute
+  const uint32_t half_sel = (gid & 1) ? 0x3244u : 0x1044u;
   uint32_t words[W];
 #pragma unroll
   for (int w = 0; w < W; ++w) words[w] = 0;
@@ -181,14 +252,16 @@ __device__ void pack_v(HalfTile<D>& sm, uint8_t* vrec, int lane, bool hybrid) {
 #pragma unroll
   for (int rho = 0; rho < D / 8; ++rho) {
     const int d = 16 * (rho / 2) + 8 * (rho % 2) + gid;
-    const float rr = sm.r[d], z = sm.z[d];
+    const float r1 = sm.r[d], z1 = sm.z[d];
+    const float2 rr = make_float2(r1, r1), nz = make_float2(-z1, -z1);
 #pragma unroll
-    for (int kh = 0; kh < 2; ++kh)
+    for (int kh = 0; kh < 2; ++kh) {
+      float xv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t x = sm.x[4 * kh + tig + 8 * e][d >> 1];
-        put_code<VB, W>(words, rho, kh, e, code_of<VB>((d & 1) ? hi_bf16(x) : lo_bf16(x), z, rr));
-      }
+      for (int e = 0; e < 4; ++e) xv[e] = __uint_as_float(__byte_perm(sm.x[4 * kh + tig + 8 * e][d >> 1], 0u, half_sel));
+      put_reg<VB, W>(words, rho, kh,
+                     code_bytes(codes2<VB>(make_float2(xv[0], xv[1]), nz, rr), codes2<VB>(make_float2(xv[2], xv[3]), nz, rr)));
+    }
   }
 #pragma unroll
   for (int c = 0; c < W / 4; ++c)
