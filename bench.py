@@ -195,6 +195,98 @@ def oracle_sample(wl, seconds=12.0):
     }
 
 
+def host_cpu():
+    """CPU model name (lscpu), logical cores and the BLAS thread count the
+    oracle runs with (pinned to every host core)."""
+    model = None
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except Exception:
+        pass
+    threads = 1
+    try:
+        from threadpoolctl import threadpool_info, threadpool_limits
+
+        threadpool_limits(os.cpu_count())
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    return {"model": model, "cores": os.cpu_count(), "blas_threads": threads}
+
+
+# streams of each workload the oracle runs (None: every stream of the cache)
+ORACLE_STREAMS = {"tiny": None, "llama3_8b": None, "long_128k": 2, "qwen3_8b": 8, "mistral_7b_b64": 2}
+
+
+def oracle_configs():
+    """The CPU oracle on every benchmark workload: quantize + pack of the
+    prefill (the cache's bytes) and one decode step (dequantize + fp64
+    attention), per stream, summed over the streams run.  Workloads whose
+    stream count is given in ORACLE_STREAMS run that many streams (the first
+    ones) and are extrapolated linearly to the whole cache, labelled so."""
+    import torch
+
+    from oracle import attention as at
+    from oracle import cache as ca
+    from oracle import quantize as qz
+    from quantized_decode_attention_head_b200 import workloads
+
+    to32 = lambda t: qz.bf16_bits_to_f32(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+    res = {}
+    for name, n_run in ORACLE_STREAMS.items():
+        wl = workloads.CONFIGS[name]
+        kb, vb = workload_bits_oracle(wl)
+        n_all = wl.n_layers * wl.batch * wl.n_kv_heads
+        keys = [(l, b, h) for l in range(wl.n_layers) for b in range(wl.batch) for h in range(wl.n_kv_heads)]
+        keys = keys[: (n_all if n_run is None else n_run)]
+        t_q = t_d = 0.0
+        q_bytes = d_bytes = 0
+        for (l, b, h) in keys:
+            one = wl.with_(n_layers=1, batch=1, n_kv_heads=1, n_q_heads=wl.group)
+            k, v, f = workloads.kv_inputs(one, "cpu", seed=wl.seed + 7919 * (1 + l * 977 + b * 31 + h))
+            q, _, _ = workloads.step_inputs(one, 1, f, "cpu", seed=wl.seed + 7919 * (1 + l * 977 + b * 31 + h))
+            kn, vn, qn = to32(k)[0, 0, 0], to32(v)[0, 0, 0], to32(q)[0, 0, 0].astype(np.float64)
+            st = ca.StreamCache(wl.head_dim, int(kb[l, h]), int(vb[l, h]), wl.n_sink, wl.n_recent)
+            t0 = time.perf_counter()
+            st.prefill(kn, vn)
+            st.records()
+            t1 = time.perf_counter()
+            kh, vh = st.dequantized()
+            at.attend(qn, kh, vh)
+            t2 = time.perf_counter()
+            t_q += t1 - t0
+            t_d += t2 - t1
+            rec = [[qz.record_bytes(int(kb[l, h]), int(vb[l, h]), wl.head_dim)]]
+            db = decode_bytes(one, rec, wl.context)
+            d_bytes += db
+            q_bytes += wl.context * wl.head_dim * 2 * 2 + db
+        scale = n_all / len(keys)
+        res[name] = {
+            "streams_run": len(keys), "streams": n_all,
+            "extrapolated": len(keys) < n_all,
+            "quantize_s": t_q * scale, "quantize_gbs": q_bytes / t_q / 1e9,
+            "decode_s": t_d * scale, "decode_gbs": d_bytes / t_d / 1e9,
+        }
+    return res
+
+
+def workload_bits_oracle(wl):
+    """Per-(layer, kv-head) K and V bit widths from the oracle's allocator."""
+    from oracle import allocation as al
+    from quantized_decode_attention_head_b200 import workloads
+
+    inp = workloads.allocation_inputs(wl)
+    shape = (wl.n_layers, wl.n_kv_heads)
+    if "kv" in inp:
+        b = al.allocate(*inp["kv"], wl.allowed)["b_int"].reshape(shape)
+        return b, b
+    return tuple(al.allocate(*inp[key], wl.allowed)["b_int"].reshape(shape) for key in ("k", "v"))
+
+
 def run_reference(args):
     from quantized_decode_attention_head_b200 import workloads
 
@@ -202,8 +294,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = workloads.CONFIGS[WORKLOAD]
-    seconds = max(5.0, 10.0 * (args.steps / max(args.steps, 1)))
-    res = oracle_sample(wl, seconds=seconds)
+    res = oracle_sample(wl, seconds=args.cpu_seconds)
     cb = {"value": res["decode_gbs"], "unit": "GB/s", "cores": res["threads"], "kind": "oracle",
           "sample": res["sample"]}
     line = {
@@ -216,6 +307,36 @@ def run_reference(args):
     }
     print(json.dumps(line))
     return 0
+
+
+def allocator_timings(repeats=5):
+    """Host allocator (rq_allocate_bits) at the pages' scale: the Qwen3-8B
+    workload's 288 (layer, kv-head) units for its K and V budgets (allowed set
+    {2, 3, 4, 8}: exact DP), the same 288 units over the contiguous set
+    {2, 3, 4} (greedy max-heap), and the long-context workload's 8 heads.
+    Best of `repeats` calls, milliseconds."""
+    from quantized_decode_attention_head_b200 import rq_allocate_bits, workloads
+
+    def best(*a):
+        t = []
+        for _ in range(repeats):
+            t0 = time.perf_counter()
+            rq_allocate_bits(*a)
+            t.append(time.perf_counter() - t0)
+        return min(t) * 1e3
+
+    qw = workloads.CONFIGS["qwen3_8b"]
+    inp = workloads.allocation_inputs(qw)
+    wk, ak, bk, avk = inp["k"]
+    wv, av, bv, avv = inp["v"]
+    lw = workloads.CONFIGS[WORKLOAD]
+    return {
+        "qwen3_8b_k_288_units_dp_ms": best(wk, ak, bk, avk, qw.allowed),
+        "qwen3_8b_v_288_units_dp_ms": best(wv, av, bv, avv, qw.allowed),
+        "qwen3_8b_k_288_units_greedy_234_ms": best(wk, ak, bk, avk, (2, 3, 4)),
+        "long_128k_8_heads_ms": best(*workloads.allocation_inputs(lw)["kv"], lw.allowed),
+        "context": "RateQuant §3.3 quotes under 10 ms for Qwen3-8B's 288 KV heads (hardware not stated)",
+    }
 
 
 # ------------------------------------------------------ secondary measurements
@@ -406,7 +527,7 @@ def traffic_record():
         return None
     rec = json.load(open(path))
     h = hashlib.sha256()
-    for name in ("rq_decode.cu", "rq_device.cuh", "rq_internal.h", "rq_pack.cuh"):
+    for name in ("rq_decode.cuh", "rq_device.cuh", "rq_internal.h", "rq_pack.cuh"):
         h.update(open(os.path.join(ROOT, "quantized_decode_attention_head_b200", "csrc", name), "rb").read())
     if rec.get("source_sha256") != h.hexdigest():
         return None
@@ -438,9 +559,16 @@ def run_gpu(args):
     alloc_ms = (time.perf_counter() - t0) * 1e3
     kb = alloc["b_int"].reshape(wl.n_layers, wl.n_kv_heads)
 
+    # Step budget per cache copy (steps go round-robin over the copies):
+    # warm-up, the K timed steps (one CUDA graph), the same K steps launched
+    # eagerly (host submit time), the isolated launches of the per-launch
+    # statistics, and the end-to-end loop.
+    n_launch_stats = 20 + args.launch_stats
     total_steps = args.warmup + args.steps
     e2e_steps = args.steps
-    j0 = (total_steps + NC - 1) // NC  # first per-copy step index of the e2e loop
+    j_eager = (total_steps + NC - 1) // NC
+    j_stats = j_eager + (args.steps + NC - 1) // NC
+    j0 = j_stats + (n_launch_stats + NC - 1) // NC  # first per-copy step index of the e2e loop
     steps_per_copy = j0 + (e2e_steps + NC - 1) // NC + 1
     max_tokens = wl.context + steps_per_copy + 32
     caches, step_in = [], []
@@ -470,62 +598,106 @@ def run_gpu(args):
     ws = caches[0].make_workspace(n_splits=args.splits)
     outs = [torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=torch.float32, device="cuda") for _ in range(NC)]
     torch.cuda.synchronize()
+    step_rows = {}  # (copy, per-copy index) -> the step's q, k_new, v_new views (made once, outside timing)
 
-    def do_step(i, timed_events=None):
+    def rows(c, j):
+        key = (c, j)
+        if key not in step_rows:
+            q, kn, vn = step_in[c]
+            step_rows[key] = (q[j, 0], kn[j, 0], vn[j, 0])
+        return step_rows[key]
+
+    def do_step(i, j_base=0):
         c = i % NC
-        j = i // NC
-        cache, (q, kn, vn) = caches[c], step_in[c]
-        if timed_events is not None:
-            timed_events[0].record(stream)
+        j = j_base + i // NC
+        q, kn, vn = rows(c, j)
         # append + decode: one fused launch, two when the append completes a tile
-        cache.rq_decode_step(0, q[j, 0], kn[j, 0], vn[j, 0], out=outs[c], n_splits=args.splits, workspace=ws)
-        if timed_events is not None:
-            timed_events[1].record(stream)
+        caches[c].rq_decode_step(0, q, kn, vn, out=outs[c], n_splits=args.splits, workspace=ws)
 
-    lengths = [caches[c].length(0) for c in range(NC)]
+    def bytes_of(i_from, n, base_len):
+        """Algorithmic bytes of n round-robin steps starting at step i_from,
+        from each copy's length base_len[c] before them; also the number of
+        two-launch steps (a flush that was not packed ahead: the first step
+        of a copy after its prefill)."""
+        tot, two_n = 0, 0
+        for i in range(i_from, i_from + n):
+            c = i % NC
+            T_old = base_len[c] + (i - i_from) // NC
+            tot += append_bytes(wl, rec, T_old) + decode_bytes(wl, rec, T_old + 1)
+            flush = (split_lengths(T_old + 1, wl.n_sink, wl.n_recent)[1] !=
+                     split_lengths(T_old, wl.n_sink, wl.n_recent)[1])
+            two_n += flush and (T_old == wl.context or wl.n_recent < 2)
+        return tot, two_n
+
     for i in range(args.warmup):
         do_step(i)
     torch.cuda.synchronize()
-    step_bytes = 0
-    fused_bytes = []  # per step: bytes of its single fused launch, or None on a two-launch step
-    n_flush = 0
-    for i in range(args.warmup, total_steps):
-        c = i % NC
-        T_old = caches[c].length(0) + (i - args.warmup) // NC  # length before this step's append
-        ab = append_bytes(wl, rec, T_old)
-        db = decode_bytes(wl, rec, T_old + 1)
-        step_bytes += ab + db
-        flush = split_lengths(T_old + 1, wl.n_sink, wl.n_recent)[1] != split_lengths(T_old, wl.n_sink, wl.n_recent)[1]
-        # the library packs a tile ahead in the fused launch of the step before
-        # its flush, so a flush step is two launches only as the first step of
-        # a cache (or with n_recent < 2)
-        two = flush and (i // NC == 0 or wl.n_recent < 2)
-        n_flush += two
-        fused_bytes.append(None if two else ab + db)
+    base_len = [caches[c].length(0) for c in range(NC)]
+    step_bytes, n_flush = bytes_of(args.warmup, args.steps, base_len)
+    for i in range(args.warmup, total_steps):  # the step views exist before capture
+        rows(i % NC, i // NC)
+    # The K timed steps are captured as one CUDA graph and replayed once: the
+    # replay performs exactly those K steps (the host-side length bookkeeping
+    # advanced during the capture), back to back, with no host gaps between
+    # launches.  A short sleep kernel keeps the GPU busy while the host submits
+    # the replay, so the start event is not stamped before the work arrives.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(args.warmup, total_steps):
+            do_step(i)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    # Events sit only around two-launch steps (if any): an
-    # event between two decode launches would stop the next launch from
-    # overlapping the previous one's tail (programmatic dependent launch).
-    flush_events = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                    for n, fb in enumerate(fused_bytes) if fb is None}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         torch.cuda.synchronize()
+        torch.cuda._sleep(2_000_000)
         start.record(stream)
-        for n, i in enumerate(range(args.warmup, total_steps)):
-            do_step(i, flush_events.get(n))
+        graph.replay()
         end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     elapsed = start.elapsed_time(end) / 1e3
-    # roofline of the fused decode kernel: the timed region minus any
-    # two-launch steps, per single-launch step
-    flush_time = sum(a.elapsed_time(b) / 1e3 for a, b in flush_events.values())
-    n_fused = sum(fb is not None for fb in fused_bytes)
-    dec_avg = (elapsed - flush_time) / n_fused
-    dec_bytes_avg = sum(fb for fb in fused_bytes if fb is not None) / n_fused
+    del graph
+    status = QuantizedKVCache.rq_decode_read_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+
+    # the same number of steps launched eagerly through the Python binding:
+    # device time and the host's submit time per step
+    base_len = [caches[c].length(0) for c in range(NC)]
+    eager_bytes, _ = bytes_of(0, args.steps, base_len)
+    for i in range(args.steps):
+        rows(i % NC, j_eager + i // NC)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    h0 = time.perf_counter()
+    for i in range(args.steps):
+        do_step(i, j_eager)
+    h1 = time.perf_counter()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    eager = {"us_per_step": e0.elapsed_time(e1) * 1e3 / args.steps,
+             "host_submit_us_per_step": (h1 - h0) * 1e6 / args.steps,
+             "gbs": eager_bytes / (e0.elapsed_time(e1) / 1e3) / 1e9}
+
+    # isolated launches: an event pair around each step (no overlap with the
+    # neighbours), 20 warm-up then args.launch_stats timed
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n_launch_stats)]
+    for i in range(n_launch_stats):
+        c = i % NC
+        q, kn, vn = rows(c, j_stats + i // NC)
+        ev[i][0].record(stream)
+        caches[c].rq_decode_step(0, q, kn, vn, out=outs[c], n_splits=args.splits, workspace=ws)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    lt = sorted(a.elapsed_time(b) * 1e3 for a, b in ev[20:])
+    pct = lambda p: lt[min(len(lt) - 1, int(round(p * (len(lt) - 1))))]
+    launch_stats = {"n": len(lt), "warmup": 20, "median_us": pct(0.5), "p10_us": pct(0.1), "p90_us": pct(0.9),
+                    "note": "one fused decode-step launch between two events (no overlap with its neighbours)"}
     status = QuantizedKVCache.rq_decode_read_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status}")
@@ -540,8 +712,9 @@ def run_gpu(args):
     for c in range(NC):
         q_c, k_c, v_c = step_in[c]
         S_c = q_c.shape[0]
-        rows = torch.cat([q_c[:, 0].reshape(S_c, -1), k_c[:, 0].reshape(S_c, -1), v_c[:, 0].reshape(S_c, -1)], dim=1)
-        pin_in.append(rows.cpu().pin_memory())
+        packed = torch.cat([q_c[:, 0].reshape(S_c, -1), k_c[:, 0].reshape(S_c, -1), v_c[:, 0].reshape(S_c, -1)],
+                           dim=1)
+        pin_in.append(packed.cpu().pin_memory())
         dev_in.append(torch.empty(nq + 2 * nk, dtype=torch.bfloat16, device="cuda"))
     dq = [d[:nq].view(step_in[0][0][0, 0].shape) for d in dev_in]
     dk = [d[nq:nq + nk].view(step_in[0][1][0, 0].shape) for d in dev_in]
@@ -578,27 +751,38 @@ def run_gpu(args):
         return 0
 
     peak, peak_kind = _peaks()
-    achieved = dec_bytes_avg / dec_avg / 1e9
+    launches = args.steps + n_flush
+    per_launch = elapsed / launches
+    bytes_per_launch = step_bytes / launches
+    achieved = bytes_per_launch / per_launch / 1e9
     tr = traffic_record()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": (tr["bytes_per_launch_scaled"] if tr else None),
-                "kernel": "decode_kernel<128,4,4> (fused append + split-K decode + combine; on the step before a tile "
-                          "flush also the pack-ahead of that tile; single-launch steps)",
-                "peak_source": f"{peak_kind} hbm_gbs (burst)", "algorithmic_bytes_per_launch": dec_bytes_avg,
-                "avg_launch_us": dec_avg * 1e6}
+                "kernel": "decode_kernel<128,4> (fused append + split-K decode + combine; on the step before a tile "
+                          "flush also the pack-ahead of that tile)",
+                "peak_source": f"{peak_kind} hbm_gbs (burst)", "algorithmic_bytes_per_launch": bytes_per_launch,
+                "avg_launch_us": per_launch * 1e6,
+                "frac_of_nominal_8000_gbs": achieved / 8000.0,
+                "timing": "CUDA events around one replay of a CUDA graph of the K timed steps (launches back to "
+                          "back; each may overlap its predecessor's tail through programmatic dependent launch)"}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         res = oracle_sample(wl, seconds=args.cpu_seconds)
+        hc = host_cpu()
         cpu = {"value": res["decode_gbs"], "unit": "GB/s", "cores": res["threads"], "kind": "oracle",
-               "sample": res["sample"]}
+               "sample": res["sample"], "cpu_model": hc["model"], "logical_cores": hc["cores"],
+               "blas_threads": hc["blas_threads"], "quantize_gbs": res["quantize_gbs"]}
+        if not args.no_sweep:
+            cpu["workloads"] = oracle_configs()
     clk = clocks.summary()
-    extra = {}
+    extra = {"eager": eager, "launch_stats": launch_stats}
     if world == 1 and not args.no_sweep:
         try:
             extra["llama3_8b_step_loop"] = step_loop_graph()
         except Exception as exc:  # a secondary figure never hides the main line
             extra["llama3_8b_step_loop"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         extra["workloads"] = sweep_workloads(["llama3_8b", "mistral_7b_b64", "qwen3_8b"], peak)
+        extra["allocator"] = allocator_timings()
     line = {
         "metric": METRIC,
         "value": bytes_all / elapsed_all / 1e9,
@@ -611,7 +795,7 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "u2+f32",
+        "dtype": "u2 codes; q and P in 16-bit fixed point (two int8 MMA terms); f32 scale/zero epilogue and softmax",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
                    "head_dim": wl.head_dim, "context": wl.context, "bits": "K=V=2 on every head (avg 2 over {2,3,4})",
@@ -619,12 +803,12 @@ def run_gpu(args):
                    f"({NC * decode_bytes(wl, rec, wl.context) / 1e6:.0f} MB > 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
         "decode_gbs": achieved,
-        "decode_us": dec_avg * 1e6,
+        "decode_us": per_launch * 1e6,
         "quantize_gbs": (qbytes / (sum(qtimes) / len(qtimes)) / 1e9) if qtimes else None,
         "alloc_ms": alloc_ms,
         "e2e": {"value": e2e_b_all / e2e_el_all / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": args.steps + n_flush,
+        "gpu_launches": launches,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "clocks": clk,
@@ -632,6 +816,44 @@ def run_gpu(args):
     line.update(extra)
     print(json.dumps(line))
     return 0
+
+
+def run_profile_target(args):
+    """A short run for profiler captures: one cache of the named workload,
+    prefill, then `--steps` all-layer decode launches (rq_decode_attention,
+    automatic plan), or fused steps (rq_decode_step) with --fused.  Prints
+    the mean launch time (CUDA events) as one JSON line; not a bench line."""
+    import torch
+
+    from quantized_decode_attention_head_b200 import QuantizedKVCache, workloads
+
+    wl = workloads.CONFIGS[args.profile]
+    kb, vb = workload_bits(wl)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = QuantizedKVCache(wl.n_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n_sink,
+                             wl.n_recent, wl.context + args.steps + 8, kb, vb, k_norm=args.k_norm)
+    cache.rq_quantize_kv(k, v)
+    del k, v
+    torch.cuda.empty_cache()
+    q, kn, vn = workloads.step_inputs(wl, args.steps, f, "cuda")
+    ws = cache.make_workspace()
+    out = torch.empty((wl.n_layers, wl.batch, wl.n_q_heads, wl.head_dim), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for t in range(args.steps):
+        if args.fused:
+            cache.rq_decode_step(-1, q[t].contiguous(), kn[t].contiguous(), vn[t].contiguous(), out=out, workspace=ws)
+        else:
+            cache.rq_decode_attention(-1, q[t].contiguous(), out=out, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    status = QuantizedKVCache.rq_decode_read_status(ws)
+    print(json.dumps({"profile_target": args.profile, "launches": args.steps, "fused": bool(args.fused),
+                      "k_norm": bool(args.k_norm), "mean_us": e0.elapsed_time(e1) * 1e3 / args.steps,
+                      "device_status": status}))
+    return 0 if status == 0 else 1
 
 
 def main():
@@ -643,10 +865,16 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--copies", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--launch-stats", type=int, default=100, help="isolated launches timed one by one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the secondary figures (other workloads, CUDA-graph step loop)")
+    ap.add_argument("--profile", default=None, help="profiler target: a workload name (see run_profile_target)")
+    ap.add_argument("--fused", action="store_true", help="with --profile: fused decode steps")
+    ap.add_argument("--k-norm", action="store_true", help="with --profile: a K-normalized cache")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile_target(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

@@ -9,8 +9,8 @@ namespace rq {
 
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
   const int part = partial_floats(G, D);
-  // merge slots + window scratch (q, one K and one V chunk)
-  int merge = (NW * part + G * D) * 4 + 2 * kWinChunk * D * 2;
+  // merge slots + window scratch (q, two buffers of one K and one V chunk)
+  int merge = (NW * part + G * D) * 4 + 2 * 2 * kWinChunk * D * 2;
   if (merge < (NW + 1) * part * 4) merge = (NW + 1) * part * 4;  // warp slots + the item partial
   const int ring = NW * stages * stage_bytes;
   int need = ring > merge ? ring : merge;

@@ -657,9 +657,25 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
   const int n_chunks = (n_tok + kWinChunk - 1) / kWinChunk;
   const int c0 = witem * kWinChunksPerItem;
   const int c1 = min(c0 + kWinChunksPerItem, n_chunks);
-  float* qs = scratch;                                              // [G][D]
-  uint32_t* kbuf = reinterpret_cast<uint32_t*>(qs + G * D);         // [32][RW]
-  uint32_t* vbuf = kbuf + kWinChunk * RW;                           // [32][RW]
+  float* qs = scratch;  // [G][D]
+  // two chunk buffers, K [32][RW] then V [32][RW] each, on barriers bar[0],
+  // bar[1]: chunk c0 + k lands in buffer k % 2, and the copy of the chunk
+  // after next starts as soon as a buffer has been read
+  uint32_t* const buf0 = reinterpret_cast<uint32_t*>(qs + G * D);
+  constexpr int kBufWords = 2 * kWinChunk * RW;  // one K and one V chunk
+  auto issue = [&](int ch) {                      // thread 0
+    const int j0 = ch * kWinChunk;
+    const int cnt = min(kWinChunk, n_tok - j0);
+    const bool newest = a.k_new != nullptr && j0 + cnt == n_tok;
+    const int bi = (ch - c0) & 1;
+    uint32_t* kb = buf0 + bi * kBufWords;
+    window_issue_chunk<D>(a, win, kb, kb + kWinChunk * RW, bar + bi, j0, cnt, newest ? a.k_new + knew_off : nullptr,
+                          newest ? a.v_new + knew_off : nullptr);
+  };
+  if (tid == 0) {
+    issue(c0);
+    if (c0 + 1 < c1) issue(c0 + 1);
+  }
   for (int i = tid; i < G * D; i += NW * 32) qs[i] = bf16_bits_to_float(qh[i]);
   // running state of this warp's heads over the item's chunks
   float m[HW], l[HW], o[HW][D / 32];
@@ -670,24 +686,23 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) o[jh][c] = 0.0f;
   }
-  int parity = 0;
-  for (int ch = c0; ch < c1; ++ch, parity ^= 1) {
+  for (int ch = c0; ch < c1; ++ch) {
     const int j0 = ch * kWinChunk;
     const int cnt = min(kWinChunk, n_tok - j0);
     // a fused append delivers the newest token (window index n_tok - 1) itself
     const bool newest = a.k_new != nullptr && j0 + cnt == n_tok;
-    if (ch > c0) {
-      __syncthreads();  // every thread has finished reading the previous chunk
-      if (tid == 0) fence_proxy_async_smem();
-    }
-    if (tid == 0)
-      window_issue_chunk<D>(a, win, kbuf, vbuf, bar, j0, cnt, newest ? a.k_new + knew_off : nullptr,
-                            newest ? a.v_new + knew_off : nullptr);
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, (uint32_t)parity));
+    const int bi = (ch - c0) & 1;
+    const uint32_t parity = ((ch - c0) >> 1) & 1;
+    uint32_t* kbuf = buf0 + bi * kBufWords;
+    uint32_t* vbuf = kbuf + kWinChunk * RW;
+    if (ch == c0) __syncthreads();  // the query is in shared memory
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar + bi, parity));
     if (!__syncthreads_and(ok)) {
       if (tid == 0) {
         raise_abort(abort_flag, a.status);
-        (void)mbar_wait_bounded(bar, (uint32_t)parity);  // let the copies land before the CTA exits
+        // let the copies in flight (this chunk and the next) land before the CTA exits
+        (void)mbar_wait_bounded(bar + bi, parity);
+        if (ch + 1 < c1) (void)mbar_wait_bounded(bar + (bi ^ 1), ((ch + 1 - c0) >> 1) & 1);
       }
       return;
     }
@@ -743,6 +758,13 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
         }
       }
       m[jh] = mn;
+    }
+    if (ch + 2 < c1) {
+      __syncthreads();  // every thread has finished reading this buffer
+      if (tid == 0) {
+        fence_proxy_async_smem();
+        issue(ch + 2);
+      }
     }
   }
 #pragma unroll

@@ -11,6 +11,7 @@ import torch
 
 from gpu_helpers import (all_streams, assert_close, check_stream_bytes, make_cache, oracle_decode, oracle_streams,
                          to_f32, workload_bits)
+from oracle import attention as at
 from oracle import cache as ca
 from oracle import quantize as qz
 from quantized_decode_attention_head_b200 import workloads
@@ -421,4 +422,32 @@ def test_hybrid_prefill_decode_and_steps(d, k_norm):
                 assert_close(out[l, b], e, f"hybrid step {t} layer {l} b {b}")
     for key, s in st.items():
         check_stream_bytes(cache, s, *key)
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+
+
+def test_single_cta_items_merge_in_two_levels():
+    """More than 8 single-CTA items per stream (80 streams of 1100 tiles: the
+    several-waves plan takes 9 tile splits + 1 window item) merge in two
+    levels: groups of 8, then the group partials.  Every stream's output
+    against the cluster-merged decode at the same split count, and sampled
+    streams against the oracle."""
+    wl = _small(n_layers=2, batch=10, n_q_heads=8, n_kv_heads=4, context=4 + 32 + 32 * 1100 + 11)
+    kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, wl.context + 4)
+    cache.rq_quantize_kv(k, v)
+    sample = [(0, 0, 0), (1, 9, 3), (0, 5, 2)]
+    st = oracle_streams(wl, kb, vb, to_f32(k[:, :, :]), to_f32(v), sample)
+    del k, v
+    torch.cuda.empty_cache()
+    q, _, _ = workloads.step_inputs(wl, 1, f, "cuda")
+    ws = cache.make_workspace(n_splits=9)
+    auto = cache.rq_decode_attention(-1, q[0].contiguous(), workspace=ws).cpu().numpy()
+    clus = cache.rq_decode_attention(-1, q[0].contiguous(), n_splits=9, workspace=ws).cpu().numpy()
+    assert_close(auto, clus, "two-level merge vs cluster merge")
+    G = wl.group
+    for (l, b, h), s in st.items():
+        kh, vh = s.dequantized()
+        e = at.attend(to_f32(q[0, l, b, h * G:(h + 1) * G]).astype(np.float64), kh, vh)
+        assert_close(auto[l, b, h * G:(h + 1) * G], e, f"two-level merge stream {(l, b, h)}")
     assert QuantizedKVCache.rq_decode_read_status(ws) == 0
