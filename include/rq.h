@@ -30,8 +30,10 @@
  *   - bf16 tensors are passed as raw 16-bit patterns (const void*), row-major
  *     and contiguous; out is float32.
  *   - Lengths are tracked on the host in the rq_cache handle, so no call reads
- *     device memory back (except rq_cache_init and rq_decode_read_status,
- *     which say so).
+ *     device memory back (except the rq_*_read_status calls, which say so).
+ *   - Device memory handed to the library is used on the stream given with
+ *     the call; a buffer must be valid on that stream (a stream-ordered
+ *     allocator such as PyTorch's hands out memory for its current stream).
  *   - A handle is not thread-safe; one handle per thread of control.
  *
  * Packed tile format (one record per 32-token tile of one (layer, batch,
@@ -181,13 +183,14 @@ typedef struct rq_cache rq_cache; /* opaque host handle */
 rq_status rq_cache_bytes(const rq_cache_config* cfg, size_t* bytes);
 
 /* Bind a caller-owned device buffer (>= rq_cache_bytes, 256-byte aligned) to
- * a new host handle with length 0.  Writes the buffer's descriptor header and
- * sets every stream's K normalization factors to 1 on a private non-blocking
- * stream of the current device and waits for that stream only (a blocking
- * call, like rq_decode_read_status; other streams are not serialised behind
- * it).  The buffer must not be in use by other streams meanwhile.  *out
- * receives the handle. */
-rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes, rq_cache** out);
+ * a new host handle with length 0.  Queues, on `stream`, the copy of the
+ * buffer's descriptor header and the reset of every stream's K normalization
+ * factors to 1 (asynchronous like every other device call; later calls on
+ * the same stream see them).  *out receives the handle.  (The call the pages'
+ * problem statement implies has no stream; the buffer is stream-ordered
+ * memory, so the stream is given here.) */
+rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes, rq_cache** out,
+                        cudaStream_t stream);
 
 /* Free the host handle (never the device buffer).  NULL is ignored. */
 void rq_cache_destroy(rq_cache* cache);
@@ -328,6 +331,10 @@ rq_status rq_decode_attention_noalloc(rq_cache* cache, int layer, const void* q,
  *   it reflects the LAST call made on the device (from any thread).
  * Errors: RQ_ERR_INVALID_ARG (null pointer), RQ_ERR_CUDA. */
 rq_status rq_decode_noalloc_read_status(int* device_status);
+
+/* Name of the last CUDA error a call of this thread reported as RQ_ERR_CUDA
+ * ("no error" if none).  Static string, never NULL. */
+const char* rq_last_cuda_error(void);
 
 /* Library build description (static string). */
 const char* rq_build_info(void);

@@ -59,12 +59,13 @@ _IP = ctypes.POINTER(ctypes.c_int)
 SIGNATURES = {
     "rq_status_string": (ctypes.c_char_p, [_I]),
     "rq_build_info": (ctypes.c_char_p, []),
+    "rq_last_cuda_error": (ctypes.c_char_p, []),
     "rq_allocate_bits": (_I, [_I, _DP, _DP, _DP, ctypes.c_double, _IP, _I, _DP, _IP, _DP]),
     "rq_measure_distortion": (_I, [_P, _I, _I, _I, _I, _IP, _I, _P, _P]),
     "rq_fit_distortion": (_I, [_I, _IP, _I, _DP, ctypes.c_double, _DP, _DP, _DP]),
     "rq_cap_weights": (_I, [_I, _DP, ctypes.c_double, _DP]),
     "rq_cache_bytes": (_I, [ctypes.POINTER(CacheConfig), ctypes.POINTER(_SZ)]),
-    "rq_cache_init": (_I, [ctypes.POINTER(CacheConfig), _P, _SZ, ctypes.POINTER(_P)]),
+    "rq_cache_init": (_I, [ctypes.POINTER(CacheConfig), _P, _SZ, ctypes.POINTER(_P), _P]),
     "rq_cache_destroy": (None, [_P]),
     "rq_cache_length": (_I, [_P, _I, _IP]),
     "rq_cache_stream_layout": (_I, [_P, _I, _I, _I, ctypes.POINTER(_SZ), _IP, _IP, ctypes.POINTER(_SZ)]),
@@ -103,4 +104,6 @@ def lib():
 def check(func: str, code: int):
     if code != 0:
         msg = lib().rq_status_string(code).decode()
+        if code == 6:  # RQ_ERR_CUDA: name the CUDA error
+            msg += ": " + lib().rq_last_cuda_error().decode()
         raise RQError(func, code, msg)

@@ -158,7 +158,7 @@ class QuantizedKVCache:
         self.buffer = self.buffer[off : off + self.nbytes]
         handle = ctypes.c_void_p(0)
         check("rq_cache_init", lib().rq_cache_init(ctypes.byref(cfg), _dptr(self.buffer), self.nbytes,
-                                                   ctypes.byref(handle)))
+                                                   ctypes.byref(handle), _stream_ptr(None, self.buffer.get_device())))
         self.handle = handle
         del keep
 

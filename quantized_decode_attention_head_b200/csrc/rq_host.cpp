@@ -145,7 +145,16 @@ int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, in
   return (int)s;
 }
 
-rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+// The last failing CUDA call of this thread (rq_last_cuda_error).
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+void note_cuda_error(cudaError_t e) {
+  if (e != cudaSuccess) g_last_cuda_error = e;
+}
+
+rq_status cuda_status(cudaError_t e) {
+  note_cuda_error(e);
+  return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
 
 // Decode arguments for layers [l0, l0 + nl) of a cache holding T tokens, with
 // the workspace checked and partitioned; the fused-append pointers are null.
@@ -224,6 +233,10 @@ const char* rq_status_string(rq_status s) {
   return "unknown status";
 }
 
+const char* rq_last_cuda_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}
+
 const char* rq_build_info(void) {
   return "librq: sm_100a; quantize/pack, append/flush, split-K mma.sync decode with bulk-copy pipeline";
 }
@@ -238,7 +251,8 @@ rq_status rq_cache_bytes(const rq_cache_config* cfg, size_t* bytes) {
   return RQ_OK;
 }
 
-rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes, rq_cache** out) {
+rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes, rq_cache** out,
+                        cudaStream_t stream) {
   if (!out || !dev_buf) return RQ_ERR_INVALID_ARG;
   const rq_status st = check_config(cfg);
   if (st != RQ_OK) return st;
@@ -265,19 +279,16 @@ rq_status rq_cache_init(const rq_cache_config* cfg, void* dev_buf, size_t bytes,
   }
   c->k_norm = cfg->k_norm ? 1 : 0;
   // The header copy and the reset of the normalization factors (to 1: a cache
-  // built by appends only) run on a private non-blocking stream that only
-  // this call waits for, so other streams of the process are not serialised
-  // behind it (the legacy default stream would be).
-  cudaStream_t s = nullptr;
-  cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
-  if (e == cudaSuccess) {
-    e = cudaMemcpyAsync(c->buf, c->desc.data(), c->desc.size() * sizeof(HeadDesc), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = rq::launch_norm_reset(c->buf, reinterpret_cast<const HeadDesc*>(c->buf), c->g, s);
-    const cudaError_t e2 = cudaStreamSynchronize(s);
-    if (e == cudaSuccess) e = e2;
-    cudaStreamDestroy(s);
-  }
+  // built by appends only) are queued on the caller's stream -- the stream on
+  // which the buffer is valid (a stream-ordered allocator may hand out memory
+  // whose previous users are still queued there) -- like every other call.
+  // The copy's source is the handle's own descriptor vector, which lives as
+  // long as the handle.
+  cudaError_t e = cudaMemcpyAsync(c->buf, c->desc.data(), c->desc.size() * sizeof(HeadDesc), cudaMemcpyHostToDevice,
+                                  stream);
+  if (e == cudaSuccess) e = rq::launch_norm_reset(c->buf, reinterpret_cast<const HeadDesc*>(c->buf), c->g, stream);
   if (e != cudaSuccess) {
+    note_cuda_error(e);
     delete c;
     return RQ_ERR_CUDA;
   }
@@ -482,7 +493,7 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
   int l0, nl;
   if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
   void* scratch = nullptr;
-  if (rq::noalloc_scratch(&scratch) != cudaSuccess) return RQ_ERR_CUDA;
+  if (cuda_status(rq::noalloc_scratch(&scratch)) != RQ_OK) return RQ_ERR_CUDA;
   rq::DecodeArgs a;
   int smem = 0;
   const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
@@ -510,7 +521,7 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
   if (st != RQ_OK) return st;
   // status word and completion counters must start at zero; the array keeps
   // whatever the previous call (on any stream) left in it
-  if (cudaMemsetAsync(scratch, 0, rq::ws_partial_offset(all_streams), stream) != cudaSuccess) return RQ_ERR_CUDA;
+  if (cuda_status(cudaMemsetAsync(scratch, 0, rq::ws_partial_offset(all_streams), stream)) != RQ_OK) return RQ_ERR_CUDA;
   return cuda_status(rq::launch_decode(a, smem, stream));
 }
 
@@ -519,6 +530,6 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
 extern "C" rq_status rq_decode_noalloc_read_status(int* device_status) {
   if (!device_status) return RQ_ERR_INVALID_ARG;
   void* scratch = nullptr;
-  if (rq::noalloc_scratch(&scratch) != cudaSuccess) return RQ_ERR_CUDA;
+  if (cuda_status(rq::noalloc_scratch(&scratch)) != RQ_OK) return RQ_ERR_CUDA;
   return cuda_status(cudaMemcpy(device_status, scratch, sizeof(int), cudaMemcpyDeviceToHost));
 }

@@ -141,10 +141,10 @@ def test_cache_init_rejects_bad_arguments_before_cuda():
 
     cfg, keep = _config(**_cfg(head_dim=80))
     h = ctypes.c_void_p(0)
-    assert lib.rq_cache_init(ctypes.byref(cfg), ctypes.c_void_p(4096), 1 << 20, ctypes.byref(h)) == 2
+    assert lib.rq_cache_init(ctypes.byref(cfg), ctypes.c_void_p(4096), 1 << 20, ctypes.byref(h), None) == 2
     cfg, keep = _config(**_cfg())
-    assert lib.rq_cache_init(ctypes.byref(cfg), ctypes.c_void_p(4096 + 16), 1 << 30, ctypes.byref(h)) == 1
-    assert lib.rq_cache_init(ctypes.byref(cfg), None, 1 << 30, ctypes.byref(h)) == 1
+    assert lib.rq_cache_init(ctypes.byref(cfg), ctypes.c_void_p(4096 + 16), 1 << 30, ctypes.byref(h), None) == 1
+    assert lib.rq_cache_init(ctypes.byref(cfg), None, 1 << 30, ctypes.byref(h), None) == 1
     # null handles everywhere
     assert lib.rq_quantize_kv(None, None, None, 0, None) == 1
     assert lib.rq_append_token(None, 0, None, None, None) == 1
