@@ -829,6 +829,10 @@ def run_profile_target(args):
 
     wl = workloads.CONFIGS[args.profile]
     kb, vb = workload_bits(wl)
+    if args.layers or args.batch:  # a smaller cache of the same workload (same per-layer bit widths)
+        nl = args.layers or wl.n_layers
+        wl = wl.with_(n_layers=nl, batch=args.batch or wl.batch)
+        kb, vb = kb[:nl], vb[:nl]
     k, v, f = workloads.kv_inputs(wl, "cuda")
     cache = QuantizedKVCache(wl.n_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n_sink,
                              wl.n_recent, wl.context + args.steps + 8, kb, vb, k_norm=args.k_norm)
@@ -872,6 +876,8 @@ def main():
     ap.add_argument("--profile", default=None, help="profiler target: a workload name (see run_profile_target)")
     ap.add_argument("--fused", action="store_true", help="with --profile: fused decode steps")
     ap.add_argument("--k-norm", action="store_true", help="with --profile: a K-normalized cache")
+    ap.add_argument("--layers", type=int, default=0, help="with --profile: first N layers only")
+    ap.add_argument("--batch", type=int, default=0, help="with --profile: batch size override")
     args = ap.parse_args()
     if args.profile:
         return run_profile_target(args)

@@ -7,19 +7,31 @@
 
 namespace rq {
 
-int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
+// per-warp scale scratch of the tile path (Cfg<D, G>::SCRATCH floats), at the
+// base of the dynamic shared memory
+constexpr int scale_scratch_bytes(int D) { return NW * 8 * ((D / 32) * 8 + 4 + (D / 8) * 2 + 4) * 4; }
+static_assert(scale_scratch_bytes(128) == NW * Cfg<128, 4>::SCRATCH * 4, "scale scratch layout");
+static_assert(scale_scratch_bytes(64) == NW * Cfg<64, 4>::SCRATCH * 4, "scale scratch layout");
+
+// Shared memory of the roles that alias the tile rings (after the scale
+// scratch): the merge slots (warp slots + the item partial), the window
+// item's two buffers of one K and one V chunk (which start at the base and
+// so also cover the scale scratch), and the pack-ahead item's staged K and V
+// tile.
+int decode_free_bytes(int G, int D) {
   const int part = partial_floats(G, D);
-  // merge slots + window scratch (q, two buffers of one K and one V chunk)
-  int merge = (NW * part + G * D) * 4 + 2 * 2 * kWinChunk * D * 2;
-  if (merge < (NW + 1) * part * 4) merge = (NW + 1) * part * 4;  // warp slots + the item partial
-  const int ring = NW * stages * stage_bytes;
-  int need = ring > merge ? ring : merge;
-  // a pack-ahead item stages one K and one V tile
+  int merge = (NW + 1) * part * 4;
+  const int win = window_smem_bytes(D) - scale_scratch_bytes(D);
+  if (merge < win) merge = win;
   const int pack = D == 128 ? (int)sizeof(TileSmem<128>) : (int)sizeof(TileSmem<64>);
-  if (need < pack) need = pack;
-  // per-warp scale scratch of the tile path (Cfg<D, G>::SCRATCH floats)
-  const int scratch = NW * 8 * ((D / 32) * 8 + 4 + (D / 8) * 2 + 4) * 4;
-  return (need + 127) / 128 * 128 + scratch;
+  return merge > pack ? merge : pack;
+}
+
+int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D) {
+  const int ring = NW * stages * stage_bytes;
+  const int other = decode_free_bytes(G, D);
+  const int need = ring > other ? ring : other;
+  return (need + 127) / 128 * 128 + scale_scratch_bytes(D);
 }
 
 int decode_resident_ctas(int D, int G, int cluster, int smem, int q_terms) {

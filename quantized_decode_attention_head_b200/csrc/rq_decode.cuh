@@ -92,30 +92,13 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return _
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-#ifndef RQ_CVT_BIAS
-#define RQ_CVT_BIAS 0
-#endif
-// tile records per warp prefetched into L2 (beyond its ring) before the
-// launch waits for its predecessor
-#ifndef RQ_L2_AHEAD
-#define RQ_L2_AHEAD 0
-#endif
-// C operand of the two-term MMAs: 0 (int32 results) or the bits of 1.5 * 2^23
-// (each result, read as a float, is 1.5 * 2^23 + the exact integer sum).
-constexpr uint32_t kTermC = RQ_CVT_BIAS ? kBiasBits : 0u;
-
 // The two-term results (hi, lo) of rows gid and gid + 8 of one MMA -> the
-// pair (256 hi + lo) of both rows in fp32, each rounded once.
+// pair (256 hi + lo) of both rows in fp32: |256 hi + lo| < 2^31 is exact in
+// int32, one rounding to fp32 per row.  (The alternative -- C = the bits of
+// 1.5 * 2^23, so that the results read as floats, and packed subtractions --
+// pairs registers of different rows and measured more instructions.)
 __device__ __forceinline__ float2 combine_terms(const uint32_t (&c)[4]) {
-  if constexpr (RQ_CVT_BIAS) {
-    const float2 nb = make_float2(-kBias, -kBias);
-    const float2 r0 = fadd2(make_float2(__uint_as_float(c[0]), __uint_as_float(c[1])), nb);  // exact integers
-    const float2 r1 = fadd2(make_float2(__uint_as_float(c[2]), __uint_as_float(c[3])), nb);
-    return make_float2(fmaf(256.0f, r0.x, r0.y), fmaf(256.0f, r1.x, r1.y));
-  } else {
-    // |256 hi + lo| < 2^31: exact in int32, one rounding to fp32 per row
-    return make_float2((float)((int)c[0] * 256 + (int)c[1]), (float)((int)c[2] * 256 + (int)c[3]));
-  }
+  return make_float2((float)((int)c[0] * 256 + (int)c[1]), (float)((int)c[2] * 256 + (int)c[3]));
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -357,7 +340,7 @@ __device__ __forceinline__ void qk_tile(const uint8_t* rec, const WarpState<D, G
           v = make_float2(fmaf(65536.0f, (float)(int)c[0], (float)((int)c[1] * 256 + (int)c3[0])),
                           fmaf(65536.0f, (float)(int)c[2], (float)((int)c[3] * 256 + (int)c3[2])));
         } else {
-          imma_u8s8(c, a, st.qb[nb][g][0], st.qb[nb][g][1], kTermC);
+          imma_u8s8(c, a, st.qb[nb][g][0], st.qb[nb][g][1], 0u);
           v = combine_terms(c);
         }
         acc[nb][mb] = ffma2(make_float2(sz.x, sz.y), v, ffma2(make_float2(sz.z, sz.w), st.qz[nb][g], acc[nb][mb]));
@@ -461,7 +444,7 @@ __device__ __forceinline__ void pv_tile(const uint8_t* vrec, WarpState<D, G, QT>
 #pragma unroll
     for (int nb = 0; nb < C::NB; ++nb) {
       uint32_t c[4];
-      imma_u8u8(c, a, pb[nb][0], pb[nb][1], kTermC);
+      imma_u8u8(c, a, pb[nb][0], pb[nb][1], 0u);
       const float2 v = combine_terms(c);
       st.o[nb][mb] = ffma2(make_float2(sz.x, sz.y), v, ffma2(make_float2(sz.z, sz.w), ps[nb], st.o[nb][mb]));
     }
@@ -497,12 +480,6 @@ __device__ void consume(WarpState<D, G, QT>& st, const uint16_t* qh, const float
                     policy);
     }
   }
-  // the next few records into L2 as well, so that while the previous launch
-  // finishes (its merge tail), this one keeps HBM busy
-  if (RQ_L2_AHEAD > 0 && lane < RQ_L2_AHEAD) {
-    const int j = stages + lane;
-    if (j < n_w) l2_prefetch(src + (int64_t)(warp + j * NW) * rec, (uint32_t)rec);
-  }
   griddep_wait();  // every earlier kernel of the stream has completed and its writes are visible
   setup_query<D, G, KB, VB, QT>(st, qh, nrm, scale_log2, lane);
   float* ks = scratch;
@@ -522,12 +499,12 @@ __device__ void consume(WarpState<D, G, QT>& st, const uint16_t* qh, const float
     uint32_t pb[C::NB][2];
     softmax_tile<D, G, QT>(st, acc, pb, lane);
     pv_tile<D, G, VB, QT>(cur + VOFF, st, vs, pb, lane);
-    __syncwarp();  // every lane has finished reading the slot and the scratch
-    if (lane == 0 && j + stages < n_w) {
-      fence_proxy_async_smem();  // generic-proxy reads of the slot precede the async refill
-      mbar_arrive_expect_tx(&bars[slot], (uint32_t)rec);
-      bulk_g2s_hint(cur, nsrc, (uint32_t)rec, &bars[slot], policy);
-    }
+    // every lane has read the slot (its values are consumed): lane 0 re-arms
+    // it for tile j + stages, as a predicated copy rather than a branch.  The
+    // slot is only ever read through the generic proxy, so the refill (async
+    // proxy) needs no proxy fence, only this ordering after the reads.
+    __syncwarp();
+    bulk_g2s_hint_if(lane == 0 && j + stages < n_w, cur, nsrc, (uint32_t)rec, &bars[slot], policy);
     nsrc += (int64_t)NW * rec;
     cur += stage_bytes;
     if (++slot == stages) {
@@ -599,93 +576,127 @@ __device__ void dump_tile_state(const WarpState<D, G, QT>& st, float* slot, int 
   }
 }
 
-// bf16 sink + recent window on CUDA cores.  The window is split into chunks
-// of 32 tokens, kWinChunksPerItem consecutive chunks per work item.  For each
-// chunk thread 0 stages its K and V rows in shared memory with at most six
-// 1-D bulk copies (the rows of a chunk form at most three contiguous runs:
-// sink, ring, ring after wrap); warp w then takes heads w, w + 4, ...:
-// lane = token for q.k (K row words read in a lane-rotated order so the 32
-// rows hit 32 banks), lane = channel for p.v, and merges the chunk into its
-// running (m, l, o).
+// bf16 sink + recent window on the tensor cores.  The window is split into
+// chunks of 32 tokens, kWinChunksPerItem consecutive chunks per work item.
+// For each chunk the lanes of warp 0 stage its K and V rows in shared memory
+// with one 1-D bulk copy per row (rows padded to 2 D + 16 bytes, so the 8
+// rows of an 8x8 ldmatrix block fall in 8 different bank quads); warp w then
+// takes tokens 8 w .. 8 w + 7 of the chunk for all G heads:
+//   scores (heads x 8 tokens) = q (A, bf16 from the caller's rows, heads in
+//     rows 0..G-1) . K^T (B, ldmatrix of the K rows), m16n8k16, fp32;
+//   o^T (channels x heads) += V^T (A, ldmatrix.trans of the V rows) . P (B,
+//     straight from the score fragments), m16n8k8, with P split into two
+//     bf16 terms p = p_hi + p_lo (relative error 2^-17 instead of bf16's
+//     2^-9), so that the products are exact and only the fp32 accumulation
+//     rounds.
+// Each warp keeps its own online-softmax state over its tokens; the warps'
+// states are merged like the tile path's.
 constexpr int kWinChunk = 32;
+__host__ __device__ constexpr int window_row_stride(int D) { return 2 * D + 16; }
+// shared memory of a window item: two buffers of one K and one V chunk
+__host__ __device__ constexpr int window_smem_bytes(int D) { return 2 * 2 * kWinChunk * window_row_stride(D); }
 
 __host__ __device__ inline int window_tokens(int T, int S, int Tq) { return (T < S ? T : S) + (T - (T < S ? T : S) - Tq); }
 
+// Lanes of one warp: the K and V rows of window tokens j0 .. j0 + cnt - 1
+// into kbuf / vbuf (row t at t * window_row_stride(D)), counted on bar.
 template <int D>
-__device__ __forceinline__ void window_issue_chunk(const DecodeArgs& a, const uint8_t* win, uint32_t* kbuf,
-                                                   uint32_t* vbuf, uint64_t* bar, int j0, int cnt,
-                                                   const uint16_t* knew, const uint16_t* vnew) {
+__device__ __forceinline__ void window_issue_chunk(const DecodeArgs& a, const uint8_t* win, uint8_t* kbuf,
+                                                   uint8_t* vbuf, uint64_t* bar, int j0, int cnt,
+                                                   const uint16_t* knew, const uint16_t* vnew, int lane) {
+  constexpr int RB = 2 * D, RS = window_row_stride(D);
+  if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(cnt * RB * 2));
+  __syncwarp();
+  if (lane < cnt) {
+    const int S = a.g.S, ring = a.g.R + kTile;
+    const int n_sink = a.T < S ? a.T : S;
+    const int j = j0 + lane;
+    const void *ks, *vs;
+    if (knew && lane == cnt - 1) {
+      // appended in the same call: the newest token comes from the caller's rows
+      ks = knew;
+      vs = vnew;
+    } else if (j < n_sink) {
+      ks = win + (size_t)j * RB;
+      vs = win + (size_t)(S + j) * RB;
+    } else {
+      const int slot = (a.Tq + (j - n_sink)) % ring;
+      ks = win + (size_t)(2 * S + slot) * RB;
+      vs = win + (size_t)(2 * S + ring + slot) * RB;
+    }
+    bulk_g2s(kbuf + lane * RS, ks, (uint32_t)RB, bar);
+    bulk_g2s(vbuf + lane * RS, vs, (uint32_t)RB, bar);
+  }
+}
+
+// L2 prefetch of the cache rows (K and V) of window tokens [j0, j1), by one
+// thread: at most three contiguous runs (sink, ring, ring after its wrap).
+// Issued before the wait on the previous kernel: a row that kernel still
+// writes is updated in L2, which the later copies read.
+template <int D>
+__device__ void window_prefetch_l2(const DecodeArgs& a, const uint8_t* win, int j0, int j1) {
+  constexpr int RB = 2 * D;
   const int S = a.g.S, ring = a.g.R + kTile;
   const int n_sink = a.T < S ? a.T : S;
-  mbar_arrive_expect_tx(bar, (uint32_t)(cnt * D * 2 * 2));
-  // appended in the same call: the newest token comes from the caller's rows
-  const int n_cache = knew ? cnt - 1 : cnt;
-  if (knew) {
-    bulk_g2s(kbuf + (size_t)n_cache * (D / 2), knew, (uint32_t)(D * 2), bar);
-    bulk_g2s(vbuf + (size_t)n_cache * (D / 2), vnew, (uint32_t)(D * 2), bar);
-  }
-  int t = 0;
-  while (t < n_cache) {
-    const int j = j0 + t;
-    size_t row;  // K row inside the window block; its V row follows its block's K rows
+  for (int j = j0; j < j1;) {
+    size_t row, v_off;
     int run;
-    size_t v_off;
     if (j < n_sink) {
       row = j;
-      run = min(n_cache - t, n_sink - j);
+      run = min(j1, n_sink) - j;
       v_off = S;
     } else {
       const int slot = (a.Tq + (j - n_sink)) % ring;
       row = (size_t)2 * S + slot;
-      run = min(n_cache - t, ring - slot);
+      run = min(j1 - j, ring - slot);
       v_off = ring;
     }
-    bulk_g2s(kbuf + (size_t)t * (D / 2), win + row * D * 2, (uint32_t)(run * D * 2), bar);
-    bulk_g2s(vbuf + (size_t)t * (D / 2), win + (row + v_off) * D * 2, (uint32_t)(run * D * 2), bar);
-    t += run;
+    l2_prefetch(win + row * RB, (uint32_t)(run * RB));
+    l2_prefetch(win + (row + v_off) * RB, (uint32_t)(run * RB));
+    j += run;
   }
 }
 
 template <int D, int G>
 __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* qh, size_t knew_off, int witem,
-                            float* scratch, uint64_t* bar, float* slot, int warp, int lane,
+                            uint8_t* scratch, uint64_t* bar, float* slot, int warp, int lane,
                             volatile int* abort_flag) {
-  constexpr int RW = D / 2;  // words per bf16 row
-  constexpr int HW = (G + NW - 1) / NW;
-  const int tid = warp * 32 + lane;
+  constexpr int RB = 2 * D, RS = window_row_stride(D);
+  constexpr int KS = D / 16;  // k16 steps of q.K^T, m16 tiles of o^T
+  const int tid = warp * 32 + lane, gid = lane >> 2, tig = lane & 3;
   const int n_tok = window_tokens(a.T, a.g.S, a.Tq);
   const int n_chunks = (n_tok + kWinChunk - 1) / kWinChunk;
   const int c0 = witem * kWinChunksPerItem;
   const int c1 = min(c0 + kWinChunksPerItem, n_chunks);
-  float* qs = scratch;  // [G][D]
-  // two chunk buffers, K [32][RW] then V [32][RW] each, on barriers bar[0],
-  // bar[1]: chunk c0 + k lands in buffer k % 2, and the copy of the chunk
-  // after next starts as soon as a buffer has been read
-  uint32_t* const buf0 = reinterpret_cast<uint32_t*>(qs + G * D);
-  constexpr int kBufWords = 2 * kWinChunk * RW;  // one K and one V chunk
-  auto issue = [&](int ch) {                      // thread 0
+  constexpr int kBufBytes = 2 * kWinChunk * RS;  // one K and one V chunk
+  // chunk c0 + k lands in buffer k % 2 on bar[k % 2]; the copy of the chunk
+  // after next starts as soon as every warp has read a buffer
+  auto issue = [&](int ch) {  // warp 0
     const int j0 = ch * kWinChunk;
     const int cnt = min(kWinChunk, n_tok - j0);
     const bool newest = a.k_new != nullptr && j0 + cnt == n_tok;
     const int bi = (ch - c0) & 1;
-    uint32_t* kb = buf0 + bi * kBufWords;
-    window_issue_chunk<D>(a, win, kb, kb + kWinChunk * RW, bar + bi, j0, cnt, newest ? a.k_new + knew_off : nullptr,
-                          newest ? a.v_new + knew_off : nullptr);
+    uint8_t* kb = scratch + bi * kBufBytes;
+    window_issue_chunk<D>(a, win, kb, kb + kWinChunk * RS, bar + bi, j0, cnt, newest ? a.k_new + knew_off : nullptr,
+                          newest ? a.v_new + knew_off : nullptr, lane);
   };
-  if (tid == 0) {
+  // (an item past the window's last chunk -- a padding item of a cluster --
+  // issues nothing and leaves empty partial states).  The buffers overlap the
+  // warp slots, which are written after the last chunk.
+  if (warp == 0 && c0 < c1) {
     issue(c0);
     if (c0 + 1 < c1) issue(c0 + 1);
   }
-  for (int i = tid; i < G * D; i += NW * 32) qs[i] = bf16_bits_to_float(qh[i]);
-  // running state of this warp's heads over the item's chunks
-  float m[HW], l[HW], o[HW][D / 32];
+  // q of head gid: bf16 A fragments (rows gid + 8 are empty), re-read from
+  // L1 for every chunk rather than held in registers
+  const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qh + (gid < G ? gid : 0) * D) + tig;
+  // running state: m, l of head gid (l summed over the quad at the end);
+  // o[mt]: channels 16 mt + gid (+ 8) x heads 2 tig, 2 tig + 1
+  float m = -INFINITY, l = 0.0f;
+  float o[KS][4];
 #pragma unroll
-  for (int jh = 0; jh < HW; ++jh) {
-    m[jh] = -INFINITY;
-    l[jh] = 0.0f;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) o[jh][c] = 0.0f;
-  }
+  for (int mt = 0; mt < KS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
+  const int n0 = 8 * warp;  // this warp's tokens in every chunk
   for (int ch = c0; ch < c1; ++ch) {
     const int j0 = ch * kWinChunk;
     const int cnt = min(kWinChunk, n_tok - j0);
@@ -693,9 +704,8 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
     const bool newest = a.k_new != nullptr && j0 + cnt == n_tok;
     const int bi = (ch - c0) & 1;
     const uint32_t parity = ((ch - c0) >> 1) & 1;
-    uint32_t* kbuf = buf0 + bi * kBufWords;
-    uint32_t* vbuf = kbuf + kWinChunk * RW;
-    if (ch == c0) __syncthreads();  // the query is in shared memory
+    uint8_t* kbuf = scratch + bi * kBufBytes;
+    uint8_t* vbuf = kbuf + kWinChunk * RS;
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar + bi, parity));
     if (!__syncthreads_and(ok)) {
       if (tid == 0) {
@@ -723,71 +733,94 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
       }
       const int c = tid % (D / 8);
       const bool isv = tid >= D / 8;
-      const uint4 x = reinterpret_cast<const uint4*>((isv ? vbuf : kbuf) + (size_t)(cnt - 1) * RW)[c];
-      reinterpret_cast<uint4*>(win + (isv ? vrow : krow) * D * 2)[c] = x;
+      const uint4 x = reinterpret_cast<const uint4*>((isv ? vbuf : kbuf) + (size_t)(cnt - 1) * RS)[c];
+      reinterpret_cast<uint4*>(win + (isv ? vrow : krow) * RB)[c] = x;
     }
-#pragma unroll
-    for (int jh = 0; jh < HW; ++jh) {
-      const int h = warp + NW * jh;
-      if (h >= G) continue;
-      float acc = 0.0f;
-      if (lane < cnt) {
-#pragma unroll 8
-        for (int w = 0; w < RW; ++w) {
-          const int wr = (w + lane) & (RW - 1);
-          const uint32_t kk = kbuf[lane * RW + wr];
-          acc = fmaf(qs[h * D + 2 * wr], bf16_bits_to_float(kk & 0xFFFFu),
-                     fmaf(qs[h * D + 2 * wr + 1], bf16_bits_to_float(kk >> 16), acc));
+    if (n0 < cnt) {  // warp-uniform
+      if (n0 + 8 > cnt) {
+        // rows past the window's end hold stale bytes: P is 0 there, but
+        // 0 * NaN is not, so their V rows are zeroed first (this is the
+        // window's last chunk: no later copy lands in this buffer)
+        for (int i = lane; i < (n0 + 8 - cnt) * (RB / 16); i += 32) {
+          const int t = cnt + i / (RB / 16);
+          reinterpret_cast<uint4*>(vbuf + (size_t)t * RS)[i % (RB / 16)] = make_uint4(0u, 0u, 0u, 0u);
         }
+        __syncwarp();
       }
-      const float x = lane < cnt ? acc * a.scale_log2 : -INFINITY;
-      const float mc = warp_max(x);
-      const float mn = fmaxf(m[jh], mc);
-      const float a_old = ex2(m[jh] - mn);  // 0 while m = -inf
-      const float p = ex2(x - mn);
-      l[jh] = l[jh] * a_old + warp_sum(p);
+      // scores: head gid (row) x tokens n0 + 2 tig, + 1 (columns), in two
+      // accumulators over even and odd k-steps
+      float s[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+      const uint32_t krow = smem_u32(kbuf) + (n0 + (lane & 7)) * RS + (lane >> 3) * 16;
+#pragma unroll 1
+      for (int p = 0; p < KS / 2; ++p) {
+        uint32_t b[4], qa[4];
+        ldsm_x4(b, krow + p * 64);  // channels 32 p .. 32 p + 31: k-steps 2 p, 2 p + 1
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) o[jh][c] *= a_old;
-      for (int t = 0; t < cnt; ++t) {
-        const float pt = __shfl_sync(0xffffffffu, p, t);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const int d = lane + 32 * c;
-          const uint32_t vv = vbuf[t * RW + d / 2];
-          o[jh][c] = fmaf(pt, (d & 1) ? bf16_bits_to_float(vv >> 16) : bf16_bits_to_float(vv & 0xFFFFu), o[jh][c]);
-        }
+        for (int i = 0; i < 4; ++i) qa[i] = gid < G ? __ldg(qrow + 16 * p + 4 * i) : 0u;
+        mma_bf16_k16(s[0], qa[0], 0u, qa[1], 0u, b[0], b[1]);
+        mma_bf16_k16(s[1], qa[2], 0u, qa[3], 0u, b[2], b[3]);
       }
-      m[jh] = mn;
+      const int t0 = n0 + 2 * tig;
+      const float x0 = t0 < cnt ? (s[0][0] + s[1][0]) * a.scale_log2 : -INFINITY;
+      const float x1 = t0 + 1 < cnt ? (s[0][1] + s[1][1]) * a.scale_log2 : -INFINITY;
+      float cm = fmaxf(x0, x1);  // token n0 is valid: finite after the quad max
+      cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+      cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+      const float mn = fmaxf(m, cm);
+      const float alpha = ex2(m - mn);  // 0 while m = -inf
+      m = mn;
+      const float p0 = ex2(x0 - mn), p1 = ex2(x1 - mn);
+      l = fmaf(l, alpha, p0 + p1);
+      // o columns are heads 2 tig, 2 tig + 1, whose state lives in lanes 8 tig, 8 tig + 4
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * tig), a1 = __shfl_sync(0xffffffffu, alpha, 8 * tig + 4);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        o[mt][0] *= a0;
+        o[mt][1] *= a1;
+        o[mt][2] *= a0;
+        o[mt][3] *= a1;
+      }
+      // B fragment of P (tokens 2 tig, 2 tig + 1 of head gid) in two bf16 terms
+      const uint32_t ph = pack_bf16x2(p0, p1);
+      const uint32_t pl = pack_bf16x2(p0 - bf16_bits_to_float(ph & 0xFFFFu), p1 - bf16_bits_to_float(ph >> 16));
+      const uint32_t vrow = smem_u32(vbuf) + (n0 + (lane & 7)) * RS + (lane >> 3) * 16;
+#pragma unroll
+      for (int p = 0; p < KS / 2; ++p) {
+        uint32_t v[4];
+        ldsm_x4_trans(v, vrow + p * 64);  // channels 32 p .. 32 p + 31: m-tiles 2 p, 2 p + 1
+        mma_bf16_k8(o[2 * p], v[0], v[1], ph);
+        mma_bf16_k8(o[2 * p + 1], v[2], v[3], ph);
+        mma_bf16_k8(o[2 * p], v[0], v[1], pl);
+        mma_bf16_k8(o[2 * p + 1], v[2], v[3], pl);
+      }
     }
     if (ch + 2 < c1) {
-      __syncthreads();  // every thread has finished reading this buffer
-      if (tid == 0) {
+      __syncthreads();  // every warp has finished reading this buffer
+      if (warp == 0) {
         fence_proxy_async_smem();
         issue(ch + 2);
       }
     }
   }
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+  __syncthreads();  // every warp has read the chunk buffers, which the warp slots overlap
+  // this warp's partial state of all G heads (m = -inf, l = 0, o = 0 when it
+  // saw no token)
 #pragma unroll
-  for (int jh = 0; jh < HW; ++jh) {
-    const int h = warp + NW * jh;
+  for (int e = 0; e < 2; ++e) {
+    const int h = 2 * tig + e;
     if (h < G) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) slot[h * D + lane + 32 * c] = o[jh][c];
-      if (lane == 0) {
-        slot[G * D + h] = m[jh];
-        slot[G * D + G + h] = l[jh];
+      for (int mt = 0; mt < KS; ++mt) {
+        slot[h * D + 16 * mt + gid] = o[mt][e];
+        slot[h * D + 16 * mt + 8 + gid] = o[mt][2 + e];
       }
     }
   }
-  // heads of the other warps: empty partial states
-  for (int h = 0; h < G; ++h) {
-    if (h % NW == warp) continue;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) slot[h * D + lane + 32 * c] = 0.0f;
-    if (lane == 0) {
-      slot[G * D + h] = -INFINITY;
-      slot[G * D + G + h] = 0.0f;
-    }
+  if (tig == 0 && gid < G) {
+    slot[G * D + gid] = m;
+    slot[G * D + G + gid] = l;
   }
 }
 
@@ -989,12 +1022,20 @@ __global__ void __launch_bounds__(kDecodeThreads, QT == 3 ? 3 : RQ_DECODE_MIN_BL
   } else if (a.n_pack && item == a.n_splits + a.n_win) {
     pack_item<D, G>(a, hd, b, area, merge, tid);
   } else {
-    griddep_wait();  // the window rows and the query may come from the previous kernel
     // 32-token chunks of the bf16 sink + recent window
     uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
+    if (tid == 0) {
+      const int n_tok = window_tokens(a.T, a.g.S, a.Tq);
+      const int j0 = (item - a.n_splits) * kWinChunksPerItem * kWinChunk;
+      const int j1 = min(j0 + kWinChunksPerItem * kWinChunk, n_tok);
+      if (j0 < j1) window_prefetch_l2<D>(a, win, j0, j1);
+    }
+    griddep_wait();  // the window rows and the query may come from the previous kernel
     const size_t knew_off = ((size_t)(lrel * a.g.B + b) * a.g.Hkv + h) * D;
-    window_item<D, G>(a, win, qh, knew_off, item - a.n_splits, merge + NW * C::PART, &bars[0],
-                      merge + warp * C::PART, warp, lane, &abort_flag);
+    // the chunk buffers start at the base of the dynamic shared memory (the
+    // tile path's scale scratch is idle here) and end inside the merge area
+    window_item<D, G>(a, win, qh, knew_off, item - a.n_splits, smem, &bars[0], merge + warp * C::PART, warp, lane,
+                      &abort_flag);
   }
   __syncthreads();
   const bool valid = !abort_flag;
@@ -1076,25 +1117,21 @@ __global__ void __launch_bounds__(kDecodeThreads, QT == 3 ? 3 : RQ_DECODE_MIN_BL
       // group partials into the output
       const int grp = item / kMergeGroup;
       const int gsize = min(kMergeGroup, NI - grp * kMergeGroup);
-      __threadfence();
       __syncthreads();
       if (tid == 0) {
         uint32_t* gc = &a.counters[(size_t)srel * kCountersPerStream + 1 + grp];
-        const int last_g = atomicAdd(gc, 1u) == (unsigned)(gsize - 1);
+        const int last_g = count_acq_rel(gc) == (unsigned)(gsize - 1);
         if (last_g) *gc = 0u;  // every item of the group has counted: reset for the next call
         is_last = last_g;
       }
       __syncthreads();
       if (!is_last) return;
-      __threadfence();
       merge_quads<D, G, kMergeGroup>(ps + (size_t)grp * kMergeGroup * C::PART, gsize, ps + (size_t)(NI + grp) * C::PART,
                                      nullptr, tid);
-      __threadfence();
       __syncthreads();
-      if (tid == 0) is_last = atomicAdd(&a.counters[(size_t)srel * kCountersPerStream], 1u) == (unsigned)(ngr - 1);
+      if (tid == 0) is_last = count_acq_rel(&a.counters[(size_t)srel * kCountersPerStream]) == (unsigned)(ngr - 1);
       __syncthreads();
       if (!is_last) return;
-      __threadfence();
       float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
       merge_quads<D, G, 12>(ps + (size_t)NI * C::PART, ngr, nullptr, outp, tid);
       if (tid == 0) a.counters[(size_t)srel * kCountersPerStream] = 0u;
@@ -1104,10 +1141,9 @@ __global__ void __launch_bounds__(kDecodeThreads, QT == 3 ? 3 : RQ_DECODE_MIN_BL
   // the first CTA publishes the cluster partial and learns whether its
   // cluster is the stream's last; it tells every CTA of the cluster
   if (crank == 0) {
-    __threadfence();
     __syncthreads();
     if (tid == 0) {
-      const int last = atomicAdd(&a.counters[(size_t)srel * kCountersPerStream], 1u) == (unsigned)(ncl - 1);
+      const int last = count_acq_rel(&a.counters[(size_t)srel * kCountersPerStream]) == (unsigned)(ncl - 1);
       if constexpr (CL > 1) {
         cg::cluster_group cluster = cg::this_cluster();
 #pragma unroll
@@ -1124,13 +1160,14 @@ __global__ void __launch_bounds__(kDecodeThreads, QT == 3 ? 3 : RQ_DECODE_MIN_BL
   }
   if (!is_last) return;
   // Level 2: the CTAs of the last cluster merge the cluster partials, each a
-  // slice of the outputs
-  __threadfence();
+  // slice of the outputs (CTAs other than the one that took the count
+  // acquire the other clusters' partials with a fence of their own)
+  if constexpr (CL > 1) __threadfence();
   float* outp = a.out + ((size_t)(lrel * a.g.B + b) * a.g.Hq + (size_t)h * G) * D;
   if constexpr (CL > 1) {
     merge_outputs<D, G, CL>(ps, ncl, outp, crank, tid);
   } else {
-    merge_quads<D, G, kMergeGroup>(ps, ncl, nullptr, outp, tid);
+    merge_quads<D, G, kOneLevelItems>(ps, ncl, nullptr, outp, tid);
   }
   if (crank == 0 && tid == 0) a.counters[(size_t)srel * kCountersPerStream] = 0u;
 }

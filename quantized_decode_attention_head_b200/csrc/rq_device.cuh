@@ -63,9 +63,11 @@ __device__ __forceinline__ void put_code(uint32_t* words, int rho, int kh, int e
 // ------------------------------------------------------------ tensor cores
 // D = A(16x32 u8, row) * B(32x8 s8 / u8, col) + C, s32 accumulate; every C
 // element is the same value c.  Results are returned as raw 32-bit words.
+// (The MMAs are pure register operations: not volatile, so the compiler may
+// schedule them freely.)
 __device__ __forceinline__ void imma_u8s8(uint32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
                                           uint32_t c) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};\n"
       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
@@ -73,11 +75,50 @@ __device__ __forceinline__ void imma_u8s8(uint32_t (&d)[4], const uint32_t (&a)[
 }
 __device__ __forceinline__ void imma_u8u8(uint32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
                                           uint32_t c) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};\n"
       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c), "r"(c), "r"(c), "r"(c));
+}
+
+// bf16 MMAs of the window path, fp32 accumulate in place:
+// m16n8k16 (A a0..a3, B b0, b1) and m16n8k8 (A a0, a1, B b0).
+__device__ __forceinline__ void mma_bf16_k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_bf16_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+// Four 8x8 b16 matrices from shared memory; lanes 8i .. 8i + 7 address the
+// rows of matrix i.  Plain: thread (g, t) receives row g, columns 2t, 2t + 1;
+// .trans: rows 2t, 2t + 1 of column g.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+// (lo, hi) -> bf16x2 bits, each rounded to nearest even; lo in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -160,11 +201,6 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
   return p;
 }
-// Prefetch of a global range into L2 (no completion to wait for); both the
-// address and the size are multiples of 16 bytes.
-__device__ __forceinline__ void l2_prefetch(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
-}
 
 // bulk_g2s with an L2 cache policy.
 __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
@@ -173,6 +209,36 @@ __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\n" ::"r"(
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Completion count of a device-scope counter, taken by one thread of a CTA
+// after a CTA barrier: the acquire-release add publishes the CTA's earlier
+// global writes (ordered before this thread by the barrier) to the CTA that
+// takes the final count, and gives that CTA the others' writes, which its
+// other threads read after the next barrier.  Returns the old value.
+__device__ __forceinline__ uint32_t count_acq_rel(uint32_t* p) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;\n" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+// L2 prefetch of a global range (no completion to wait for); address and
+// size multiples of 16 bytes.
+__device__ __forceinline__ void l2_prefetch(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// When p: arms bar for `bytes` and starts the bulk copy src -> dst with an L2
+// policy.  Both steps are predicated inside one asm block, so a caller that
+// passes a lane-dependent p does not branch.
+__device__ __forceinline__ void bulk_g2s_hint_if(bool p, void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %0, 0;\n"
+      " @p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n"
+      " @p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%3], [%4], %2, [%1], %5;\n"
+      "}\n" ::"r"((int)p),
+      "r"(smem_u32(bar)), "r"(bytes), "r"(smem_u32(dst)), "l"(src), "l"(policy)
       : "memory");
 }
 

@@ -102,41 +102,27 @@ int max_record(const rq_cache* c, int l0, int nl) {
   return r;
 }
 
-// Tile splits per stream and cluster size of a decode call (auto mode).
-// One wave -- every stream's items fit the resident slots once in clusters
-// of kDecodeCluster: the splits fill the slots and the window items share the
-// stream's last cluster.  Several waves: single-CTA items of about
-// kWaveTilesPerItem tiles (more when the slots allow), so that no CTA holds
-// a slot at a cluster barrier while the others of its cluster still work.
-#ifndef RQ_BALANCED
-#define RQ_BALANCED 0
-#endif
+// Tile splits per stream and cluster size of a decode call (auto mode):
+// single-CTA items (no cluster barrier holds a slot, the cluster scheduler
+// leaves no slot empty), merged in two levels by the last items to finish.
+// One wave when every stream gets at least two tile items besides its window
+// items; several waves of items of about kWaveTilesPerItem tiles otherwise.
+// (Explicit split counts run in clusters of kDecodeCluster.)
 int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win, int* cluster) {
-  *cluster = rq::kDecodeCluster;
+  *cluster = 1;
   if (n_tiles <= 0) return 0;
-  const int smem = rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes), stage_bytes, c->g.G, c->g.D);
-  if (RQ_BALANCED) {
-    // one wave of single-CTA items filling every resident slot
-    const long slots1 = rq::decode_resident_ctas(c->g.D, c->g.G, 1, smem, c->k_norm ? 3 : 2);
-    if (slots1 / streams >= 2 + n_win) {
-      *cluster = 1;
-      long s = slots1 / streams - n_win;
-      if (s > n_tiles) s = n_tiles;
-      if (s > rq::kMaxItems - n_win) s = rq::kMaxItems - n_win;
-      return (int)s;
-    }
-  }
-  const long slots = rq::decode_resident_ctas(c->g.D, c->g.G, rq::kDecodeCluster, smem, c->k_norm ? 3 : 2);
-  const long per = (slots / streams) / rq::kDecodeCluster * rq::kDecodeCluster;
+  const int smem = rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes),
+                                         stage_bytes, c->g.G, c->g.D);
+  const long slots1 = rq::decode_resident_ctas(c->g.D, c->g.G, 1, smem, c->k_norm ? 3 : 2);
   const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;  // keep a CTA's pipeline busy
   long s;
-  if (per >= 2 * rq::kDecodeCluster) {
-    s = per - n_win;
+  if (slots1 / streams >= 2 + n_win) {
+    // one wave: each stream takes an equal share of the resident slots, so
+    // every SM holds the same number of equally sized tile items
+    s = slots1 / streams - n_win;
   } else {
-    *cluster = 1;
-    const long slots1 = rq::decode_resident_ctas(c->g.D, c->g.G, 1, smem, c->k_norm ? 3 : 2);
+    // several waves of items of about kWaveTilesPerItem tiles
     s = (n_tiles + rq::kWaveTilesPerItem - 1) / rq::kWaveTilesPerItem;
-    if (slots1 / streams - n_win > s) s = slots1 / streams - n_win;
   }
   if (s < 1) s = 1;
   if (s > max_by_work) s = max_by_work;

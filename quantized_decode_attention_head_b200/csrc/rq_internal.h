@@ -129,12 +129,15 @@ __host__ __device__ inline int cluster_items(int items, int cluster) {
 // Floats of one partial softmax state (o[G][D], m[G], l[G]), padded to a
 // multiple of four so that every partial starts on a 16-byte boundary.
 __host__ __device__ constexpr int partial_floats(int G, int D) { return (G * D + 2 * G + 3) / 4 * 4; }
-// Single-CTA items (cluster 1) of a stream merge in groups of kMergeGroup:
-// the last item of a group to finish merges the group into one more partial,
-// the last group merger merges the group partials into the output.
+// Single-CTA items (cluster 1) of a stream: up to kOneLevelItems, the last
+// item to finish merges all partials into the output (one round of loads);
+// beyond, they merge in groups of kMergeGroup: the last item of a group to
+// finish merges the group into one more partial, the last group merger
+// merges the group partials into the output.
 constexpr int kMergeGroup = 8;
+constexpr int kOneLevelItems = 16;
 __host__ __device__ inline int merge_groups(int items) {
-  return items > kMergeGroup ? (items + kMergeGroup - 1) / kMergeGroup : 0;
+  return items > kOneLevelItems ? (items + kMergeGroup - 1) / kMergeGroup : 0;
 }
 // partial slots of one stream: one per item plus one per merge group
 __host__ __device__ inline int partial_slots(int items) { return items + merge_groups(items); }
@@ -173,6 +176,8 @@ cudaError_t launch_measure_distortion(const uint16_t* x, int n_heads, int n_toke
                                       const int* bits, int n_bits, double* mse, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int smem_bytes, cudaStream_t s);
 int decode_smem_bytes(int n_items, int stages, int stage_bytes, int G, int D);
+// shared memory the non-ring roles of a decode CTA need (the rings may use it)
+int decode_free_bytes(int G, int D);
 // CTAs of the decode kernel resident on the device at once, in whole clusters
 // of `cluster` CTAs
 int decode_resident_ctas(int D, int G, int cluster, int smem_bytes, int q_terms);
@@ -196,9 +201,9 @@ constexpr int kDecodeConsumerWarps = 4;
 #define RQ_STAGE_BUDGET 6144
 #endif
 constexpr int kDecodeThreads = kDecodeConsumerWarps * 32;
-// per-warp ring depth: about 6 KB of records in flight per warp (at least two)
+// per-warp ring depth: about 6 KB of records in flight per warp (2 to 8)
 inline int decode_stages(int stage_bytes) {
-  int p = RQ_STAGE_BUDGET / stage_bytes;
+  const int p = RQ_STAGE_BUDGET / stage_bytes;
   return p < 2 ? 2 : (p > 8 ? 8 : p);
 }
 constexpr int kDeviceTimeout = 7;  // == RQ_ERR_DEVICE_TIMEOUT

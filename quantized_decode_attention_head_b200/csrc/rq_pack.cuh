@@ -95,16 +95,21 @@ __device__ __forceinline__ uint32_t code_of(float x, float z, float r) {
 // (packed pairs), and rint done by adding 1.5 * 2^23: for 0 <= y < 2^22 the
 // sum rounds to y's nearest integer (ties to even) + 1.5 * 2^23 exactly.
 // x >= z holds for every element of its group (z is the group minimum, or
-// -M), so y >= 0 and only the top clamp applies (it binds only for
-// subnormal or saturated fp16 scales; larger y round wrongly but clamp).
+// -M), so y >= 0; y is clamped to 2^B - 1 before the rounding add (the clamp
+// binds only for subnormal or saturated fp16 scales).  The clamp also keeps
+// the multiply and the rounding add apart: a multiply feeding an add
+// directly may be contracted into one fused multiply-add by the code
+// generator -- on packed pairs even when both carry an explicit rounding
+// modifier -- which would round the exact product once instead of twice and
+// change the codes of products that round to a half-way point.
 // Returns the sums' bit patterns, the code in the low byte.
 constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
 template <int B>
 __device__ __forceinline__ uint2 codes2(float2 x, float2 nz, float2 r) {
-  constexpr uint32_t kTop = 0x4B400000u + (1u << B) - 1u;
+  constexpr float kTop = (float)((1 << B) - 1);
   const float2 y = __fmul2_rn(__fadd2_rn(x, nz), r);
-  const float2 m = __fadd2_rn(y, make_float2(kRound, kRound));
-  return make_uint2(min(__float_as_uint(m.x), kTop), min(__float_as_uint(m.y), kTop));
+  const float2 m = __fadd2_rn(make_float2(fminf(y.x, kTop), fminf(y.y, kTop)), make_float2(kRound, kRound));
+  return make_uint2(__float_as_uint(m.x), __float_as_uint(m.y));
 }
 
 // Four codes (low bytes of the code_of2 results) into the four bytes of one

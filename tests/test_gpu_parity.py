@@ -152,13 +152,11 @@ def test_decode_all_layers_call():
 
 
 def test_many_streams_single_cta_items():
-    """A call with more streams than the device holds clusters for in one
-    wave: the automatic plan runs single-CTA work items (no clusters) in
-    several waves.  Every stream's output against the oracle, for the
+    """Many streams: the automatic plan runs single-CTA work items (no
+    clusters).  Every stream's output against the oracle, for the
     all-layers decode, a fused decode step and an explicit split count (which
-    keeps clusters), before and after a step."""
-    # 80 streams of 40 tiles: more than the 68 that one wave of clusters holds
-    # on a 148-SM device, few enough that the plan takes several splits each
+    runs in clusters), before and after a step."""
+    # 80 streams of 40 tiles: several single-CTA splits each
     wl = _small(n_layers=2, batch=10, context=4 + 32 * 40 + 32 + 11)
     kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
     cache, st, (k, v, f) = _build(wl, kb, vb)
@@ -426,17 +424,17 @@ def test_hybrid_prefill_decode_and_steps(d, k_norm):
 
 
 def test_single_cta_items_merge_in_two_levels():
-    """More than 8 single-CTA items per stream (80 streams of 1100 tiles: the
-    several-waves plan takes 9 tile splits + 1 window item) merge in two
-    levels: groups of 8, then the group partials.  Every stream's output
-    against the cluster-merged decode at the same split count, and sampled
-    streams against the oracle."""
-    wl = _small(n_layers=2, batch=10, n_q_heads=8, n_kv_heads=4, context=4 + 32 + 32 * 1100 + 11)
+    """More than 16 single-CTA items per stream (20 streams of 1100 tiles: the
+    automatic plan takes about 28 tile splits + 1 window item on a 148-SM
+    device) merge in two levels: groups of 8, then the group partials.  Every
+    stream's output against the cluster-merged decode at 9 splits, and
+    sampled streams against the oracle."""
+    wl = _small(n_layers=1, batch=5, n_q_heads=8, n_kv_heads=4, context=4 + 32 + 32 * 1100 + 11)
     kb, vb = _bits_grid(wl.n_layers, wl.n_kv_heads)
     k, v, f = workloads.kv_inputs(wl, "cuda")
     cache = make_cache(wl, kb, vb, wl.context + 4)
     cache.rq_quantize_kv(k, v)
-    sample = [(0, 0, 0), (1, 9, 3), (0, 5, 2)]
+    sample = [(0, 0, 0), (0, 4, 3), (0, 2, 2)]
     st = oracle_streams(wl, kb, vb, to_f32(k[:, :, :]), to_f32(v), sample)
     del k, v
     torch.cuda.empty_cache()
