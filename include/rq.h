@@ -245,7 +245,10 @@ rq_status rq_decode_workspace_init(void* workspace, size_t ws_bytes, cudaStream_
  *   with a fused log-sum-exp combine.
  * q: device bf16 [B][Hq][D] (layer >= 0) or [L][B][Hq][D] (layer = -1).
  * out: device float32, same shape.  softmax_scale <= 0 selects 1/sqrt(D).
- * n_splits: tile splits per stream, 0 = automatic; capped to the tile count.
+ * n_splits: tile splits per stream, 0 = automatic; capped to the tile count
+ *   and raised to ceil(tiles / 128): an item holds at most 128 tiles, since
+ *   each warp's probabilities are kept in 16-bit fixed point relative to its
+ *   running maximum and their rounding grows over longer sequences.
  * Errors: RQ_ERR_INVALID_ARG, RQ_ERR_WORKSPACE, RQ_ERR_CUDA. */
 rq_status rq_decode_attention(rq_cache* cache, int layer, const void* q, float* out,
                               float softmax_scale, int n_splits, void* workspace,
@@ -314,12 +317,14 @@ rq_status rq_selftest_device_timeout(void* workspace, size_t ws_bytes, unsigned 
  *   before the kernel runs, so a pipeline wait that gives up on the device
  *   (the kernel then leaves out untouched) shows only in the array's status
  *   word: read it with rq_decode_noalloc_read_status.
- * n_splits = 0 takes the automatic plan, reduced to the most splits whose
- *   partials fit the array (in the plan's own cluster size) when the plan
- *   needs more.
- * Errors: RQ_ERR_INVALID_ARG; RQ_ERR_WORKSPACE when the split partials of the
- *   call (about (n_splits + 2) * streams * (G*D + 2G) * 4 bytes) exceed the
- *   array -- reduce n_splits or decode fewer layers per call; RQ_ERR_CUDA. */
+ * n_splits = 0 takes the automatic plan.  No plan goes below ceil(tiles /
+ *   128) splits (see rq_decode_attention), so a call is only as small as
+ *   that: about (ceil(tiles / 128) + window items) * streams * (G*D + 2G) * 4
+ *   bytes of partials, which a one-wave plan keeps far below the array and a
+ *   many-stream call (several waves) may exceed.
+ * Errors: RQ_ERR_INVALID_ARG; RQ_ERR_WORKSPACE when the call's split
+ *   partials exceed the array (nothing is launched) -- decode fewer layers
+ *   per call; RQ_ERR_CUDA. */
 rq_status rq_decode_attention_noalloc(rq_cache* cache, int layer, const void* q, float* out,
                                       float softmax_scale, int n_splits, cudaStream_t stream);
 

@@ -578,10 +578,12 @@ __device__ void dump_tile_state(const WarpState<D, G, QT>& st, float* slot, int 
 
 // bf16 sink + recent window on the tensor cores.  The window is split into
 // chunks of 32 tokens, kWinChunksPerItem consecutive chunks per work item.
-// For each chunk the lanes of warp 0 stage its K and V rows in shared memory
-// with one 1-D bulk copy per row (rows padded to 2 D + 16 bytes, so the 8
-// rows of an 8x8 ldmatrix block fall in 8 different bank quads); warp w then
-// takes tokens 8 w .. 8 w + 7 of the chunk for all G heads:
+// For each chunk lane 0 of warp 0 stages its K and V rows in shared memory
+// with a few 1-D bulk copies of contiguous rows (measured faster than one
+// copy per row into padded, bank-conflict-free rows: the TMA engine is shared
+// with the tile streams, and its per-copy cost outweighs the ldmatrix bank
+// conflicts of 256-byte rows); warp w then takes tokens 8 w .. 8 w + 7 of the
+// chunk for all G heads:
 //   scores (heads x 8 tokens) = q (A, bf16 from the caller's rows, heads in
 //     rows 0..G-1) . K^T (B, ldmatrix of the K rows), m16n8k16, fp32;
 //   o^T (channels x heads) += V^T (A, ldmatrix.trans of the V rows) . P (B,
@@ -592,40 +594,48 @@ __device__ void dump_tile_state(const WarpState<D, G, QT>& st, float* slot, int 
 // Each warp keeps its own online-softmax state over its tokens; the warps'
 // states are merged like the tile path's.
 constexpr int kWinChunk = 32;
-__host__ __device__ constexpr int window_row_stride(int D) { return 2 * D + 16; }
+__host__ __device__ constexpr int window_row_stride(int D) { return 2 * D; }
 // shared memory of a window item: two buffers of one K and one V chunk
 __host__ __device__ constexpr int window_smem_bytes(int D) { return 2 * 2 * kWinChunk * window_row_stride(D); }
 
 __host__ __device__ inline int window_tokens(int T, int S, int Tq) { return (T < S ? T : S) + (T - (T < S ? T : S) - Tq); }
 
-// Lanes of one warp: the K and V rows of window tokens j0 .. j0 + cnt - 1
-// into kbuf / vbuf (row t at t * window_row_stride(D)), counted on bar.
+// Lane 0 of a warp: the K and V rows of window tokens j0 .. j0 + cnt - 1
+// into kbuf / vbuf (row t at t * window_row_stride(D)), counted on bar, with
+// one bulk copy per contiguous run of rows (at most three: sink, ring, ring
+// after its wrap) and one for the newest token of a fused append.
 template <int D>
 __device__ __forceinline__ void window_issue_chunk(const DecodeArgs& a, const uint8_t* win, uint8_t* kbuf,
                                                    uint8_t* vbuf, uint64_t* bar, int j0, int cnt,
                                                    const uint16_t* knew, const uint16_t* vnew, int lane) {
-  constexpr int RB = 2 * D, RS = window_row_stride(D);
-  if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(cnt * RB * 2));
-  __syncwarp();
-  if (lane < cnt) {
-    const int S = a.g.S, ring = a.g.R + kTile;
-    const int n_sink = a.T < S ? a.T : S;
-    const int j = j0 + lane;
-    const void *ks, *vs;
-    if (knew && lane == cnt - 1) {
-      // appended in the same call: the newest token comes from the caller's rows
-      ks = knew;
-      vs = vnew;
-    } else if (j < n_sink) {
-      ks = win + (size_t)j * RB;
-      vs = win + (size_t)(S + j) * RB;
+  constexpr int RB = 2 * D;
+  if (lane != 0) return;
+  const int S = a.g.S, ring = a.g.R + kTile;
+  const int n_sink = a.T < S ? a.T : S;
+  mbar_arrive_expect_tx(bar, (uint32_t)(cnt * RB * 2));
+  const int n_cache = knew ? cnt - 1 : cnt;
+  if (knew) {
+    bulk_g2s(kbuf + (size_t)n_cache * RB, knew, (uint32_t)RB, bar);
+    bulk_g2s(vbuf + (size_t)n_cache * RB, vnew, (uint32_t)RB, bar);
+  }
+  int t = 0;
+  while (t < n_cache) {
+    const int j = j0 + t;
+    size_t row, v_off;
+    int run;
+    if (j < n_sink) {
+      row = j;
+      run = min(n_cache - t, n_sink - j);
+      v_off = S;
     } else {
       const int slot = (a.Tq + (j - n_sink)) % ring;
-      ks = win + (size_t)(2 * S + slot) * RB;
-      vs = win + (size_t)(2 * S + ring + slot) * RB;
+      row = (size_t)2 * S + slot;
+      run = min(n_cache - t, ring - slot);
+      v_off = ring;
     }
-    bulk_g2s(kbuf + lane * RS, ks, (uint32_t)RB, bar);
-    bulk_g2s(vbuf + lane * RS, vs, (uint32_t)RB, bar);
+    bulk_g2s(kbuf + (size_t)t * RB, win + row * RB, (uint32_t)(run * RB), bar);
+    bulk_g2s(vbuf + (size_t)t * RB, win + (row + v_off) * RB, (uint32_t)(run * RB), bar);
+    t += run;
   }
 }
 

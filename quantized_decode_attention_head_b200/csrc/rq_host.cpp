@@ -104,30 +104,29 @@ int max_record(const rq_cache* c, int l0, int nl) {
 
 // Tile splits per stream and cluster size of a decode call (auto mode):
 // single-CTA items (no cluster barrier holds a slot, the cluster scheduler
-// leaves no slot empty), merged in two levels by the last items to finish.
-// One wave when every stream gets at least two tile items besides its window
-// items; several waves of items of about kWaveTilesPerItem tiles otherwise.
-// (Explicit split counts run in clusters of kDecodeCluster.)
+// leaves no slot empty), merged by the last items to finish.  One wave when
+// every stream gets at least two tile items of at most kMaxTilesPerItem tiles
+// besides its window items; several waves of items of kMaxTilesPerItem tiles
+// otherwise.  (Explicit split counts run in clusters of kDecodeCluster.)
 int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win, int* cluster) {
   *cluster = 1;
   if (n_tiles <= 0) return 0;
   const int smem = rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes),
                                          stage_bytes, c->g.G, c->g.D);
   const long slots1 = rq::decode_resident_ctas(c->g.D, c->g.G, 1, smem, c->k_norm ? 3 : 2);
-  const int max_by_work = n_tiles / 8 > 0 ? n_tiles / 8 : 1;  // keep a CTA's pipeline busy
+  const int need = rq::min_splits(n_tiles);
+  const int max_by_work = n_tiles / 8 > need ? n_tiles / 8 : need;  // keep a CTA's pipeline busy
   long s;
-  if (slots1 / streams >= 2 + n_win) {
+  const long one_wave = slots1 / streams - n_win;
+  if (one_wave >= 2 && one_wave >= need) {
     // one wave: each stream takes an equal share of the resident slots, so
     // every SM holds the same number of equally sized tile items
-    s = slots1 / streams - n_win;
+    s = one_wave;
   } else {
-    // several waves of items of about kWaveTilesPerItem tiles
-    s = (n_tiles + rq::kWaveTilesPerItem - 1) / rq::kWaveTilesPerItem;
+    s = need;  // several waves
   }
-  if (s < 1) s = 1;
   if (s > max_by_work) s = max_by_work;
   if (s > n_tiles) s = n_tiles;
-  if (s > rq::kMaxItems - n_win) s = rq::kMaxItems - n_win;
   return (int)s;
 }
 
@@ -144,12 +143,9 @@ rq_status cuda_status(cudaError_t e) {
 
 // Decode arguments for layers [l0, l0 + nl) of a cache holding T tokens, with
 // the workspace checked and partitioned; the fused-append pointers are null.
-// a.cluster is set before the workspace check, so a caller whose workspace
-// was too small for the automatic plan can retry with fewer splits and the
-// same cluster size (cluster_override != 0 replaces the plan's choice).
 rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, float* out, float softmax_scale,
                       int n_splits, void* workspace, size_t ws_bytes, rq::DecodeArgs& a, int& smem,
-                      int n_pack = 0, int cluster_override = 0) {
+                      int n_pack = 0) {
   const int Tq = rq::quantized_tokens(T, c->g.S, c->g.R);
   const int n_tiles = Tq / rq::kTile;
   const int streams = nl * c->g.B * c->g.Hkv;
@@ -159,8 +155,8 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   int cluster = rq::kDecodeCluster;  // explicit split counts run in clusters
   int splits =
       n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win + n_pack, &cluster) : n_splits;
-  if (cluster_override != 0) cluster = cluster_override;
   a.cluster = cluster;
+  if (splits < rq::min_splits(n_tiles)) splits = rq::min_splits(n_tiles);  // at most kMaxTilesPerItem per item
   if (splits > n_tiles) splits = n_tiles;
   if (n_tiles > 0 && splits < 1) splits = 1;
   const int items = splits + n_win + n_pack;
@@ -485,24 +481,6 @@ extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const v
   const int64_t all_streams = (int64_t)c->g.L * c->g.B * c->g.Hkv;
   rq_status st = fill_decode(c, l0, nl, c->length[l0], q, out, softmax_scale, n_splits, scratch,
                              rq::kNoAllocScratchBytes, a, smem);
-  if (st == RQ_ERR_WORKSPACE && n_splits == 0) {
-    // the automatic plan needs more partials than the array holds: take the
-    // most splits whose partials fit, in the plan's own cluster size (with
-    // clusters the items are padded to whole clusters)
-    const int cluster = a.cluster;
-    const int64_t streams = (int64_t)nl * c->g.B * c->g.Hkv;
-    const size_t avail = rq::kNoAllocScratchBytes > rq::ws_partial_offset(all_streams)
-                             ? rq::kNoAllocScratchBytes - rq::ws_partial_offset(all_streams)
-                             : 0;
-    const int64_t slots = (int64_t)avail / (streams * (int64_t)rq::partial_floats(c->g.G, c->g.D) * 4);
-    int64_t items = slots;
-    while (items > 0 && rq::partial_slots((int)items) > slots) --items;
-    items = items / cluster * cluster;
-    const int64_t s = items - rq::window_items(c->length[l0], c->g.S, c->g.R);
-    if (s >= 1)
-      st = fill_decode(c, l0, nl, c->length[l0], q, out, softmax_scale, (int)s, scratch, rq::kNoAllocScratchBytes,
-                       a, smem, 0, cluster);
-  }
   if (st == RQ_ERR_WORKSPACE) return RQ_ERR_WORKSPACE;  // more split partials than the fixed array holds
   if (st != RQ_OK) return st;
   // status word and completion counters must start at zero; the array keeps

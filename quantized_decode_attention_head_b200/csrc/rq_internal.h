@@ -120,8 +120,15 @@ constexpr int kDecodeCluster = RQ_DECODE_CLUSTER;
 #endif
 constexpr int kCountersPerStream = 64;
 constexpr int kMaxItems = 496;
-// tiles per work item aimed at when a call runs in several waves
-constexpr int kWaveTilesPerItem = 128;
+// Most tiles per work item (32 per warp).  A warp keeps P in 16-bit fixed
+// point relative to its running maximum; over many tokens that maximum sits
+// far above most scores and the rounding of the small probabilities grows
+// (measured on a 33K-token stream: 256 tiles per warp exceed max-abs 2e-3,
+// 32 stay near a third of it).  Every plan splits a stream into items of at
+// most this many tiles; calls that run in several waves use items of this
+// size.
+constexpr int kMaxTilesPerItem = 128;
+inline int min_splits(int n_tiles) { return (n_tiles + kMaxTilesPerItem - 1) / kMaxTilesPerItem; }
 __host__ __device__ inline int cluster_items(int items, int cluster) {
   return (items + cluster - 1) / cluster * cluster;
 }
@@ -156,8 +163,10 @@ inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int item
   return ws_partial_offset(all_streams) + (size_t)call_streams * partial_slots(items) * (size_t)partial_floats(G, D) * 4;
 }
 // bf16 window tokens of a T-token cache and the number of window work items
-// (kWinChunksPerItem chunks of 32 tokens each; at least one item)
-constexpr int kWinChunksPerItem = 3;
+// (kWinChunksPerItem chunks of 32 tokens each; at least one item).  Two chunks
+// per item: both copies start at once, so an item waits for one round trip
+// (measured on the Llama-3-8B decode: 14.7 us at 2, 15.4 at 3, 17.5 at 4).
+constexpr int kWinChunksPerItem = 2;
 inline int window_items(int T, int S, int R) {
   const int n_tok = T - quantized_tokens(T, S, R);
   const int chunks = (n_tok + kTile - 1) / kTile;

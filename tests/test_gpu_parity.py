@@ -151,6 +151,33 @@ def test_decode_all_layers_call():
         assert_close(got[l, b], e, f"layer {l} b {b}")
 
 
+def test_explicit_split_count_keeps_items_short():
+    """n_splits = 1 on a stream of 1024 tiles: a warp keeps P in 16-bit fixed
+    point relative to its running maximum, and over 256 tiles per warp the
+    rounding of the small probabilities exceeds the tolerance, so every plan
+    holds an item to at most 128 tiles -- the call runs 8 splits and matches
+    the oracle and the explicit 8-split call bit for bit."""
+    wl = workloads.Workload("long_items", n_layers=1, batch=1, n_q_heads=16, n_kv_heads=2, head_dim=128,
+                            context=4 + 32 + 32 * 1024 + 20, n_sink=4, n_recent=32, k_sigma=1.0, allowed=(2,),
+                            avg_bits=2.0, seed=13)
+    kb = np.full((1, 2), 2)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, kb, wl.context)
+    cache.rq_quantize_kv(k, v)
+    q, _, _ = workloads.step_inputs(wl, 1, f, "cuda")
+    qq = q[0, 0].contiguous()
+    one = cache.rq_decode_attention(0, qq, n_splits=1).cpu().numpy()
+    eight = cache.rq_decode_attention(0, qq, n_splits=8).cpu().numpy()
+    assert np.array_equal(one, eight)
+    G = wl.group
+    for h in range(wl.n_kv_heads):
+        s = ca.StreamCache(wl.head_dim, 2, 2, wl.n_sink, wl.n_recent)
+        s.prefill(to_f32(k[0, 0, h]), to_f32(v[0, 0, h]))
+        kh, vh = s.dequantized()
+        e = at.attend(to_f32(q[0, 0, 0, h * G:(h + 1) * G]).astype(np.float64), kh, vh)
+        assert_close(one[0, h * G:(h + 1) * G], e, f"n_splits=1 kv-head {h}")
+
+
 def test_many_streams_single_cta_items():
     """Many streams: the automatic plan runs single-CTA work items (no
     clusters).  Every stream's output against the oracle, for the
@@ -275,12 +302,16 @@ def test_decode_step_without_room_for_the_pack_item():
     q, kn, vn = workloads.step_inputs(wl, steps, f, "cuda")
     knp, vnp, qnp = to_f32(kn), to_f32(vn), to_f32(q).astype(np.float64)
     # layout: [status, counters: 64 u32 per stream][partials: streams x items x (G*D + 2G) floats];
-    # the full size holds splits + 3 window items + 1 pack item, every window here needs one item
+    # the full size holds splits + 3 window items (one per chunk, the most any
+    # length needs) + 1 pack item; the windows here take at most 3 chunks =
+    # 2 items of 2 chunks, so splits + 2 items always decode, and the step
+    # before a flush (window at S + R + 31 tokens, 2 items) has no room for
+    # the pack item
     streams = wl.batch * wl.n_kv_heads
     offset = 256 + streams * 64 * 4
     part = (wl.group * wl.head_dim + 2 * wl.group) * 4
     assert cache.rq_decode_workspace_bytes(splits) == offset + streams * (splits + 3 + 1) * part
-    ws = torch.zeros(offset + streams * (splits + 1) * part, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(offset + streams * (splits + 2) * part, dtype=torch.uint8, device="cuda")
     flushes = 0
     for t in range(steps):
         for (l, b, h), s in st.items():
