@@ -77,6 +77,18 @@ def decode_bytes(wl, rec, T):
     return total
 
 
+def arm_config(wl, nc, splits, world):
+    """The workload description both arms print (same keys and values)."""
+    cpw = 16  # 2-bit codes per 32-bit word (every long-context head is at 2 bits)
+    rec = 2 * (-(-wl.head_dim // cpw) * 128) + 8 * wl.head_dim
+    per_cache = decode_bytes(wl, [[rec] * wl.n_kv_heads] * wl.n_layers, wl.context)
+    return {"workload": WORKLOAD, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
+            "head_dim": wl.head_dim, "context": wl.context, "bits": "K=V=2 on every head (avg 2 over {2,3,4})",
+            "splits": splits or "auto",
+            "l2": f"{nc} caches decoded round-robin ({nc * per_cache / 1e6:.0f} MB > 126 MB L2)",
+            "parallelism": f"replicas x{world}"}
+
+
 def append_bytes(wl, rec, T_old):
     D = wl.head_dim
     s, tq, r = split_lengths(T_old, wl.n_sink, wl.n_recent)
@@ -301,7 +313,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": res["decode_gbs"], "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["decode_s"] * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": res["sample"]},
+        "config": arm_config(wl, args.copies, args.splits, args.gpus),
         "cpu_baseline": cb,
         "e2e": {"value": res["decode_gbs"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -854,11 +866,7 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "u2 codes; q and P in 16-bit fixed point (two int8 MMA terms); f32 scale/zero epilogue and softmax",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
-                   "head_dim": wl.head_dim, "context": wl.context, "bits": "K=V=2 on every head (avg 2 over {2,3,4})",
-                   "splits": args.splits or "auto", "l2": f"{NC} caches decoded round-robin "
-                   f"({NC * decode_bytes(wl, rec, wl.context) / 1e6:.0f} MB > 126 MB L2)",
-                   "parallelism": f"replicas x{world}"},
+        "config": arm_config(wl, NC, args.splits, world),
         "decode_gbs": achieved,
         "decode_us": per_launch * 1e6,
         "quantize_gbs": (qbytes / (sum(qtimes) / len(qtimes)) / 1e9) if qtimes else None,
