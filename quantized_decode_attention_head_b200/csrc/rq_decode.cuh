@@ -101,17 +101,6 @@ __device__ __forceinline__ float2 combine_terms(const uint32_t (&c)[4]) {
   return make_float2((float)((int)c[0] * 256 + (int)c[1]), (float)((int)c[2] * 256 + (int)c[3]));
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 
 // q of the G heads -> per-head 16-bit fixed point (sq = max|q_h| / 32639)

@@ -112,7 +112,7 @@ __device__ __forceinline__ uint2 codes2(float2 x, float2 nz, float2 r) {
   return make_uint2(__float_as_uint(m.x), __float_as_uint(m.y));
 }
 
-// Four codes (low bytes of the code_of2 results) into the four bytes of one
+// Four codes (low bytes of the codes2 results) into the four bytes of one
 // register, byte e = code e.
 __device__ __forceinline__ uint32_t code_bytes(uint2 c01, uint2 c23) {
   return __byte_perm(__byte_perm(c01.x, c01.y, 0x0040), __byte_perm(c23.x, c23.y, 0x0040), 0x5410);
