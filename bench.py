@@ -675,6 +675,21 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     elapsed = start.elapsed_time(end) / 1e3
+    # The same K steps again, five more timed replays: the graph's arguments
+    # (lengths, slots) are those of the capture, so each replay rewrites the
+    # same appended rows and packed tile and performs identical work; their
+    # spread is the run-to-run spread of the timed region.
+    rep_us = []
+    for _ in range(5):
+        torch.cuda._sleep(2_000_000)
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+        rep_us.append(start.elapsed_time(end) * 1e3 / args.steps)
+    rep_us.sort()
+    repeats = {"n": len(rep_us), "median_us_per_step": rep_us[len(rep_us) // 2], "p10_us_per_step": rep_us[0],
+               "p90_us_per_step": rep_us[-1], "note": "five more replays of the timed graph (min and max as p10 / p90)"}
     del graph
     status = QuantizedKVCache.rq_decode_read_status(ws)
     if status != 0:
@@ -844,7 +859,7 @@ def run_gpu(args):
         if not args.no_sweep:
             cpu["workloads"] = oracle_configs()
     clk = clocks.summary()
-    extra = {"eager": eager, "launch_stats": launch_stats}
+    extra = {"eager": eager, "launch_stats": launch_stats, "repeats": repeats}
     if world == 1 and not args.no_sweep:
         try:
             extra["llama3_8b_step_loop"] = step_loop_graph()
