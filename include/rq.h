@@ -321,7 +321,7 @@ rq_status rq_selftest_device_timeout(void* workspace, size_t ws_bytes, unsigned 
  *   128) splits (see rq_decode_attention), so a call is only as small as
  *   that: about (ceil(tiles / 128) + window items) * streams * (G*D + 2G) * 4
  *   bytes of partials, which a one-wave plan keeps far below the array and a
- *   many-stream call (several waves) may exceed.
+ *   call of very many streams (several waves) may exceed.
  * Errors: RQ_ERR_INVALID_ARG; RQ_ERR_WORKSPACE when the call's split
  *   partials exceed the array (nothing is launched) -- decode fewer layers
  *   per call; RQ_ERR_CUDA. */

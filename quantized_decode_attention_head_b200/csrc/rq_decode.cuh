@@ -566,7 +566,7 @@ __device__ void dump_tile_state(const WarpState<D, G, QT>& st, float* slot, int 
 }
 
 // bf16 sink + recent window on the tensor cores.  The window is split into
-// chunks of 32 tokens, kWinChunksPerItem consecutive chunks per work item.
+// chunks of 32 tokens, a.win_chunks consecutive chunks per work item.
 // For each chunk lane 0 of warp 0 stages its K and V rows in shared memory
 // with a few 1-D bulk copies of contiguous rows (measured faster than one
 // copy per row into padded, bank-conflict-free rows: the TMA engine is shared
@@ -665,8 +665,8 @@ __device__ void window_item(const DecodeArgs& a, uint8_t* win, const uint16_t* q
   const int tid = warp * 32 + lane, gid = lane >> 2, tig = lane & 3;
   const int n_tok = window_tokens(a.T, a.g.S, a.Tq);
   const int n_chunks = (n_tok + kWinChunk - 1) / kWinChunk;
-  const int c0 = witem * kWinChunksPerItem;
-  const int c1 = min(c0 + kWinChunksPerItem, n_chunks);
+  const int c0 = witem * a.win_chunks;
+  const int c1 = min(c0 + a.win_chunks, n_chunks);
   constexpr int kBufBytes = 2 * kWinChunk * RS;  // one K and one V chunk
   // chunk c0 + k lands in buffer k % 2 on bar[k % 2]; the copy of the chunk
   // after next starts as soon as every warp has read a buffer
@@ -1025,8 +1025,8 @@ __global__ void __launch_bounds__(kDecodeThreads, QT == 3 ? 3 : RQ_DECODE_MIN_BL
     uint8_t* win = a.buf + hd.win_base + (int64_t)b * a.g.win_bytes;
     if (tid == 0) {
       const int n_tok = window_tokens(a.T, a.g.S, a.Tq);
-      const int j0 = (item - a.n_splits) * kWinChunksPerItem * kWinChunk;
-      const int j1 = min(j0 + kWinChunksPerItem * kWinChunk, n_tok);
+      const int j0 = (item - a.n_splits) * a.win_chunks * kWinChunk;
+      const int j1 = min(j0 + a.win_chunks * kWinChunk, n_tok);
       if (j0 < j1) window_prefetch_l2<D>(a, win, j0, j1);
     }
     griddep_wait();  // the window rows and the query may come from the previous kernel

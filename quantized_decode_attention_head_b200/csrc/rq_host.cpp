@@ -108,8 +108,10 @@ int max_record(const rq_cache* c, int l0, int nl) {
 // every stream gets at least two tile items of at most kMaxTilesPerItem tiles
 // besides its window items; several waves of items of kMaxTilesPerItem tiles
 // otherwise.  (Explicit split counts run in clusters of kDecodeCluster.)
-int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win, int* cluster) {
+int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, int n_win, int* cluster,
+                bool* one_wave_plan = nullptr) {
   *cluster = 1;
+  if (one_wave_plan) *one_wave_plan = false;
   if (n_tiles <= 0) return 0;
   const int smem = rq::decode_smem_bytes(2, rq::decode_stages(stage_bytes),
                                          stage_bytes, c->g.G, c->g.D);
@@ -122,6 +124,7 @@ int auto_splits(const rq_cache* c, int streams, int n_tiles, int stage_bytes, in
     // one wave: each stream takes an equal share of the resident slots, so
     // every SM holds the same number of equally sized tile items
     s = one_wave;
+    if (one_wave_plan) *one_wave_plan = true;
   } else {
     s = need;  // several waves
   }
@@ -151,10 +154,20 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   const int streams = nl * c->g.B * c->g.Hkv;
   if (streams > 65535) return RQ_ERR_UNSUPPORTED;
   const int stage_bytes = max_record(c, l0, nl);
-  const int n_win = rq::window_items(T, c->g.S, c->g.R);
+  // window items of two chunks, unless the automatic plan runs in several
+  // waves (then one item takes the whole window)
+  int win_chunks = rq::kWinChunksOneWave;
+  int n_win = rq::window_items(T, c->g.S, c->g.R, win_chunks);
   int cluster = rq::kDecodeCluster;  // explicit split counts run in clusters
-  int splits =
-      n_splits == 0 ? auto_splits(c, streams, n_tiles, stage_bytes, n_win + n_pack, &cluster) : n_splits;
+  int splits = n_splits;
+  if (n_splits == 0) {
+    bool one_wave = false;
+    splits = auto_splits(c, streams, n_tiles, stage_bytes, n_win + n_pack, &cluster, &one_wave);
+    if (!one_wave && n_tiles > 0) {
+      win_chunks = rq::kWinChunksWaves;
+      n_win = rq::window_items(T, c->g.S, c->g.R, win_chunks);
+    }
+  }
   a.cluster = cluster;
   if (splits < rq::min_splits(n_tiles)) splits = rq::min_splits(n_tiles);  // at most kMaxTilesPerItem per item
   if (splits > n_tiles) splits = n_tiles;
@@ -177,6 +190,7 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
   a.n_tiles = n_tiles;
   a.n_splits = splits;
   a.n_win = n_win;
+  a.win_chunks = win_chunks;
   a.n_pack = n_pack;
   a.pack_pos = 0;
   a.pack_tile = 0;

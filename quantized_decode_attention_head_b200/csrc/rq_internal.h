@@ -92,6 +92,7 @@ struct DecodeArgs {
   int n_streams;          // streams of this call
   int cluster;            // CTAs per thread-block cluster: kDecodeCluster or 1
   int q_terms;            // s8 terms of the fixed-point query: 2 (16 bits) or 3 (24 bits, K-normalized caches)
+  int win_chunks;         // 32-token window chunks per window item
   int stages;             // per-warp ring depth (2..8)
   int stage_bytes;        // bytes per stage (max record size in the call)
   float* partials;        // [streams][n_splits+1][G*D + 2G]
@@ -163,14 +164,18 @@ inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int item
   return ws_partial_offset(all_streams) + (size_t)call_streams * partial_slots(items) * (size_t)partial_floats(G, D) * 4;
 }
 // bf16 window tokens of a T-token cache and the number of window work items
-// (kWinChunksPerItem chunks of 32 tokens each; at least one item).  Two chunks
-// per item: both copies start at once, so an item waits for one round trip
-// (measured on the Llama-3-8B decode: 14.7 us at 2, 15.4 at 3, 17.5 at 4).
-constexpr int kWinChunksPerItem = 2;
-inline int window_items(int T, int S, int R) {
+// of `per` chunks of 32 tokens each (at least one item).  A one-wave plan
+// takes two chunks per item: both copies start at once, so an item waits for
+// one round trip and the window items stay off the critical path (measured
+// on the Llama-3-8B decode: 14.7 us at 2, 15.4 at 3, 17.5 at 4).  A plan of
+// several waves takes the whole window in one item: its CTAs compete for
+// slots, and fewer, longer window items cost less slot time.
+constexpr int kWinChunksOneWave = 2;
+constexpr int kWinChunksWaves = 8;
+inline int window_items(int T, int S, int R, int per) {
   const int n_tok = T - quantized_tokens(T, S, R);
   const int chunks = (n_tok + kTile - 1) / kTile;
-  const int n = (chunks + kWinChunksPerItem - 1) / kWinChunksPerItem;
+  const int n = (chunks + per - 1) / per;
   return n > 0 ? n : 1;
 }
 
