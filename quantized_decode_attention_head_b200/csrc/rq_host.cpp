@@ -166,6 +166,12 @@ rq_status fill_decode(const rq_cache* c, int l0, int nl, int T, const void* q, f
     if (!one_wave && n_tiles > 0) {
       win_chunks = rq::kWinChunksWaves;
       n_win = rq::window_items(T, c->g.S, c->g.R, win_chunks);
+    } else if (one_wave && splits > 0 && n_tiles / splits >= rq::kWholeWindowTiles) {
+      // long tile items: one window item of the whole window finishes well
+      // before them, and the slots it frees go to tile items
+      win_chunks = rq::kWinChunksWaves;
+      n_win = rq::window_items(T, c->g.S, c->g.R, win_chunks);
+      splits = auto_splits(c, streams, n_tiles, stage_bytes, n_win + n_pack, &cluster, &one_wave);
     }
   }
   a.cluster = cluster;

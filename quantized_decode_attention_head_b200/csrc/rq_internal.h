@@ -169,9 +169,13 @@ inline size_t ws_total_bytes(int64_t all_streams, int64_t call_streams, int item
 // one round trip and the window items stay off the critical path (measured
 // on the Llama-3-8B decode: 14.7 us at 2, 15.4 at 3, 17.5 at 4).  A plan of
 // several waves takes the whole window in one item: its CTAs compete for
-// slots, and fewer, longer window items cost less slot time.
+// slots, and fewer, longer window items cost less slot time; so does a
+// one-wave plan whose tile items are long enough to hide it.
 constexpr int kWinChunksOneWave = 2;
 constexpr int kWinChunksWaves = 8;
+// A one-wave plan whose tile items hold at least this many tiles (10 per
+// warp) also takes the whole window in one item.
+constexpr int kWholeWindowTiles = 40;
 inline int window_items(int T, int S, int R, int per) {
   const int n_tok = T - quantized_tokens(T, S, R);
   const int chunks = (n_tok + kTile - 1) / kTile;
