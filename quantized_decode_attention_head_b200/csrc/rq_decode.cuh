@@ -4,16 +4,19 @@
 #pragma once
 //
 //
-// One CTA = one work item of one (layer, batch, kv-head) stream: either a
-// contiguous range of packed tiles (items 0..n_splits-1) or the bf16 sink +
-// recent window (items n_splits..).  Four warps process tiles; lane 0 of each
-// streams the warp's own tile records into a private ring of shared-memory
-// stages with 1-D bulk copies (cp.async.bulk, TMA engine) completing on
-// mbarriers.  Consecutive items of a stream form thread-block clusters; the
-// first CTA of each cluster merges its cluster's partial softmax states
-// (log-sum-exp) from distributed shared memory, and the CTAs of the stream's
-// last cluster to finish merge the cluster partials and write the output --
-// no second launch.
+// One CTA = one work item of one (layer, batch, kv-head) stream: a
+// contiguous range of at most 128 packed tiles (items 0..n_splits-1), chunks
+// of the bf16 sink + recent window (the next items, on the bf16 tensor
+// cores), or, in a fused step before a tile flush, the pack-ahead of that
+// tile.  Four warps process tiles; lane 0 of each streams the warp's own tile
+// records into a private ring of shared-memory stages with 1-D bulk copies
+// (cp.async.bulk, TMA engine) completing on mbarriers.  Each CTA merges its
+// warps' partial softmax states (log-sum-exp) and publishes one partial; the
+// last item of a stream to finish (or, past 16 items, of each group of 8,
+// then of the groups) merges the partials and writes the output -- no second
+// launch.  With an explicit split count, consecutive items form
+// thread-block clusters whose first CTA merges the cluster through
+// distributed shared memory.
 //
 // Per tile (32 tokens), with the G query heads that share the kv head:
 //   q.K^T  : integer tensor-core MMA (mma.sync m16n8k32, u8 x s8 -> s32).

@@ -102,15 +102,15 @@ struct DecodeArgs {
   const uint16_t* v_new;
 };
 
-// Split-K combine.  The work items of a stream (tile splits, then window
-// chunks) form thread-block clusters of `cluster` consecutive items (the grid
-// is padded with empty items to whole clusters); a cluster merges its items
-// through distributed shared memory, and the CTAs of the last cluster of the
-// stream to finish merge the cluster partials, each a slice of the outputs.
-// Per stream counter [0] counts finished clusters.  Calls whose items fill
-// the device once run in clusters of kDecodeCluster; calls that need several
-// waves of CTAs run single-CTA items (cluster 1), so that no CTA holds a slot
-// at a cluster barrier while the others of its cluster still work.
+// Split-K combine.  The automatic plan runs single-CTA items (cluster 1):
+// each publishes its partial, and the last to finish merges them (two levels
+// past kOneLevelItems items).  An explicit split count runs the items of a
+// stream (tile splits, then window chunks) in thread-block clusters of
+// `cluster` consecutive items (the grid padded with empty items to whole
+// clusters); a cluster merges its items through distributed shared memory,
+// and the CTAs of the last cluster of the stream to finish merge the cluster
+// partials, each a slice of the outputs.  Per stream counter [0] counts
+// finished items, groups or clusters.
 #ifndef RQ_DECODE_CLUSTER
 #define RQ_DECODE_CLUSTER 4
 #endif
