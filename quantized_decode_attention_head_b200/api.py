@@ -160,12 +160,16 @@ class QuantizedKVCache:
         check("rq_cache_init", lib().rq_cache_init(ctypes.byref(cfg), _dptr(self.buffer), self.nbytes,
                                                    ctypes.byref(handle), _stream_ptr(None, self.buffer.get_device())))
         self.handle = handle
+        # kept for the destructor, which may run while the interpreter is
+        # tearing module globals down
+        self._destroy = lib().rq_cache_destroy
         del keep
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h is not None and h.value:
-            lib().rq_cache_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self.handle = None
 
     # -- queries -----------------------------------------------------------
