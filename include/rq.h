@@ -29,6 +29,9 @@
  *     launch, a CUDA launch error is reported as RQ_ERR_CUDA.
  *   - bf16 tensors are passed as raw 16-bit patterns (const void*), row-major
  *     and contiguous; out is float32.
+ *   - k, v, q, k_new, v_new, out and workspace start on a 16-byte boundary
+ *     (the kernels move them in 16-byte vectors and bulk copies); a pointer
+ *     that does not is rejected with RQ_ERR_INVALID_ARG before any launch.
  *   - Lengths are tracked on the host in the rq_cache handle, so no call reads
  *     device memory back (except the rq_*_read_status calls, which say so).
  *   - Device memory handed to the library is used on the stream given with

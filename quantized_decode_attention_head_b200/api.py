@@ -28,12 +28,12 @@ def _dptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _check_tensor(name, t, dtype, shape=None, device_type="cuda"):
+def _check_tensor(name, t, dtype, shape=None, device_type="cuda", align=16):
     import torch
 
     # one cheap test on the common path; the detailed message only on failure
     if (isinstance(t, torch.Tensor) and t.dtype is dtype and t.is_cuda == (device_type == "cuda")
-            and t.is_contiguous() and (shape is None or t.shape == tuple(shape))):
+            and t.is_contiguous() and (shape is None or t.shape == tuple(shape)) and t.data_ptr() % align == 0):
         return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -43,7 +43,9 @@ def _check_tensor(name, t, dtype, shape=None, device_type="cuda"):
         raise ValueError(f"{name} must be on {device_type}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if shape is not None and t.shape != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    raise ValueError(f"{name} must start on a {align}-byte boundary (a view at an offset into a larger tensor?)")
 
 
 def rq_allocate_bits(w, alpha, beta, avg_bits, allowed):
@@ -82,7 +84,7 @@ def rq_measure_distortion(x, role, bits, stream=None):
 
     if x.dim() != 3:
         raise ValueError("x must be [n_heads, n_tokens, head_dim]")
-    _check_tensor("x", x, torch.bfloat16)
+    _check_tensor("x", x, torch.bfloat16, align=2)
     h, t, d = x.shape
     bits = np.ascontiguousarray(bits, dtype=np.int32)
     mse = torch.empty((h, bits.size), dtype=torch.float64, device=x.device)

@@ -30,6 +30,8 @@ struct rq_cache {
 namespace {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+// Device arguments the kernels move in 16-byte vectors or bulk copies.
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
 
@@ -320,6 +322,7 @@ rq_status rq_cache_stream_layout(const rq_cache* c, int layer, int b, int kv_hea
 
 rq_status rq_quantize_kv(rq_cache* c, const void* k, const void* v, int n_tokens, cudaStream_t stream) {
   if (!c || n_tokens < 0 || (n_tokens > 0 && (!k || !v))) return RQ_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (!aligned16(k) || !aligned16(v))) return RQ_ERR_INVALID_ARG;
   if (n_tokens > c->max_tokens) return RQ_ERR_CAPACITY;
   rq::QuantizeArgs a;
   a.g = c->g;
@@ -342,7 +345,7 @@ rq_status rq_quantize_kv(rq_cache* c, const void* k, const void* v, int n_tokens
 }
 
 rq_status rq_append_token(rq_cache* c, int layer, const void* k_new, const void* v_new, cudaStream_t stream) {
-  if (!c || !k_new || !v_new) return RQ_ERR_INVALID_ARG;
+  if (!c || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return RQ_ERR_INVALID_ARG;
   int l0, nl;
   if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
   const int T_old = c->length[l0];
@@ -386,13 +389,14 @@ rq_status rq_decode_workspace_bytes(const rq_cache* c, int n_splits, size_t* byt
 }
 
 rq_status rq_decode_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream) {
-  if (!workspace || ws_bytes < rq::ws_counter_offset()) return RQ_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || ws_bytes < rq::ws_counter_offset()) return RQ_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(workspace, 0, ws_bytes, stream));
 }
 
 rq_status rq_selftest_device_timeout(void* workspace, size_t ws_bytes, unsigned long long limit_ns,
                                      cudaStream_t stream) {
-  if (!workspace || ws_bytes < rq::ws_counter_offset() || limit_ns > 1000000000ull) return RQ_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || ws_bytes < rq::ws_counter_offset() || limit_ns > 1000000000ull)
+    return RQ_ERR_INVALID_ARG;
   return cuda_status(rq::launch_wait_timeout_selftest(static_cast<int*>(workspace), limit_ns, stream));
 }
 
@@ -404,6 +408,7 @@ rq_status rq_decode_read_status(const void* workspace, int* device_status) {
 rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out, float softmax_scale, int n_splits,
                               void* workspace, size_t ws_bytes, cudaStream_t stream) {
   if (!c || !q || !out || !workspace || n_splits < 0) return RQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return RQ_ERR_INVALID_ARG;
   int l0, nl;
   if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
   rq::DecodeArgs a;
@@ -416,6 +421,8 @@ rq_status rq_decode_attention(rq_cache* c, int layer, const void* q, float* out,
 rq_status rq_decode_step(rq_cache* c, int layer, const void* q, const void* k_new, const void* v_new, float* out,
                          float softmax_scale, int n_splits, void* workspace, size_t ws_bytes, cudaStream_t stream) {
   if (!c || !q || !k_new || !v_new || !out || !workspace || n_splits < 0) return RQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out) || !aligned16(workspace))
+    return RQ_ERR_INVALID_ARG;
   int l0, nl;
   if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
   const int T_old = c->length[l0];
@@ -478,6 +485,7 @@ extern "C" rq_status rq_measure_distortion(const void* x, int n_heads, int n_tok
                                            const int* bits, int n_bits, double* mse, cudaStream_t stream) {
   if (!x || !bits || !mse || n_heads < 1 || n_tokens < 1 || n_bits < 1 || (role != 0 && role != 1))
     return RQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 1u) || (reinterpret_cast<uintptr_t>(mse) & 7u)) return RQ_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return RQ_ERR_UNSUPPORTED;
   if (role == 1 && n_tokens % rq::kTile != 0) return RQ_ERR_INVALID_ARG;
   if (n_heads > 65535) return RQ_ERR_UNSUPPORTED;
@@ -491,7 +499,7 @@ extern "C" rq_status rq_measure_distortion(const void* x, int n_heads, int n_tok
 // library's own device scratch array; allocates nothing.
 extern "C" rq_status rq_decode_attention_noalloc(rq_cache* c, int layer, const void* q, float* out,
                                                   float softmax_scale, int n_splits, cudaStream_t stream) {
-  if (!c || !q || !out || n_splits < 0) return RQ_ERR_INVALID_ARG;
+  if (!c || !q || !out || n_splits < 0 || !aligned16(q) || !aligned16(out)) return RQ_ERR_INVALID_ARG;
   int l0, nl;
   if (!layer_range(c, layer, l0, nl)) return RQ_ERR_INVALID_ARG;
   void* scratch = nullptr;

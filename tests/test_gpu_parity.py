@@ -399,6 +399,82 @@ def test_workspace_too_small_is_rejected():
     assert e.value.status == "RQ_ERR_WORKSPACE"
 
 
+def test_misaligned_device_pointers_are_rejected_before_launch():
+    """The kernels move k, v, q, k_new, v_new, out and the workspace in
+    16-byte vectors and bulk copies, so each must start on a 16-byte
+    boundary.  A view a few bytes into a larger tensor is refused by the
+    binding (ValueError) and, passed straight to the C ABI, by the host
+    checks (RQ_ERR_INVALID_ARG = 1) before anything is launched: the cache
+    keeps its length, and the aligned calls that follow match the oracle."""
+    import ctypes
+
+    from quantized_decode_attention_head_b200 import _lib
+
+    P = ctypes.c_void_p
+    wl = workloads.CONFIGS["tiny"]
+    (kb, vb), (okb, ovb) = workload_bits(wl)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, wl.context + 4)
+
+    def shifted(t):  # the same values, starting one element past a 16-byte boundary
+        buf = torch.empty(t.numel() + 16, dtype=t.dtype, device=t.device)
+        view = buf[1:1 + t.numel()].view(t.shape)
+        view.copy_(t)
+        assert view.data_ptr() % 16 != 0
+        return view
+
+    L = _lib.lib()
+    ks = shifted(k)
+    with pytest.raises(ValueError):
+        cache.rq_quantize_kv(ks, v)
+    assert L.rq_quantize_kv(cache.handle, P(ks.data_ptr()), P(v.data_ptr()), k.shape[3], None) == 1
+    assert L.rq_quantize_kv(cache.handle, P(k.data_ptr()), P(shifted(v).data_ptr()), k.shape[3], None) == 1
+    assert cache.length(0) == 0
+    cache.rq_quantize_kv(k, v)
+    T = cache.length(0)
+
+    q, kn, vn = workloads.step_inputs(wl, 1, f, "cuda")
+    q0, kn0, vn0 = q[0, 0].contiguous(), kn[0, 0].contiguous(), vn[0, 0].contiguous()
+    qs, kns, vns = shifted(q0), shifted(kn0), shifted(vn0)
+    ws = cache.make_workspace()
+    out = torch.empty(q0.shape, dtype=torch.float32, device="cuda")
+    outs = shifted(out)
+    wsb = torch.zeros(ws.numel() + 16, dtype=torch.uint8, device="cuda")[8:8 + ws.numel()]
+    n = ws.numel()
+    for call in (lambda: cache.rq_append_token(0, kns, vn0),
+                 lambda: cache.rq_decode_attention(0, qs, workspace=ws),
+                 lambda: cache.rq_decode_attention(0, q0, out=outs, workspace=ws),
+                 lambda: cache.rq_decode_step(0, q0, kn0, vns, workspace=ws)):
+        with pytest.raises(ValueError):
+            call()
+    f0 = ctypes.c_float(0.0)
+    assert L.rq_append_token(cache.handle, 0, P(kns.data_ptr()), P(vn0.data_ptr()), None) == 1
+    assert L.rq_append_token(cache.handle, 0, P(kn0.data_ptr()), P(vns.data_ptr()), None) == 1
+    assert L.rq_decode_attention(cache.handle, 0, P(qs.data_ptr()), P(out.data_ptr()), f0, 0, P(ws.data_ptr()), n,
+                                 None) == 1
+    assert L.rq_decode_attention(cache.handle, 0, P(q0.data_ptr()), P(outs.data_ptr()), f0, 0, P(ws.data_ptr()), n,
+                                 None) == 1
+    assert L.rq_decode_attention(cache.handle, 0, P(q0.data_ptr()), P(out.data_ptr()), f0, 0, P(wsb.data_ptr()), n,
+                                 None) == 1
+    for a, b_, c in ((qs, kn0, vn0), (q0, kns, vn0), (q0, kn0, vns)):
+        assert L.rq_decode_step(cache.handle, 0, P(a.data_ptr()), P(b_.data_ptr()), P(c.data_ptr()),
+                                P(out.data_ptr()), f0, 0, P(ws.data_ptr()), n, None) == 1
+    assert L.rq_decode_attention_noalloc(cache.handle, 0, P(qs.data_ptr()), P(out.data_ptr()), f0, 0, None) == 1
+    assert L.rq_decode_attention_noalloc(cache.handle, 0, P(q0.data_ptr()), P(outs.data_ptr()), f0, 0, None) == 1
+    assert L.rq_decode_workspace_init(P(wsb.data_ptr()), n, None) == 1
+    torch.cuda.synchronize()
+    assert cache.length(0) == T
+
+    st = oracle_streams(wl, okb, ovb, to_f32(k), to_f32(v), all_streams(wl))
+    cache.rq_decode_step(0, q0, kn0, vn0, out=out, workspace=ws)
+    for (l, b, h), s in st.items():
+        s.append(to_f32(kn[0, l, b, h]), to_f32(vn[0, l, b, h]))
+    exp = oracle_decode(wl, st, to_f32(q[0]).astype(np.float64), [(0, 0)])[(0, 0)]
+    assert_close(out.cpu().numpy()[0], exp, "aligned step after the rejected calls")
+    assert cache.length(0) == T + 1
+    assert QuantizedKVCache.rq_decode_read_status(ws) == 0
+
+
 def test_tiny_workload_end_to_end():
     wl = workloads.CONFIGS["tiny"]
     (kb, vb), (okb, ovb) = workload_bits(wl)

@@ -188,3 +188,17 @@ def test_timeout_selftest_rejects_bad_arguments_before_cuda():
     assert L.rq_selftest_device_timeout(None, 4096, 1000, None) == 1
     assert L.rq_selftest_device_timeout(ctypes.c_void_p(256), 16, 1000, None) == 1
     assert L.rq_selftest_device_timeout(ctypes.c_void_p(256), 4096, 2_000_000_000, None) == 1
+
+
+def test_misaligned_device_pointers_are_rejected_before_cuda():
+    """A device pointer the kernels move in 16-byte vectors (the workspace,
+    k, v, q, out) is refused on the host when it does not start on a 16-byte
+    boundary, before any CUDA call; so are calibration samples off a 2-byte
+    boundary and an fp64 result array off an 8-byte one."""
+    L = _lib.lib()
+    P = ctypes.c_void_p
+    assert L.rq_decode_workspace_init(P(0x1008), 4096, None) == 1
+    assert L.rq_selftest_device_timeout(P(0x1004), 4096, 1000, None) == 1
+    bits = (ctypes.c_int * 1)(2)
+    assert L.rq_measure_distortion(P(0x1001), 1, 32, 128, 0, bits, 1, P(0x2000), None) == 1
+    assert L.rq_measure_distortion(P(0x1000), 1, 32, 128, 0, bits, 1, P(0x2004), None) == 1
