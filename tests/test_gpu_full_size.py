@@ -80,7 +80,8 @@ def test_full_size_sampled_streams(name):
 
 def test_long_context_named_split_counts():
     """long_128k at 64, 128 and 256 splits per head (then the combine), every
-    one of its 8 streams against the oracle, plus a fused step at 256 splits."""
+    one of its 8 streams against the oracle; the automatic plan repeated five
+    times (bit-identical, within tolerance); a fused step at 256 splits."""
     wl = workloads.CONFIGS["long_128k"]
     (kb, vb), (okb, ovb) = workload_bits(wl)
     k, v, f = workloads.kv_inputs(wl, "cuda")
@@ -104,6 +105,14 @@ def test_long_context_named_split_counts():
         out = cache.rq_decode_attention(0, q[0, 0].contiguous(), n_splits=splits, workspace=ws).cpu().numpy()
         for h in streams:
             assert_close(out[0, h * G:(h + 1) * G], exp[h], f"splits {splits} kv-head {h}")
+    # The automatic plan (one wave of single-CTA items, merged in two levels
+    # by the last items to finish): the merge order is fixed by item index,
+    # so repeated calls agree bit for bit whatever order the items finish in.
+    auto = [cache.rq_decode_attention(0, q[0, 0].contiguous(), workspace=ws).cpu().numpy() for _ in range(5)]
+    for o in auto[1:]:
+        assert np.array_equal(o, auto[0])
+    for h in streams:
+        assert_close(auto[0][0, h * G:(h + 1) * G], exp[h], f"automatic plan kv-head {h}")
     out = cache.rq_decode_step(0, q[1, 0].contiguous(), kn[1, 0].contiguous(), vn[1, 0].contiguous(),
                                n_splits=max(wl.splits), workspace=ws).cpu().numpy()
     for h, s in streams.items():
