@@ -475,6 +475,39 @@ def test_misaligned_device_pointers_are_rejected_before_launch():
     assert QuantizedKVCache.rq_decode_read_status(ws) == 0
 
 
+@pytest.mark.parametrize("scale", [0.03, 0.5])
+def test_softmax_scale_argument(scale):
+    """An explicit softmax scale (flatter, and four times sharper than
+    1/sqrt(D) = 0.125 at head_dim 64) against the oracle's attention with the
+    same scale, every stream of the small cache, through the plain and the
+    fused-step calls."""
+    wl = workloads.CONFIGS["tiny"]
+    (kb, vb), (okb, ovb) = workload_bits(wl)
+    k, v, f = workloads.kv_inputs(wl, "cuda")
+    cache = make_cache(wl, kb, vb, wl.context + 2)
+    cache.rq_quantize_kv(k, v)
+    st = oracle_streams(wl, okb, ovb, to_f32(k), to_f32(v), all_streams(wl))
+    q, kn, vn = workloads.step_inputs(wl, 2, f, "cuda")
+    G = wl.group
+
+    def check(out, qf, what):
+        for (l, b, h), s in st.items():
+            if l != 0:
+                continue
+            kh, vh = s.dequantized()
+            e = at.attend(qf[0, b, h * G:(h + 1) * G].astype(np.float64), kh, vh, scale)
+            assert_close(out[b, h * G:(h + 1) * G], e, f"{what} scale {scale} (b {b}, h {h})")
+
+    out = cache.rq_decode_attention(0, q[0, 0].contiguous(), softmax_scale=scale).cpu().numpy()
+    check(out, to_f32(q[0]), "decode")
+    out = cache.rq_decode_step(0, q[1, 0].contiguous(), kn[1, 0].contiguous(), vn[1, 0].contiguous(),
+                               softmax_scale=scale).cpu().numpy()
+    for (l, b, h), s in st.items():
+        if l == 0:
+            s.append(to_f32(kn[1, 0, b, h]), to_f32(vn[1, 0, b, h]))
+    check(out, to_f32(q[1]), "fused step")
+
+
 def test_tiny_workload_end_to_end():
     wl = workloads.CONFIGS["tiny"]
     (kb, vb), (okb, ovb) = workload_bits(wl)
